@@ -1,0 +1,306 @@
+/*
+ * BATQuant online path — plain CPU oracle (TEST INFRASTRUCTURE ONLY).
+ *
+ * Only the tests, the package smoke check and the benchmark's CPU-baseline leg
+ * may load this library. The product path never does: it shares no code,
+ * header, table or helper with the CUDA kernels.
+ *
+ * Everything is written the slow, obvious way, in double precision unless a
+ * step is defined in fp32:
+ *
+ *   - the block transform builds the explicit 32x32 block P_b = B_b (x) A
+ *     (Kronecker product) and multiplies the row vector x by it, following the
+ *     "Global and Private Kronecker decomposition" (BATQuant note,
+ *     en.papernotes.org, Method > Key Designs 2; nubint.ai review, proposed
+ *     method: P_i = B_i (x) A, A shared, B_i private, block size g = 32);
+ *   - the clip uses per-block ratios sigma(gamma) on the block minimum and
+ *     maximum (Key Designs 3, "Block-wise learnable clipping");
+ *   - MXFP4: E2M1 elements on the grid {0, .5, 1, 1.5, 2, 3, 4, 6} with one
+ *     UE8M0 (power-of-two) scale per 32 elements (Background & Motivation);
+ *     the encoder searches the grid exhaustively for the nearest point;
+ *   - the linear layer is Y = Q(XP) Q(P^-1 W^T) (Key Designs 1), evaluated as
+ *     an fp64 dot product of the dequantized operands;
+ *   - P^-1 comes from a Gauss-Jordan inverse with partial pivoting, in fp64.
+ *
+ * Readings of points the pages leave open (all shared with the CUDA path only
+ * through their written statement, never through code):
+ *   - x's 32 elements are read as a row-major 4x8 matrix X_r[i][p] = x[8i+p];
+ *     then x P_b = vec_row(B_b^T X_r A).
+ *   - lo = fp32(r_lo * min), hi = fp32(r_hi * max), c = min(max(y, lo), hi)
+ *     (hi wins if lo > hi); r = fp32 of the fp64 logistic function.
+ *   - scale exponent e = floor(log2(amax)) - 2, clamped to [-127, 127]; amax = 0
+ *     gives e = -127; scale byte = e + 127.
+ *   - a clipped value that is exactly zero encodes as +0 (code 0x0); any other
+ *     value keeps its sign bit, so a negative value that rounds to zero is 0x8.
+ *   - ties on the grid go to the even code (mantissa bit 0); |v| > 6 gives 6.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_G 32
+
+static const double kGrid[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+static double bf16_bits_to_double(uint16_t h) {
+  uint32_t u = (uint32_t)h << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* Explicit Kronecker product: P[(8i+p)][(8j+q)] = B[i][j] * A[p][q]. */
+void orc_kron(const double* B /*4x4*/, const double* A /*8x8*/, double* P /*32x32*/) {
+  for (int i = 0; i < 4; ++i)
+    for (int j = 0; j < 4; ++j)
+      for (int p = 0; p < 8; ++p)
+        for (int q = 0; q < 8; ++q)
+          P[(8 * i + p) * 32 + (8 * j + q)] = B[i * 4 + j] * A[p * 8 + q];
+}
+
+/* y = x . P_b for every row and block, fp64 result (not rounded). */
+void orc_transform_f64(const uint16_t* X, int64_t M, int64_t K, const float* A, const float* B,
+                       double* Y) {
+  const int64_t nb = K / ORC_G;
+  double Ad[64];
+  for (int t = 0; t < 64; ++t) Ad[t] = A[t];
+  double* P = (double*)malloc(sizeof(double) * 1024 * (size_t)nb);
+  for (int64_t b = 0; b < nb; ++b) {
+    double Bd[16];
+    for (int t = 0; t < 16; ++t) Bd[t] = B[b * 16 + t];
+    orc_kron(Bd, Ad, P + 1024 * b);
+  }
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t b = 0; b < nb; ++b) {
+      const double* Pb = P + 1024 * b;
+      double x[32];
+      for (int k = 0; k < 32; ++k) x[k] = bf16_bits_to_double(X[m * K + b * 32 + k]);
+      for (int j = 0; j < 32; ++j) {
+        double s = 0.0;
+        for (int k = 0; k < 32; ++k) s += x[k] * Pb[k * 32 + j];
+        Y[m * K + b * 32 + j] = s;
+      }
+    }
+  }
+  free(P);
+}
+
+/* The "transformed values": the fp64 product rounded once to fp32. */
+void orc_transform(const uint16_t* X, int64_t M, int64_t K, const float* A, const float* B,
+                   float* Y) {
+  double* Yd = (double*)malloc(sizeof(double) * (size_t)(M * K));
+  orc_transform_f64(X, M, K, A, B, Yd);
+  for (int64_t t = 0; t < M * K; ++t) Y[t] = (float)Yd[t];
+  free(Yd);
+}
+
+/* Clip ratio sigma(gamma) = 1 / (1 + exp(-gamma)), in fp64, rounded once to fp32. */
+float orc_clip_ratio(float gamma) {
+  if (isinf(gamma) && gamma > 0) return 1.0f;
+  return (float)(1.0 / (1.0 + exp(-(double)gamma)));
+}
+
+void orc_clip_ratios(const float* gamma, int64_t n, float* r) {
+  for (int64_t t = 0; t < n; ++t) r[t] = gamma ? orc_clip_ratio(gamma[t]) : 1.0f;
+}
+
+/* E2M1 encoder: nearest grid magnitude by exhaustive search, ties to the even
+ * code, saturating at 6. Returns 0xFF for NaN input. */
+uint8_t orc_e2m1_encode(float v) {
+  if (isnan(v)) return 0xFF;
+  double a = fabs((double)v);
+  int best = 0;
+  double best_d = fabs(a - kGrid[0]);
+  for (int c = 1; c < 8; ++c) {
+    double d = fabs(a - kGrid[c]);
+    if (d < best_d || (d == best_d && (c % 2 == 0) && (best % 2 != 0))) {
+      best = c;
+      best_d = d;
+    }
+  }
+  if (a > 6.0) best = 7;
+  return (uint8_t)(best | (signbit(v) ? 8 : 0));
+}
+
+void orc_e2m1_encode_array(const float* v, int64_t n, uint8_t* codes) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < n; ++t) codes[t] = orc_e2m1_encode(v[t]);
+}
+
+double orc_e2m1_value(uint8_t code) {
+  double m = kGrid[code & 7];
+  return (code & 8) ? -m : m;
+}
+
+/* Quantize one 32-element block of transformed values. Returns 0, or 1 if the
+ * block holds a non-finite value (outside the contract; scale byte 0xFF). */
+int orc_quantize_block(const float* y, float r_lo, float r_hi, uint8_t* codes, uint8_t* scale,
+                       float* clipped /* nullable, 32 */) {
+  float mn = y[0], mx = y[0];
+  for (int k = 0; k < 32; ++k) {
+    if (!isfinite(y[k])) {
+      *scale = 0xFF;
+      for (int t = 0; t < 32; ++t) codes[t] = 0;
+      return 1;
+    }
+    if (y[k] < mn) mn = y[k];
+    if (y[k] > mx) mx = y[k];
+  }
+  const float lo = r_lo * mn; /* one fp32 multiply */
+  const float hi = r_hi * mx;
+  float c[32];
+  float amax = 0.0f;
+  for (int k = 0; k < 32; ++k) {
+    float v = y[k];
+    if (v < lo) v = lo;
+    if (v > hi) v = hi;
+    if (v == 0.0f) v = 0.0f; /* exact zero of either sign becomes +0 */
+    c[k] = v;
+    if (fabsf(v) > amax) amax = fabsf(v);
+  }
+  int e;
+  if (amax == 0.0f) {
+    e = -127;
+  } else {
+    int ex;
+    frexpf(amax, &ex); /* amax = m * 2^ex, m in [0.5, 1): floor(log2 amax) = ex - 1 */
+    e = (ex - 1) - 2;
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+  }
+  *scale = (uint8_t)(e + 127);
+  for (int k = 0; k < 32; ++k) {
+    float v = ldexpf(c[k], -e);
+    codes[k] = orc_e2m1_encode(v);
+    if (clipped) clipped[k] = c[k];
+  }
+  return 0;
+}
+
+/* Quantize a [rows][K] matrix of transformed values, one ratio pair per block
+ * (shared by all rows: r_lo[nb], r_hi[nb]) or one per row and block
+ * (per_row != 0: r_lo[rows][nb]). Codes come out one per byte [rows][K]
+ * (unpacked); scales plain row-major [rows][nb]. Returns the number of
+ * non-finite blocks. */
+int64_t orc_quantize_matrix(const float* Y, int64_t rows, int64_t K, const float* r_lo,
+                            const float* r_hi, int per_row, uint8_t* codes, uint8_t* scales) {
+  const int64_t nb = K / ORC_G;
+  int64_t bad = 0;
+#pragma omp parallel for schedule(static) reduction(+ : bad)
+  for (int64_t m = 0; m < rows; ++m) {
+    for (int64_t b = 0; b < nb; ++b) {
+      const int64_t ri = per_row ? m * nb + b : b;
+      const float rl = r_lo ? r_lo[ri] : 1.0f;
+      const float rh = r_hi ? r_hi[ri] : 1.0f;
+      bad += orc_quantize_block(Y + m * K + b * 32, rl, rh, codes + m * K + b * 32,
+                                scales + m * nb + b, NULL);
+    }
+  }
+  return bad;
+}
+
+/* Dequantize: value = grid(code) * 2^(scale - 127). */
+void orc_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t K,
+                    double* out) {
+  const int64_t nb = K / ORC_G;
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < rows; ++m)
+    for (int64_t k = 0; k < K; ++k) {
+      const uint8_t s = scales[m * nb + k / 32];
+      const double sc = (s == 0xFF) ? NAN : ldexp(1.0, (int)s - 127);
+      out[m * K + k] = orc_e2m1_value(codes[m * K + k]) * sc;
+    }
+}
+
+/* Y[i][j] = sum_k Xd[rows[i]][k] * Wd[cols[j]][k] in fp64, serial sum per output
+ * (so the result does not depend on the thread count). */
+void orc_gemm_sampled(const double* Xd, const double* Wd, int64_t K, const int64_t* rows,
+                      int64_t nrows, const int64_t* cols, int64_t ncols, double* Y) {
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t i = 0; i < nrows; ++i) {
+    const double* x = Xd + rows[i] * K;
+    for (int64_t j = 0; j < ncols; ++j) {
+      const double* w = Wd + cols[j] * K;
+      double s = 0.0;
+      for (int64_t k = 0; k < K; ++k) s += x[k] * w[k];
+      Y[i * ncols + j] = s;
+    }
+  }
+}
+
+/* Gauss-Jordan inverse with partial pivoting, fp64. Returns 0 on success, 1 if
+ * a pivot is zero (singular). */
+int orc_inverse(int n, const double* Min, double* Mout) {
+  double* a = (double*)malloc(sizeof(double) * (size_t)(n * 2 * n));
+  for (int r = 0; r < n; ++r)
+    for (int c = 0; c < 2 * n; ++c)
+      a[r * 2 * n + c] = c < n ? Min[r * n + c] : (c - n == r ? 1.0 : 0.0);
+  for (int col = 0; col < n; ++col) {
+    int piv = col;
+    for (int r = col + 1; r < n; ++r)
+      if (fabs(a[r * 2 * n + col]) > fabs(a[piv * 2 * n + col])) piv = r;
+    if (a[piv * 2 * n + col] == 0.0) {
+      free(a);
+      return 1;
+    }
+    if (piv != col)
+      for (int c = 0; c < 2 * n; ++c) {
+        double t = a[col * 2 * n + c];
+        a[col * 2 * n + c] = a[piv * 2 * n + c];
+        a[piv * 2 * n + c] = t;
+      }
+    const double d = a[col * 2 * n + col];
+    for (int c = 0; c < 2 * n; ++c) a[col * 2 * n + c] /= d;
+    for (int r = 0; r < n; ++r) {
+      if (r == col) continue;
+      const double f = a[r * 2 * n + col];
+      if (f == 0.0) continue;
+      for (int c = 0; c < 2 * n; ++c) a[r * 2 * n + c] -= f * a[col * 2 * n + c];
+    }
+  }
+  for (int r = 0; r < n; ++r)
+    for (int c = 0; c < n; ++c) Mout[r * n + c] = a[r * 2 * n + n + c];
+  free(a);
+  return 0;
+}
+
+/* Weight side: row n, block b of W becomes w_b . (B_b^-T (x) A^-T), i.e. the
+ * rows of (P^-1 W^T)^T = W P^-T. fp64 result, not rounded. Returns 0, or 1 if
+ * A or some B_b is singular. */
+int orc_weight_transform_f64(const uint16_t* W, int64_t N, int64_t K, const float* A,
+                             const float* B, double* Wt) {
+  const int64_t nb = K / ORC_G;
+  double Ad[64], Ainv[64], AinvT[64];
+  for (int t = 0; t < 64; ++t) Ad[t] = A[t];
+  if (orc_inverse(8, Ad, Ainv)) return 1;
+  for (int p = 0; p < 8; ++p)
+    for (int q = 0; q < 8; ++q) AinvT[p * 8 + q] = Ainv[q * 8 + p];
+  double* P = (double*)malloc(sizeof(double) * 1024 * (size_t)nb);
+  for (int64_t b = 0; b < nb; ++b) {
+    double Bd[16], Binv[16], BinvT[16];
+    for (int t = 0; t < 16; ++t) Bd[t] = B[b * 16 + t];
+    if (orc_inverse(4, Bd, Binv)) {
+      free(P);
+      return 1;
+    }
+    for (int i = 0; i < 4; ++i)
+      for (int j = 0; j < 4; ++j) BinvT[i * 4 + j] = Binv[j * 4 + i];
+    orc_kron(BinvT, AinvT, P + 1024 * b);
+  }
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t b = 0; b < nb; ++b) {
+      const double* Pb = P + 1024 * b;
+      double w[32];
+      for (int k = 0; k < 32; ++k) w[k] = bf16_bits_to_double(W[n * K + b * 32 + k]);
+      for (int j = 0; j < 32; ++j) {
+        double s = 0.0;
+        for (int k = 0; k < 32; ++k) s += w[k] * Pb[k * 32 + j];
+        Wt[n * K + b * 32 + j] = s;
+      }
+    }
+  free(P);
+  return 0;
+}

@@ -1,0 +1,355 @@
+"""Pins for the CPU oracle: each check ties it to something other than itself.
+
+Sources are the pages (BATQuant note on en.papernotes.org, the nubint.ai review,
+the BRQ article on 10100.com), closed forms, library routines (numpy/scipy),
+brute force and exact rational arithmetic. Every test here runs on the CPU.
+"""
+from __future__ import annotations
+
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.linalg
+import scipy.special
+
+import oracle
+from oracle import formats
+import workloads as wl
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _read_pairs(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            a, b = line.split()
+            rows.append((a, b))
+    return rows
+
+
+def _bf16_to_f64(h):
+    return wl.bf16_bits_to_f32(h).astype(np.float64)
+
+
+# --- MXFP4 element grid and encoder -------------------------------------------------
+
+def test_grid_matches_pages():
+    """Code -> value table equals the grid the note prints (Background & Motivation)."""
+    table = {int(a): float(b) for a, b in _read_pairs("e2m1_grid.txt")}
+    codes = np.arange(16, dtype=np.uint8)
+    vals = oracle.e2m1_value(codes)
+    for c in range(8):
+        assert vals[c] == table[c]
+        assert vals[c + 8] == -table[c]
+
+
+def test_e2m1_ties_fixture():
+    for v, code in _read_pairs("e2m1_ties.txt"):
+        assert oracle.e2m1_encode(np.array([np.float32(v)]))[0] == int(code), v
+
+
+def _e2m1_by_binade(v: np.ndarray) -> np.ndarray:
+    """E2M1 as a 1-mantissa-bit float: round-half-even on each binade's step.
+
+    Below 2 the step is 0.5 (subnormal code range and the [1, 2) binade),
+    on [2, 4) it is 1, on [4, 8) it is 2; anything above 6 saturates. This is
+    textbook IEEE-style rounding with numpy's rint (ties to even), a different
+    formulation from the oracle's nearest-point search.
+    """
+    a = np.abs(v.astype(np.float64))
+    q = np.where(a < 2.0, np.rint(a * 2.0) / 2.0,
+                 np.where(a < 4.0, np.rint(a), 2.0 * np.rint(a / 2.0)))
+    q = np.minimum(q, 6.0)
+    lut = {0.0: 0, 0.5: 1, 1.0: 2, 1.5: 3, 2.0: 4, 3.0: 5, 4.0: 6, 6.0: 7}
+    keys = np.array(sorted(lut))
+    code = np.searchsorted(keys, q).astype(np.uint8)
+    assert np.all(keys[code] == q)
+    return code | (np.signbit(v).astype(np.uint8) << 3)
+
+
+def test_e2m1_bruteforce_all_fp32_up_to_8():
+    """Every fp32 bit pattern in [0, 8] (about 1.09e9 values), plus sampled negatives."""
+    top = np.float32(8.0).view(np.uint32)
+    step = 1 << 26
+    for start in range(0, int(top) + 1, step):
+        bits = np.arange(start, min(start + step, int(top) + 1), dtype=np.uint32)
+        v = bits.view(np.float32)
+        got = oracle.e2m1_encode(v)
+        want = _e2m1_by_binade(v)
+        bad = np.nonzero(got != want)[0]
+        assert bad.size == 0, (v[bad[:5]], got[bad[:5]], want[bad[:5]])
+    rng = np.random.default_rng(1)
+    bits = rng.integers(0, int(top) + 1, size=2_000_000, dtype=np.uint32) | np.uint32(0x80000000)
+    v = bits.view(np.float32)
+    assert np.array_equal(oracle.e2m1_encode(v), _e2m1_by_binade(v))
+
+
+# --- GPK structure ----------------------------------------------------------------
+
+def test_param_counts_printed():
+    g = dict(_read_pairs("gpk_param_counts.txt"))
+    counts = oracle.gpk_param_counts(int(g["hidden"]))
+    assert counts["gpk"] == int(g["gpk"])
+    assert counts["naive_kronecker"] == int(g["naive_kronecker"])
+    assert counts["full_blocks"] == int(g["full_blocks"])
+    # the review's ">74%-79%" reduction claim
+    assert 100 * (1 - counts["gpk"] / int(g["flatquant"])) > int(g["reduction_vs_flatquant_min_pct"])
+    assert 100 * (1 - counts["gpk"] / counts["naive_kronecker"]) > int(g["reduction_vs_naive_min_pct"])
+
+
+def test_kron_block_equals_numpy_kron():
+    A, B, _, _ = wl.random_factors(3, seed=5)
+    for b in range(3):
+        P = oracle.kron_block(B[b], A)
+        assert np.array_equal(P, np.kron(B[b].astype(np.float64), A.astype(np.float64)))
+
+
+def test_transform_equals_block_diagonal_matmul():
+    """x P with P = blockdiag(B_b (x) A) built by scipy, and the factored form."""
+    inp = wl.make_inputs("tiny")
+    nb = inp.B.shape[0]
+    P = scipy.linalg.block_diag(*[np.kron(inp.B[b].astype(np.float64), inp.A.astype(np.float64))
+                                  for b in range(nb)])
+    X = _bf16_to_f64(inp.X)
+    Y = oracle.transform_f64(inp.X, inp.A, inp.B)
+    ref = X @ P
+    assert np.max(np.abs(Y - ref)) <= 1e-14 * np.max(np.abs(ref))
+    # factored form vec_row(B_b^T X_r A), X_r[i][p] = x[8i+p]
+    A64 = inp.A.astype(np.float64)
+    for b in range(nb):
+        Xr = X[:, 32 * b:32 * b + 32].reshape(-1, 4, 8)
+        fac = (inp.B[b].astype(np.float64).T[None] @ Xr @ A64[None]).reshape(-1, 32)
+        blk = Y[:, 32 * b:32 * b + 32]
+        assert np.max(np.abs(blk - fac)) <= 1e-14 * np.max(np.abs(fac))
+    # the fp32 transformed values are that product rounded once
+    assert np.array_equal(oracle.transform(inp.X, inp.A, inp.B), Y.astype(np.float32))
+
+
+def test_block_locality():
+    """Changing block b of x changes only block b's transform, codes and scale."""
+    inp = wl.make_inputs("tiny")
+    X = inp.X.copy()
+    Y0, c0, s0 = oracle.quantize_act(X, inp.A, inp.B, inp.g_lo, inp.g_hi)
+    b = 3
+    X[:, 32 * b:32 * b + 32] = wl.random_bf16((X.shape[0], 32), seed=9, scale=20.0)
+    Y1, c1, s1 = oracle.quantize_act(X, inp.A, inp.B, inp.g_lo, inp.g_hi)
+    other = np.ones(X.shape[1], bool)
+    other[32 * b:32 * b + 32] = False
+    assert np.array_equal(Y0[:, other], Y1[:, other])
+    assert np.array_equal(c0[:, other], c1[:, other])
+    keep = np.arange(s0.shape[1]) != b
+    assert np.array_equal(s0[:, keep], s1[:, keep])
+    assert not np.array_equal(Y0[:, ~other], Y1[:, ~other])
+
+
+# --- inverse and weight-side fusion -------------------------------------------------
+
+def test_inverse_roundtrip_and_library():
+    rng = np.random.default_rng(3)
+    for n in (4, 8):
+        for _ in range(20):
+            M = np.eye(n) + 0.3 * rng.standard_normal((n, n))
+            inv = oracle.inverse(M)
+            assert np.max(np.abs(inv @ M - np.eye(n))) < 1e-12
+            assert np.allclose(inv, np.linalg.inv(M), rtol=1e-12, atol=1e-12)
+    with pytest.raises(np.linalg.LinAlgError):
+        oracle.inverse(np.zeros((4, 4)))
+
+
+def test_inverse_fusion_preserves_output():
+    """(X P)(P^-1 W^T) = X W^T before quantization (Key Designs 1)."""
+    inp = wl.make_inputs("tiny")
+    XP = oracle.transform_f64(inp.X, inp.A, inp.B)
+    WPt = oracle.weight_transform_f64(inp.W, inp.A, inp.B)
+    ref = _bf16_to_f64(inp.X) @ _bf16_to_f64(inp.W).T
+    got = XP @ WPt.T
+    assert np.linalg.norm(got - ref) <= 1e-10 * np.linalg.norm(ref)
+
+
+def test_hadamard_special_case():
+    """A = H8/sqrt8, B_b = H4/2 gives P_b = H32/sqrt32 (Sylvester), the block rotation of BRQ."""
+    H8 = scipy.linalg.hadamard(8) / np.sqrt(8.0)
+    H4 = scipy.linalg.hadamard(4) / 2.0
+    H32 = scipy.linalg.hadamard(32) / np.sqrt(32.0)
+    A = H8.astype(np.float32)
+    nb = 8
+    B = np.repeat(H4[None].astype(np.float32), nb, axis=0)
+    assert np.allclose(oracle.kron_block(B[0], A), H32, atol=1e-7)
+    X = wl.random_bf16((16, 32 * nb), seed=11)
+    Y = oracle.transform_f64(X, A, B)
+    Xd = _bf16_to_f64(X)
+    n_in = np.linalg.norm(Xd.reshape(16, nb, 32), axis=2)
+    n_out = np.linalg.norm(Y.reshape(16, nb, 32), axis=2)
+    assert np.allclose(n_in, n_out, rtol=1e-6)
+    # orthonormal and symmetric, so P^-T = P: the weight side equals the activation side
+    assert np.allclose(oracle.weight_transform_f64(X, A, B), Y, rtol=1e-6, atol=1e-6)
+
+
+# --- quantizer ----------------------------------------------------------------------
+
+def _rtn_mxfp4(x: np.ndarray):
+    """Plain MXFP4 round-to-nearest of a matrix, written independently of the oracle."""
+    rows, K = x.shape
+    blocks = x.reshape(rows, K // 32, 32).astype(np.float32)
+    amax = np.max(np.abs(blocks), axis=2)
+    with np.errstate(divide="ignore"):
+        e = np.where(amax > 0, np.floor(np.log2(amax.astype(np.float64))) - 2, -127)
+    e = np.clip(e, -127, 127).astype(np.int32)
+    v = blocks.astype(np.float64) / np.exp2(e.astype(np.float64))[..., None]
+    v = np.where(v == 0, 0.0, v)  # exact zeros become +0
+    codes = _e2m1_by_binade(v.astype(np.float32)).reshape(rows, K)
+    return codes, (e + 127).astype(np.uint8)
+
+
+def test_rtn_special_case():
+    """Identity factors with no clip reduce to plain MXFP4 RTN (the RTN row of Table 2)."""
+    inp = wl.make_inputs("tiny")
+    nb = inp.B.shape[0]
+    A = np.eye(8, dtype=np.float32)
+    B = np.repeat(np.eye(4, dtype=np.float32)[None], nb, axis=0)
+    Y, codes, scales = oracle.quantize_act(inp.X, A, B, None, None)
+    x = wl.bf16_bits_to_f32(inp.X)
+    assert np.array_equal(Y, x)
+    rc, rs = _rtn_mxfp4(x)
+    assert np.array_equal(scales, rs)
+    assert np.array_equal(codes, rc)
+    # gamma = +inf is the same as "no clip" (ratio exactly 1)
+    inf = np.full(nb, np.inf, np.float32)
+    _, c2, s2 = oracle.quantize_act(inp.X, A, B, inf, inf)
+    assert np.array_equal(c2, codes) and np.array_equal(s2, scales)
+
+
+@pytest.mark.parametrize("name", ["tiny"])
+def test_grid_and_scale_rule(name):
+    inp = wl.make_inputs(name)
+    Y, codes, scales = oracle.quantize_act(inp.X, inp.A, inp.B, inp.g_lo, inp.g_hi)
+    deq = oracle.dequantize(codes, scales)
+    rows, K = codes.shape
+    e = scales.astype(np.int64) - 127
+    assert np.all(scales < 255)
+    mant = deq.reshape(rows, K // 32, 32) / np.exp2(e)[..., None]
+    assert np.all(np.isin(np.abs(mant), oracle.GRID))
+    # the block maximum lands on 4 or 6: amax * 2^-e in [4, 8) for every non-zero block
+    nz = np.any(codes.reshape(rows, K // 32, 32) & 7, axis=2)
+    top = np.max(np.abs(mant), axis=2)
+    assert np.all(np.isin(top[nz], [4.0, 6.0]))
+    r_lo = oracle.clip_ratios(inp.g_lo)
+    r_hi = oracle.clip_ratios(inp.g_hi)
+    blk = Y.reshape(rows, K // 32, 32)
+    lo = (r_lo[None] * blk.min(axis=2)).astype(np.float32)
+    hi = (r_hi[None] * blk.max(axis=2)).astype(np.float32)
+    c = np.minimum(np.maximum(blk, lo[..., None]), hi[..., None])
+    amax = np.max(np.abs(c), axis=2).astype(np.float64)
+    ratio = amax[nz] / np.exp2(e[nz])
+    assert np.all((ratio >= 4.0) & (ratio < 8.0))
+
+
+def test_clip_properties():
+    rng = np.random.default_rng(7)
+    Y = (rng.standard_normal((50, 64)) * rng.uniform(0.1, 50, size=(50, 1))).astype(np.float32)
+    Y[0, :32] = np.abs(Y[0, :32]) + 1.0          # all-positive block: lower bound inert
+    Y[1, 32:] = -np.abs(Y[1, 32:]) - 1.0         # all-negative block: upper bound inert
+    r_lo = np.array([0.7, 0.9], np.float32)
+    r_hi = np.array([0.8, 0.6], np.float32)
+    codes, scales, bad = oracle.quantize(Y, r_lo, r_hi)
+    assert bad == 0
+    # no clip when both ratios are 1
+    c1, s1, _ = oracle.quantize(Y, np.ones(2, np.float32), np.ones(2, np.float32))
+    c0, s0, _ = oracle.quantize(Y, None, None)
+    assert np.array_equal(c1, c0) and np.array_equal(s1, s0)
+    blk = Y.reshape(50, 2, 32)
+    lo = (r_lo[None] * blk.min(axis=2)).astype(np.float32)
+    hi = (r_hi[None] * blk.max(axis=2)).astype(np.float32)
+    clipped = np.clip(blk, lo[..., None], hi[..., None])
+    amax = np.abs(clipped).max(axis=2)
+    assert np.all(amax <= np.maximum(np.abs(lo), np.abs(hi)))
+    # the quantized block equals RTN of the numpy-clipped values (hi wins if lo > hi)
+    rc, rs = _rtn_mxfp4(np.minimum(np.maximum(blk, lo[..., None]), hi[..., None]).reshape(50, 64))
+    assert np.array_equal(codes, rc) and np.array_equal(scales, rs)
+    # bounds are inert on one-signed blocks
+    assert lo[0, 0] <= blk[0, 0].min() and hi[1, 1] >= blk[1, 1].max()
+
+
+def test_sigmoid_ratios():
+    g = np.array([0.0, 1.0, 2.5, 4.0, -3.0, 30.0], np.float32)
+    r = oracle.clip_ratios(g)
+    assert r[0] == np.float32(0.5)
+    assert np.array_equal(r, scipy.special.expit(g.astype(np.float64)).astype(np.float32))
+    assert oracle.clip_ratios(np.array([np.inf], np.float32))[0] == 1.0
+    assert np.all(oracle.clip_ratios(None, 4) == 1.0)
+
+
+def test_zero_and_degenerate_blocks():
+    Y = np.zeros((2, 64), np.float32)
+    Y[1, :] = -0.0
+    Y[1, 40] = 3.0
+    codes, scales, _ = oracle.quantize(Y, None, None)
+    assert np.all(scales[0] == 0) and np.all(codes[0] == 0)   # amax = 0: e = -127, byte 0
+    assert scales[1, 0] == 0 and np.all(codes[1, :32] == 0)   # -0 encodes as +0
+    # 3.0: floor(log2 3) - 2 = -1, byte 126, 3 * 2 = 6 -> code 7
+    assert scales[1, 1] == 126 and codes[1, 40] == 7
+    # non-finite input is flagged
+    Y2 = np.zeros((1, 32), np.float32)
+    Y2[0, 5] = np.inf
+    _, s2, bad = oracle.quantize(Y2, None, None)
+    assert bad == 1 and s2[0, 0] == 0xFF
+
+
+# --- GEMM ---------------------------------------------------------------------------
+
+def test_dequantize_closed_form():
+    codes = np.array([[7, 15, 1, 9] * 8], np.uint8)
+    scales = np.array([[127 + 3]], np.uint8)
+    d = oracle.dequantize(codes, scales)
+    assert np.array_equal(d[0, :4], np.array([6.0, -6.0, 0.5, -0.5]) * 8.0)
+
+
+def test_gemm_exact_rational():
+    """fp64 dot products of dequantized MXFP4 operands against exact Fractions."""
+    inp = wl.make_inputs("tiny")
+    _, xc, xs = oracle.quantize_act(inp.X, inp.A, inp.B, inp.g_lo, inp.g_hi)
+    _, wc, ws = oracle.prepare_weight(inp.W, inp.A, inp.B)
+    Xd = oracle.dequantize(xc, xs)
+    Wd = oracle.dequantize(wc, ws)
+    rows = [0, 17, 63]
+    cols = [0, 5, 64, 127]
+    Y = oracle.gemm_sampled(Xd, Wd, rows, cols)
+    K = Xd.shape[1]
+    for i, m in enumerate(rows):
+        for j, n in enumerate(cols):
+            exact = Fraction(0)
+            mag = Fraction(0)
+            for k in range(K):
+                t = Fraction(Xd[m, k]) * Fraction(Wd[n, k])
+                exact += t
+                mag += abs(t)
+            assert abs(Fraction(Y[i, j]) - exact) <= mag * Fraction(1, 2 ** 50)
+    # the full product is the matrix product (library routine)
+    full = oracle.gemm_sampled(Xd, Wd)
+    assert np.allclose(full, Xd @ Wd.T, rtol=1e-12, atol=1e-12)
+
+
+# --- storage formats ----------------------------------------------------------------
+
+def test_formats_roundtrip():
+    rng = np.random.default_rng(0)
+    codes = rng.integers(0, 16, size=(5, 64), dtype=np.uint8)
+    assert np.array_equal(formats.unpack_codes(formats.pack_codes(codes)), codes)
+    assert formats.pack_codes(np.array([[1, 2]], np.uint8))[0, 0] == 0x21
+    for rows, nb in [(1, 1), (130, 9), (256, 128)]:
+        plain = rng.integers(0, 255, size=(rows, nb), dtype=np.uint8)
+        tiled = formats.tile_scales(plain)
+        assert tiled.size == formats.scale_bytes(rows, nb)
+        assert np.array_equal(formats.untile_scales(tiled, rows, nb), plain)
+        idx = formats.scale_index(rows, nb).reshape(-1)
+        assert np.unique(idx).size == idx.size
+    I = formats.scale_index(256, 12)
+    nbp4 = 3
+    assert I[0, 0] == 0 and I[1, 0] == 16 and I[32, 0] == 4 and I[0, 1] == 1
+    assert I[0, 4] == 512 and I[128, 0] == nbp4 * 512 and I[31, 3] == 31 * 16 + 3
