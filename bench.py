@@ -1,0 +1,366 @@
+"""Benchmark of the BATQuant W4A4 linear layer on B200: Y = Q(XP) . Q(P^-1 W^T).
+
+One step = the whole online path over one batch: the fused prologue (GPK block
+transform + block clip + MXFP4 quantize/pack of X) and the block-scaled MXFP4
+GEMM against weights prepared offline. Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of the
+same layer (replicated weights, independent token batches, no collective on the
+data path) -> weak scaling; time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as wl  # noqa: E402
+
+METRIC = "W4A4 BAT linear TFLOP/s (% FP4 peak); act-quant prologue GB/s (% HBM)"
+PROLOGUE_BYTES_PER_ELT = 2.0 + 0.5 + 1.0 / 32.0  # bf16 in, 4-bit code out, 1/32 scale byte
+FP4_OVER_BF16 = 9.0 / 2.25  # nominal dense FP4 / BF16 tensor throughput on B200
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ---------------------------------------------------------------- clocks during the timed region
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="bat_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for n, v in zip(names, r[3][1:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows), "power_w_max": max(r[2] for r in rows)}
+
+
+# ---------------------------------------------------------------- CPU oracle leg
+def oracle_sample(inp, w, budget_s: float, seed: int = 0):
+    """Time the oracle (as it stands) on a bounded sample of the layer.
+
+    The sample is `rows` token rows against `cols` weight rows: the oracle's
+    transform + clip + quantize of those rows, their dequantization, and the fp64
+    dot products. Weight preparation is offline on both sides and not timed.
+    Returns (flop/s, seconds, description, threads).
+    """
+    import oracle
+    rng = np.random.default_rng(seed)
+    _, wc, ws = oracle.prepare_weight(inp.W, inp.A, inp.B)
+    Wd = oracle.dequantize(wc, ws)
+
+    def run(rows, cols):
+        t0 = time.perf_counter()
+        X = inp.X[rows]
+        _, xc, xs = oracle.quantize_act(X, inp.A, inp.B, inp.g_lo, inp.g_hi)
+        Xd = oracle.dequantize(xc, xs)
+        oracle.gemm_sampled(Xd, Wd, None, cols)
+        return time.perf_counter() - t0
+
+    cols = np.arange(w.N)
+    t1 = run(rng.integers(0, w.M, size=1), cols)
+    nrows = int(max(1, min(w.M, budget_s / max(t1, 1e-6))))
+    ncols = w.N
+    if t1 > budget_s:  # a single full row is already over budget: sample columns too
+        nrows = 1
+        ncols = int(max(1, w.N * budget_s / t1))
+    rows = rng.choice(w.M, size=nrows, replace=False)
+    cols = np.sort(rng.choice(w.N, size=ncols, replace=False))
+    dt = run(rows, cols)
+    flops = 2.0 * nrows * ncols * w.K
+    desc = (f"{nrows} random token rows x {ncols} weight rows of {w.name} "
+            f"(K={w.K}): transform+clip+quantize, dequantize, fp64 dot products")
+    return flops / dt, dt, desc, oracle.num_threads()
+
+
+def run_reference(args, w, inp):
+    """The oracle timed as the reference arm, on the same config and metric."""
+    steps, warm = args.steps, args.warmup
+    per_step = max(0.05, min(2.0, args.ref_budget_s / max(1, steps + warm)))
+    import oracle
+    _, wc, ws = oracle.prepare_weight(inp.W, inp.A, inp.B)
+    Wd = oracle.dequantize(wc, ws)
+    rng = np.random.default_rng(1)
+
+    def step(ncols):
+        rows = rng.integers(0, w.M, size=1)
+        cols = np.sort(rng.choice(w.N, size=ncols, replace=False))
+        t0 = time.perf_counter()
+        _, xc, xs = oracle.quantize_act(inp.X[rows], inp.A, inp.B, inp.g_lo, inp.g_hi)
+        oracle.gemm_sampled(oracle.dequantize(xc, xs), Wd, None, cols)
+        return time.perf_counter() - t0
+
+    t_full = step(w.N)
+    ncols = int(max(1, min(w.N, w.N * per_step / max(t_full, 1e-6))))
+    for _ in range(warm):
+        step(ncols)
+    total = 0.0
+    for _ in range(steps):
+        total += step(ncols)
+    flops = 2.0 * ncols * w.K * steps
+    value = flops / total / 1e12
+    desc = f"per step: 1 random token row x {ncols} weight rows of {w.name} (K={w.K})"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": steps, "warmup": warm,
+        "ms_per_step": 1e3 * total / steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU leg
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="mlp_gate_up", choices=wl.ORDER)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--ref-budget-s", type=float, default=90.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank, world, local = dist_env()
+    w = wl.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, w, wl.make_inputs(w.name, seed=0))
+        return
+
+    import torch
+    import w4a4_bit_gemm_b200 as bat
+
+    bat.lib()  # fail loudly if the CUDA library is missing
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    # rank r draws its own token batch; weights and transform factors are shared
+    inp = wl.make_inputs(w.name, seed=0)
+    X_host = inp.X if rank == 0 else wl.make_inputs(w.name, seed=rank, with_weight=False).X
+
+    def bf16(bits):
+        return torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(dev)
+
+    def f32(a):
+        return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev)
+
+    X = bf16(X_host)
+    A, B = f32(inp.A), f32(inp.B)
+    gl, gh = f32(inp.g_lo), f32(inp.g_hi)
+    Wq = bat.bat_prepare_weight(bf16(inp.W), A, B)
+    Xq = bat.MXFP4.empty(w.M, w.K, dev)
+    Y = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        bat.bat_quantize_act(X, A, B, gl, gh, Xq=Xq, stream=stream)
+        bat.bat_mxfp4_gemm(Xq, Wq, Y=Y, out_dtype=torch.bfloat16, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+
+    K_ = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K_)]
+    sampler = ClockSampler(local)
+    if not args.no_clocks and rank == 0:
+        sampler.start()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    for i in range(K_):
+        flush.fill_(i & 0xFF)  # evict L2 between steps (outside the timed events)
+        ev[i][0].record(stream)
+        bat.bat_quantize_act(X, A, B, gl, gh, Xq=Xq, stream=stream)
+        ev[i][1].record(stream)
+        bat.bat_mxfp4_gemm(Xq, Wq, Y=Y, out_dtype=torch.bfloat16, stream=stream)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    clocks = sampler.stop() if (not args.no_clocks and rank == 0) else None
+    t_pro = [ev[i][0].elapsed_time(ev[i][1]) * 1e-3 for i in range(K_)]
+    t_gemm = [ev[i][1].elapsed_time(ev[i][2]) * 1e-3 for i in range(K_)]
+    t_step = sum(t_pro) + sum(t_gemm)
+    if pg:
+        t = torch.tensor([t_step, sum(t_pro), sum(t_gemm)], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        t_step, sp, sg = t.tolist()
+    else:
+        sp, sg = sum(t_pro), sum(t_gemm)
+    assert bat.bat_device_error() == 0, "a kernel reported a stalled wait"
+
+    flop = 2.0 * w.M * w.N * w.K
+    value = flop * K_ * world / t_step / 1e12
+    peaks, peak_src = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    gemm_tf = flop / (sg / K_) / 1e12
+    pro_bytes = PROLOGUE_BYTES_PER_ELT * w.M * w.K
+    pro_gbs = pro_bytes / (sp / K_) / 1e9
+
+    # end to end through the public API: pinned host X -> device, linear, Y -> pinned host
+    e2e = None
+    if not args.no_e2e:
+        Xh = torch.from_numpy(X_host.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+        Yh = torch.empty(w.M, w.N, dtype=torch.bfloat16).pin_memory()
+        Xdev = torch.empty_like(X)
+        ws = torch.empty(bat.bat_linear_workspace_bytes(w.M, w.K), dtype=torch.uint8, device=dev)
+
+        def e2e_step():
+            Xdev.copy_(Xh, non_blocking=True)
+            bat.bat_linear(Xdev, Wq, A, B, gl, gh, Y=Y, out_dtype=torch.bfloat16, workspace=ws,
+                           stream=stream)
+            Yh.copy_(Y, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        if pg:
+            pg.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = e0.elapsed_time(e1) * 1e-3
+        if pg:
+            t = torch.tensor([te], dtype=torch.float64, device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            te = t.item()
+        e2e = {"value": flop * args.e2e_steps * world / te / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(X.numel() * 2), "d2h_bytes_per_step": int(Y.numel() * 2)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        fl, dt, desc, thr = oracle_sample(inp, w, args.cpu_budget_s)
+        cpu = {"value": fl / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+               "sample": desc, "seconds": round(dt, 2)}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": K_, "warmup": args.warmup, "ms_per_step": 1e3 * t_step / K_,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "mxfp4", "data": "synthetic",
+            "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "out": "bf16",
+                       "l2": "flushed between steps (256 MiB write outside the timed events)",
+                       "parallelism": f"replicas x{world} (independent token batches)"},
+            "gpu_launches": 2 * K_ * world,
+            "roofline": {"bound": "tensor", "achieved": gemm_tf, "peak": fp4_peak,
+                         "unit": "TFLOP/s", "frac": gemm_tf / fp4_peak, "traffic": None,
+                         "kernel": "bat_mxf4_gemm_kernel",
+                         "peak_source": f"{peak_src} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/BF16)"},
+            "prologue": {"bound": "hbm", "achieved": pro_gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": pro_gbs / peaks["hbm_gbs"],
+                         "us_per_launch": 1e6 * sp / K_, "traffic": None,
+                         "kernel": "bat_prologue_kernel", "peak_source": peak_src},
+            "gemm_us_per_launch": 1e6 * sg / K_,
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,191 @@
+/*
+ * bat.h — C-ABI of the BATQuant W4A4 (MXFP4) linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The operation (BATQuant note, en.papernotes.org, "Method > Key Designs 1-3";
+ * nubint.ai review, "proposed method"):
+ *
+ *   Y = Q(X P) . Q(P^-1 W^T)
+ *
+ * X is M x K bf16 (tokens x in-features), W is N x K bf16 (out x in), P is
+ * block-diagonal with one 32 x 32 block per 32-channel MXFP4 block b, and each
+ * block is the Global-and-Private Kronecker product P_b = B_b (x) A: A is one
+ * 8 x 8 factor shared by every block, B_b a private 4 x 4 factor. A block x of
+ * 32 values read as the row-major 4 x 8 matrix X_r[i][p] = x[8i+p] maps to
+ * y = x P_b = vec_row(B_b^T X_r A). Q is block-wise learnable clipping to
+ * [sigma(g_lo_b) * min(y), sigma(g_hi_b) * max(y)] followed by MXFP4
+ * quantization: E2M1 codes (grid 0, .5, 1, 1.5, 2, 3, 4, 6 and negatives),
+ * one UE8M0 scale 2^e per 32 elements with e = floor(log2 amax) - 2,
+ * round-to-nearest-even, saturating at +-6 ("Background & Motivation").
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller. The online entry
+ *     points never allocate device memory; the offline bat_prepare_weight
+ *     allocates (and frees, stream-ordered) one temporary of 256 + 64*K/32 bytes
+ *     for the inverted factors. No state is kept between calls except a sticky
+ *     device error word (see bat_device_error).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
+ *     asynchronous on it unless stated otherwise.
+ *   - Arguments are validated on the host before any CUDA call; a bad argument
+ *     returns an error status and launches nothing. CUDA failures return
+ *     BAT_ERR_CUDA. The device must be sm_100 (B200); other devices get
+ *     BAT_ERR_UNSUPPORTED.
+ *   - Calls are thread-safe (no mutable global state on the host).
+ *
+ * Storage formats (bat_mxfp4_t):
+ *   codes : [rows][k/2] bytes, row-major, two E2M1 codes per byte, element 2i in
+ *           the low nibble and 2i+1 in the high nibble; sign in bit 3 of a code.
+ *   scales: UE8M0 bytes (value 2^(byte-127)) in a tiled order the GEMM reads
+ *           directly: rows padded to a multiple of 128, blocks (k/32) padded to a
+ *           multiple of 4; the byte of (row m, block b) sits at
+ *             ((m/128)*nbp4 + b/4)*512 + (m%32)*16 + ((m%128)/32)*4 + b%4,
+ *           nbp4 = ceil((k/32)/4). Padding bytes are written as 0.
+ */
+#ifndef BAT_H_
+#define BAT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BAT_API __attribute__((visibility("default")))
+#else
+#define BAT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BAT_OK = 0,
+  BAT_ERR_INVALID_ARG = 1, /* null pointer, negative or zero size, bad enum */
+  BAT_ERR_SHAPE = 2,       /* k % 32 != 0, operand shapes disagree, size over a limit */
+  BAT_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned */
+  BAT_ERR_SINGULAR = 4,    /* A or some B_b is singular or ill-conditioned */
+  BAT_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
+  BAT_ERR_UNSUPPORTED = 6, /* device is not sm_100, or a feature outside this build */
+  BAT_ERR_WORKSPACE = 7,   /* workspace pointer null or smaller than required */
+  BAT_ERR_DEVICE = 8       /* a kernel reported a failure through the device error word */
+} bat_status_t;
+
+typedef enum { BAT_OUT_BF16 = 0, BAT_OUT_F32 = 1 } bat_out_dtype_t;
+
+/* An MXFP4 matrix with `rows` rows of `k` elements; buffers owned by the caller. */
+typedef struct {
+  void* codes;  /* device, bat_mxfp4_codes_bytes(rows, k) bytes, 16-byte aligned */
+  void* scales; /* device, bat_mxfp4_scales_bytes(rows, k) bytes, 16-byte aligned */
+  int64_t rows;
+  int64_t k;
+} bat_mxfp4_t;
+
+/* Sizes of the two buffers of an MXFP4 matrix (0 if k % 32 != 0 or a size < 1). */
+BAT_API size_t bat_mxfp4_codes_bytes(int64_t rows, int64_t k);
+BAT_API size_t bat_mxfp4_scales_bytes(int64_t rows, int64_t k);
+
+/* Human-readable name of a status code (static storage). */
+BAT_API const char* bat_status_string(bat_status_t status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+BAT_API int bat_version(void);
+
+/*
+ * Online activation path: block transform, block clip, MXFP4 quantize + pack.
+ * (Key Designs 2 "GPK decomposition" and 3 "Block-wise learnable clipping";
+ * Method > "Overall Architecture": activation-side transforms run online.)
+ *
+ *   X     : bf16 [M][K] row-major, 16-byte aligned.
+ *   A     : fp32 [8][8] row-major (shared factor).
+ *   B     : fp32 [K/32][4][4] row-major (private factors, one per block).
+ *   g_lo, g_hi : fp32 [K/32] clip logits, or both NULL for no clipping.
+ *                Ratios are sigma(g) evaluated in fp64 and rounded to fp32;
+ *                g = +inf gives ratio 1.
+ *   Xq    : output; Xq->rows must equal M and Xq->k must equal K.
+ * Requirements: M >= 1, K >= 32, K % 32 == 0, K <= 262144.
+ */
+BAT_API bat_status_t bat_quantize_act(const void* X, int64_t M, int64_t K, const float* A, const float* B,
+                              const float* g_lo, const float* g_hi, const bat_mxfp4_t* Xq,
+                              void* stream);
+
+/*
+ * Same as bat_quantize_act, and also writes the fp32 transformed values y
+ * (before clipping) to `y_out` (device fp32 [M][K]). For testing and
+ * inspection; slower because of the extra 4 bytes per element.
+ */
+BAT_API bat_status_t bat_quantize_act_trace(const void* X, int64_t M, int64_t K, const float* A,
+                                    const float* B, const float* g_lo, const float* g_hi,
+                                    const bat_mxfp4_t* Xq, float* y_out, void* stream);
+
+/*
+ * The clip ratios the prologue uses: r[t] = fp32(1 / (1 + exp(-g[t]))) computed
+ * in fp64 on the device (g = +inf gives 1; g == NULL gives all ones).
+ * g, r: device fp32 [n].
+ */
+BAT_API bat_status_t bat_clip_ratios(const float* g, int64_t n, float* r, void* stream);
+
+/*
+ * MXFP4 element conversion as the prologue performs it: codes[t] = E2M1 code of
+ * v[t] (round-to-nearest-even, saturating at +-6, sign in bit 3), one code per
+ * byte. Values are converted in pairs (2t, 2t+1) exactly as the prologue packs
+ * them. v: device fp32 [n]; codes: device uint8 [n].
+ */
+BAT_API bat_status_t bat_e2m1_encode(const float* v, int64_t n, uint8_t* codes, void* stream);
+
+/*
+ * Offline weight side (Method > "Overall Architecture": the inverse transform is
+ * fused into the weights once). Row n, block b of W becomes
+ * w_b (B_b^-T (x) A^-T) = vec_row(B_b^-1 W_r A^-T), the rows of (P^-1 W^T)^T;
+ * then optional per-(row, block) clipping and MXFP4 packing.
+ *
+ *   W      : bf16 [N][K] row-major, 16-byte aligned.
+ *   A, B   : as in bat_quantize_act (device). They are copied to the host and
+ *            inverted in fp64 with partial pivoting; a factor whose 1-norm
+ *            condition number exceeds 1e6 returns BAT_ERR_SINGULAR.
+ *   gw_lo, gw_hi : fp32 [N][K/32] weight clip logits, or both NULL (default: no clip).
+ *   Wq     : output, Wq->rows == N, Wq->k == K.
+ *   wt_out : optional device fp32 [N][K] for the transformed weights (NULL to skip).
+ * This call synchronizes `stream` (it reads A and B on the host). It is meant to
+ * run once per layer and is not on the timed path.
+ */
+BAT_API bat_status_t bat_prepare_weight(const void* W, int64_t N, int64_t K, const float* A,
+                                const float* B, const float* gw_lo, const float* gw_hi,
+                                const bat_mxfp4_t* Wq, float* wt_out, void* stream);
+
+/*
+ * Block-scaled MXFP4 GEMM on the 5th-generation tensor cores (tcgen05,
+ * kind::mxf4, fp32 accumulation in tensor memory):
+ *   Y[m][n] = sum_b 2^(eX[m][b] + eW[n][b]) * sum_{j<32} x[m][32b+j] * w[n][32b+j]
+ * (the low-bit product Q(XP) . Q(P^-1 W^T) of Key Designs 1).
+ *
+ *   Xq : M x K MXFP4 activations; Wq : N x K MXFP4 weights (Xq->k == Wq->k).
+ *   Y  : device [M][N] row-major, bf16 or fp32 per `out_dtype`, 16-byte aligned.
+ */
+BAT_API bat_status_t bat_mxfp4_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
+                            bat_out_dtype_t out_dtype, void* stream);
+
+/* Workspace bytes bat_linear needs for M rows of K inputs (the quantized X). */
+BAT_API size_t bat_linear_workspace_bytes(int64_t M, int64_t K);
+
+/*
+ * The whole online linear layer Y = Q(XP) . Q(P^-1 W^T): bat_quantize_act into
+ * `workspace`, then bat_mxfp4_gemm, on one stream.
+ *   X  : bf16 [M][K]; Wq from bat_prepare_weight (Wq->k == K); A, B, g_lo, g_hi
+ *        as in bat_quantize_act; Y: [M][Wq->rows] in `out_dtype`.
+ *   workspace : device, >= bat_linear_workspace_bytes(M, K) bytes, 256-byte aligned.
+ */
+BAT_API bat_status_t bat_linear(const void* X, int64_t M, const bat_mxfp4_t* Wq, const float* A,
+                        const float* B, const float* g_lo, const float* g_hi, void* Y,
+                        bat_out_dtype_t out_dtype, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/*
+ * Reads and clears the sticky device error word the kernels set when a bounded
+ * wait runs out (a pipeline stall that should never happen). Returns 0 if no
+ * kernel reported a failure since the last call; synchronizes the device.
+ */
+BAT_API int bat_device_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BAT_H_ */

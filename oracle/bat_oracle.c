@@ -35,6 +35,9 @@
  *   - ties on the grid go to the even code (mantissa bit 0); |v| > 6 gives 6.
  */
 #include <math.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -303,4 +306,13 @@ int orc_weight_transform_f64(const uint16_t* W, int64_t N, int64_t K, const floa
     }
   free(P);
   return 0;
+}
+
+/* Threads the OpenMP loops above use (1 without OpenMP). */
+int orc_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
 }

@@ -44,6 +44,7 @@ def lib():
         L.orc_weight_transform_f64.argtypes = [P, I64, I64, P, P, P]
         L.orc_weight_transform_f64.restype = ctypes.c_int
         L.orc_kron.argtypes = [P, P, P]
+        L.orc_num_threads.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -200,3 +201,8 @@ def gpk_param_counts(K: int, shared: int = 8, private: int = 4) -> dict:
         "naive_kronecker": nb * (shared * shared + private * private),
         "full_blocks": nb * g * g,
     }
+
+
+def num_threads() -> int:
+    """Host threads the oracle's parallel loops use."""
+    return int(lib().orc_num_threads())

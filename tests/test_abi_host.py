@@ -1,0 +1,86 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function the
+header declares, and rejects bad arguments on the host before any CUDA call."""
+from __future__ import annotations
+
+import ctypes
+
+import pytest
+
+import w4a4_bit_gemm_b200 as bat
+from oracle import formats
+
+
+@pytest.fixture(scope="module")
+def L():
+    from w4a4_bit_gemm_b200 import build
+    build.build()
+    return bat.lib()
+
+
+def test_exports_every_declared_function(L):
+    names = bat.declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_only_declared_functions_exported():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", bat.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    ours = {n for n in exported if n.startswith("bat_")}
+    assert ours == set(bat.declared_functions())
+
+
+def test_sizes_match_documented_layout(L):
+    for rows, k in [(1, 32), (64, 256), (130, 160), (2048, 4096), (16384, 4096), (6144, 4096)]:
+        assert bat.bat_mxfp4_codes_bytes(rows, k) == rows * k // 2
+        assert bat.bat_mxfp4_scales_bytes(rows, k) == formats.scale_bytes(rows, k // 32)
+    assert bat.bat_mxfp4_codes_bytes(4, 48) == 0
+    assert bat.bat_mxfp4_scales_bytes(0, 64) == 0
+    assert bat.bat_linear_workspace_bytes(100, 64) == 3328 + formats.scale_bytes(100, 2)
+
+
+def test_status_strings(L):
+    assert bat.bat_status_string(0) == "BAT_OK"
+    assert bat.bat_status_string(4) == "BAT_ERR_SINGULAR"
+    assert bat.bat_version() >= 100
+
+
+def _fake_ptr(offset=0):
+    return ctypes.c_void_p(0x7F0000000000 + offset)
+
+
+def test_host_validation_returns_before_cuda(L):
+    S = bat.MXFP4Struct
+    good = S(0x7F0000100000, 0x7F0000200000, 4, 64)
+    p = _fake_ptr()
+    # null X
+    assert L.bat_quantize_act(None, 4, 64, p, p, None, None, ctypes.byref(good), None) == 1
+    # K not a multiple of 32
+    g48 = S(0x7F0000100000, 0x7F0000200000, 4, 48)
+    assert L.bat_quantize_act(p, 4, 48, p, p, None, None, ctypes.byref(g48), None) == 2
+    # only one of the clip logits
+    assert L.bat_quantize_act(p, 4, 64, p, p, p, None, ctypes.byref(good), None) == 1
+    # output shape disagrees with X
+    bad_rows = S(0x7F0000100000, 0x7F0000200000, 5, 64)
+    assert L.bat_quantize_act(p, 4, 64, p, p, None, None, ctypes.byref(bad_rows), None) == 2
+    # misaligned X
+    assert L.bat_quantize_act(_fake_ptr(2), 4, 64, p, p, None, None, ctypes.byref(good), None) == 3
+    # GEMM: K mismatch, bad dtype enum, misaligned Y
+    w = S(0x7F0000300000, 0x7F0000400000, 8, 96)
+    assert L.bat_mxfp4_gemm(ctypes.byref(good), ctypes.byref(w), p, 0, None) == 2
+    w64 = S(0x7F0000300000, 0x7F0000400000, 8, 64)
+    assert L.bat_mxfp4_gemm(ctypes.byref(good), ctypes.byref(w64), p, 7, None) == 1
+    assert L.bat_mxfp4_gemm(ctypes.byref(good), ctypes.byref(w64), _fake_ptr(4), 0, None) == 3
+    # linear: workspace too small or missing
+    assert L.bat_linear(p, 4, ctypes.byref(w64), p, p, None, None, p, 0, None, 0, None) == 7
+    assert L.bat_linear(p, 4, ctypes.byref(w64), p, p, None, None, p, 0, p, 16, None) == 7
+    # weight prep: K too large / invalid N
+    w_big = S(0x7F0000300000, 0x7F0000400000, 8, 262144 + 32)
+    assert L.bat_prepare_weight(p, 8, 262144 + 32, p, p, None, None, ctypes.byref(w_big), None, None) == 2
+    assert L.bat_prepare_weight(p, 0, 64, p, p, None, None, ctypes.byref(w64), None, None) == 1
+    # element conversion / ratios: bad sizes
+    assert L.bat_e2m1_encode(p, 0, p, None) == 1
+    assert L.bat_clip_ratios(p, 0, p, None) == 1

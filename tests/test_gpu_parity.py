@@ -1,0 +1,275 @@
+"""CUDA path vs the CPU oracle, element by element, through the C-ABI.
+
+Bars (BATQuant W4A4 linear; readings of the pages as stated in the oracle):
+  * E2M1 codes and UE8M0 scale bytes: bit-exact when the oracle quantizer is fed
+    the GPU's fp32 transformed values and the GPU's fp32 clip ratios;
+  * transformed values: block-normwise |y_gpu - y_ref|_inf <= 1e-5 |y_ref|_inf;
+  * GEMM: relative Frobenius error <= 1e-3 against the oracle's fp64 product of
+    the same dequantized operands (fp32 output), and bf16 output against the
+    bf16-rounded fp64 product.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import formats
+import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+TRANSFORM_TOL = 1e-5
+GEMM_TOL = 1e-3
+
+
+@pytest.fixture(scope="module")
+def bat():
+    import w4a4_bit_gemm_b200 as m
+    m.lib()
+    return m
+
+
+def _dev_bf16(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).cuda()
+
+
+def _dev_f32(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda()
+
+
+def _host(q, rows, K):
+    codes = formats.unpack_codes(q.codes.cpu().numpy().reshape(rows, K // 2))
+    tiled = q.scales.cpu().numpy()
+    scales = formats.untile_scales(tiled, rows, K // 32)
+    return codes, scales, tiled
+
+
+def _check_transform(y_gpu: np.ndarray, y_ref: np.ndarray):
+    rows, K = y_ref.shape
+    g = y_gpu.reshape(rows, K // 32, 32).astype(np.float64)
+    r = y_ref.reshape(rows, K // 32, 32).astype(np.float64)
+    err = np.max(np.abs(g - r), axis=2)
+    ref = np.max(np.abs(r), axis=2)
+    bad = err > TRANSFORM_TOL * ref
+    assert not bad.any(), (np.argwhere(bad)[:5], (err / np.maximum(ref, 1e-300)).max())
+
+
+def _run_act(bat, X, A, B, g_lo, g_hi):
+    Xd = _dev_bf16(X)
+    Ad, Bd = _dev_f32(A), _dev_f32(B)
+    gl = None if g_lo is None else _dev_f32(g_lo)
+    gh = None if g_hi is None else _dev_f32(g_hi)
+    Xq, y = bat.bat_quantize_act_trace(Xd, Ad, Bd, gl, gh)
+    Xq2 = bat.bat_quantize_act(Xd, Ad, Bd, gl, gh)
+    torch.cuda.synchronize()
+    assert torch.equal(Xq.codes, Xq2.codes) and torch.equal(Xq.scales, Xq2.scales)
+    nb = X.shape[1] // 32
+    r_lo = bat.bat_clip_ratios(gl, nb).cpu().numpy()
+    r_hi = bat.bat_clip_ratios(gh, nb).cpu().numpy()
+    return Xq, y.cpu().numpy(), r_lo, r_hi
+
+
+def _check_act(bat, X, A, B, g_lo, g_hi):
+    rows, K = X.shape
+    Xq, y_gpu, r_lo, r_hi = _run_act(bat, X, A, B, g_lo, g_hi)
+    nb = K // 32
+    assert np.array_equal(r_lo, oracle.clip_ratios(g_lo, nb))
+    assert np.array_equal(r_hi, oracle.clip_ratios(g_hi, nb))
+    _check_transform(y_gpu, oracle.transform(X, A, B))
+    codes, scales, tiled = _host(Xq, rows, K)
+    oc, os_, bad = oracle.quantize(y_gpu, r_lo, r_hi)
+    assert bad == 0
+    mism = np.argwhere(codes != oc)
+    assert mism.size == 0, (mism[:5], codes[tuple(mism[0])], oc[tuple(mism[0])])
+    assert np.array_equal(scales, os_)
+    assert np.all(tiled[formats.padding_mask(rows, nb)] == 0)
+    return Xq, codes, scales
+
+
+# ---------------------------------------------------------------- element conversion
+def test_e2m1_conversion_every_fp32_up_to_8(bat):
+    top = int(np.float32(8.0).view(np.uint32))
+    step = 1 << 26
+    for start in range(0, top + 1, step):
+        bits = np.arange(start, min(start + step, top + 1), dtype=np.uint32)
+        v = bits.view(np.float32)
+        got = bat.bat_e2m1_encode(_dev_f32(v)).cpu().numpy()
+        assert np.array_equal(got, oracle.e2m1_encode(v)), start
+    rng = np.random.default_rng(2)
+    bits = rng.integers(0, 0x7F800000, size=1 << 22, dtype=np.uint32) | np.uint32(0x80000000)
+    v = np.concatenate([bits.view(np.float32), np.array([-0.0, 0.0, -1e-30, 1e-30, -7.0, 1e30], np.float32)])
+    got = bat.bat_e2m1_encode(_dev_f32(v)).cpu().numpy()
+    assert np.array_equal(got, oracle.e2m1_encode(v))
+
+
+def test_clip_ratios(bat):
+    g = np.concatenate([np.linspace(-20, 20, 4001, dtype=np.float32),
+                        np.array([np.inf, 0.0, 1e-8], np.float32)])
+    r = bat.bat_clip_ratios(_dev_f32(g)).cpu().numpy()
+    assert np.array_equal(r, oracle.clip_ratios(g))
+    assert np.all(bat.bat_clip_ratios(None, 7).cpu().numpy() == 1.0)
+
+
+# ---------------------------------------------------------------- prologue
+@pytest.mark.parametrize("name", wl.ORDER)
+def test_quantize_act_workloads(bat, name):
+    inp = wl.make_inputs(name, with_weight=False)
+    _check_act(bat, inp.X, inp.A, inp.B, inp.g_lo, inp.g_hi)
+
+
+@pytest.mark.parametrize("M,K", [(1, 32), (1, 4096), (17, 96), (130, 160), (3, 1056), (129, 4128),
+                                 (64, 1024 + 96)])
+def test_quantize_act_ragged(bat, M, K):
+    X = wl.random_bf16((M, K), seed=M * 7 + K, scale=3.0)
+    A, B, g_lo, g_hi = wl.random_factors(K // 32, seed=K)
+    _check_act(bat, X, A, B, g_lo, g_hi)
+
+
+def test_quantize_act_no_clip_identity_is_rtn(bat):
+    """Identity factors and no clip give plain MXFP4 round-to-nearest of X."""
+    inp = wl.make_inputs("tiny", with_weight=False)
+    nb = inp.B.shape[0]
+    A = np.eye(8, dtype=np.float32)
+    B = np.repeat(np.eye(4, dtype=np.float32)[None], nb, axis=0)
+    Xq, codes, scales = _check_act(bat, inp.X, A, B, None, None)
+    _, oc, os_ = oracle.quantize_act(inp.X, A, B, None, None)
+    assert np.array_equal(codes, oc) and np.array_equal(scales, os_)
+
+
+def test_quantize_act_zero_and_constant_rows(bat):
+    M, K = 8, 256
+    X = np.zeros((M, K), np.uint16)
+    X[1] = wl.f32_to_bf16_bits(np.full(K, -2.5, np.float32))
+    X[2, :32] = wl.f32_to_bf16_bits(np.full(32, 1e-30, np.float32))
+    X[3] = wl.f32_to_bf16_bits(np.full(K, 1e30, np.float32))
+    A, B, g_lo, g_hi = wl.random_factors(K // 32, seed=4)
+    _check_act(bat, X, A, B, g_lo, g_hi)
+
+
+# ---------------------------------------------------------------- weight side
+@pytest.mark.parametrize("clip", [False, True])
+@pytest.mark.parametrize("N,K", [(128, 256), (200, 96), (1, 4096), (384, 4096)])
+def test_prepare_weight(bat, N, K, clip):
+    W = wl.random_bf16((N, K), seed=N + K, scale=0.02)
+    A, B, _, _ = wl.random_factors(K // 32, seed=K + 1)
+    rng = np.random.default_rng(N)
+    gw_lo = rng.uniform(1, 4, size=(N, K // 32)).astype(np.float32) if clip else None
+    gw_hi = rng.uniform(1, 4, size=(N, K // 32)).astype(np.float32) if clip else None
+    wt = torch.empty(N, K, dtype=torch.float32, device="cuda")
+    Wq = bat.bat_prepare_weight(_dev_bf16(W), _dev_f32(A), _dev_f32(B),
+                                None if gw_lo is None else _dev_f32(gw_lo),
+                                None if gw_hi is None else _dev_f32(gw_hi), wt_out=wt)
+    torch.cuda.synchronize()
+    wt_gpu = wt.cpu().numpy()
+    _check_transform(wt_gpu, oracle.weight_transform_f64(W, A, B).astype(np.float32))
+    r_lo = None if gw_lo is None else oracle.clip_ratios(gw_lo.reshape(-1)).reshape(N, -1)
+    r_hi = None if gw_hi is None else oracle.clip_ratios(gw_hi.reshape(-1)).reshape(N, -1)
+    oc, os_, _ = oracle.quantize(wt_gpu, r_lo, r_hi, per_row=True)
+    codes, scales, tiled = _host(Wq, N, K)
+    assert np.array_equal(codes, oc)
+    assert np.array_equal(scales, os_)
+    assert np.all(tiled[formats.padding_mask(N, K // 32)] == 0)
+
+
+def test_prepare_weight_singular(bat):
+    K = 64
+    W = wl.random_bf16((8, K), seed=1)
+    A, B, _, _ = wl.random_factors(K // 32, seed=2)
+    B[1] = 0.0
+    with pytest.raises(bat.BatError) as e:
+        bat.bat_prepare_weight(_dev_bf16(W), _dev_f32(A), _dev_f32(B))
+    assert e.value.status == 4
+
+
+# ---------------------------------------------------------------- GEMM
+def _gemm_check(bat, Xq, Wq, M, N, K, rows=None, cols=None):
+    xc, xs, _ = _host(Xq, M, K)
+    wc, ws, _ = _host(Wq, N, K)
+    Xd = oracle.dequantize(xc, xs)
+    Wd = oracle.dequantize(wc, ws)
+    Y32 = bat.bat_mxfp4_gemm(Xq, Wq, out_dtype=torch.float32)
+    Y16 = bat.bat_mxfp4_gemm(Xq, Wq, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    ref = oracle.gemm_sampled(Xd, Wd, rows, cols)
+    r = np.arange(M) if rows is None else np.asarray(rows)
+    c = np.arange(N) if cols is None else np.asarray(cols)
+    y32 = Y32.cpu().numpy()[np.ix_(r, c)].astype(np.float64)
+    y16 = Y16.float().cpu().numpy()[np.ix_(r, c)].astype(np.float64)
+    assert np.all(np.isfinite(y32))
+    rel = np.linalg.norm(y32 - ref) / max(np.linalg.norm(ref), 1e-300)
+    assert rel <= GEMM_TOL, rel
+    # each output's error is far inside fp32 accumulation of the absolute terms
+    mag = oracle.gemm_sampled(np.abs(Xd), np.abs(Wd), rows, cols)
+    assert np.all(np.abs(y32 - ref) <= 1e-5 * mag + 1e-30), np.max(np.abs(y32 - ref) / (mag + 1e-30))
+    ref16 = torch.from_numpy(ref).to(torch.bfloat16).float().numpy().astype(np.float64)
+    rel16 = np.linalg.norm(y16 - ref16) / max(np.linalg.norm(ref16), 1e-300)
+    assert rel16 <= GEMM_TOL, rel16
+    return rel
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (64, 128, 256), (1, 8, 32), (17, 200, 96),
+                                   (130, 300, 160), (256, 512, 1024), (200, 264, 4128),
+                                   (300, 1000, 2048)])
+def test_gemm_shapes(bat, M, N, K):
+    X = wl.random_bf16((M, K), seed=M + 3 * K, scale=2.0)
+    W = wl.random_bf16((N, K), seed=N + 5 * K, scale=0.02)
+    A, B, g_lo, g_hi = wl.random_factors(K // 32, seed=K + 9)
+    Xq = bat.bat_quantize_act(_dev_bf16(X), _dev_f32(A), _dev_f32(B), _dev_f32(g_lo), _dev_f32(g_hi))
+    Wq = bat.bat_prepare_weight(_dev_bf16(W), _dev_f32(A), _dev_f32(B))
+    _gemm_check(bat, Xq, Wq, M, N, K)
+
+
+def _sample(n, count, seed):
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, n // 2, n - 1] + ([127, 128] if n > 128 else [])
+    return np.unique(np.concatenate([fixed, rng.integers(0, n, size=count)]))
+
+
+@pytest.mark.parametrize("name", wl.ORDER)
+def test_linear_workloads(bat, name):
+    """bat_linear at the full workload sizes, as the benchmark launches it; sampled outputs."""
+    inp = wl.make_inputs(name)
+    w = wl.WORKLOADS[name]
+    Xd = _dev_bf16(inp.X)
+    Ad, Bd = _dev_f32(inp.A), _dev_f32(inp.B)
+    gl, gh = _dev_f32(inp.g_lo), _dev_f32(inp.g_hi)
+    Wq = bat.bat_prepare_weight(_dev_bf16(inp.W), Ad, Bd)
+    Y = bat.bat_linear(Xd, Wq, Ad, Bd, gl, gh, out_dtype=torch.float32)
+    Xq = bat.bat_quantize_act(Xd, Ad, Bd, gl, gh)
+    Y2 = bat.bat_mxfp4_gemm(Xq, Wq, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y2)  # unfused linear == quantize then GEMM, bit for bit
+    rows = None if w.M <= 64 else _sample(w.M, 24, 1)
+    cols = None if w.N <= 512 else _sample(w.N, 200, 2)
+    # oracle path end to end (its own quantizer on its own transform)
+    x_codes, x_scales, _ = _host(Xq, w.M, w.K)
+    w_codes, w_scales, _ = _host(Wq, w.N, w.K)
+    ref = oracle.gemm_sampled(oracle.dequantize(x_codes, x_scales),
+                              oracle.dequantize(w_codes, w_scales), rows, cols)
+    r = np.arange(w.M) if rows is None else rows
+    c = np.arange(w.N) if cols is None else cols
+    y = Y.cpu().numpy()[np.ix_(r, c)].astype(np.float64)
+    rel = np.linalg.norm(y - ref) / np.linalg.norm(ref)
+    assert rel <= GEMM_TOL, rel
+    # and against the oracle's own quantization of its own transform (same codes almost everywhere)
+    if w.M * w.K <= 2048 * 4096:
+        _, oc, os_ = oracle.quantize_act(inp.X, inp.A, inp.B, inp.g_lo, inp.g_hi)
+        agree = np.mean(oc == x_codes)
+        assert agree > 0.999, agree
+    assert bat.bat_device_error() == 0
+
+
+def test_argument_errors_launch_nothing(bat):
+    X = torch.zeros(4, 64, dtype=torch.bfloat16, device="cuda")
+    A = torch.eye(8, device="cuda")
+    B = torch.eye(4, device="cuda").repeat(2, 1, 1).contiguous()
+    Xq = bat.MXFP4.empty(4, 64)
+    bad = bat.MXFP4(Xq.codes, Xq.scales, 5, 64)
+    with pytest.raises(bat.BatError) as e:
+        bat.bat_quantize_act(X, A, B, Xq=bad)
+    assert e.value.status == 2
+    st = bat.lib().bat_quantize_act(None, 4, 64, None, None, None, None, None, None)
+    assert st == 1
+    assert bat.bat_device_error() == 0

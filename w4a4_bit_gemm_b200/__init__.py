@@ -1,0 +1,269 @@
+"""BATQuant W4A4 (MXFP4) linear layer for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C-ABI in ``include/bat.h`` (``libbat.so``, built
+in-tree by ``w4a4_bit_gemm_b200.build``). Every function here only marshals
+torch tensors into pointers and sizes; all arithmetic runs in the library's
+CUDA kernels. There is no CPU fallback: if the library cannot be loaded the
+calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbat.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "bat.h")
+
+BAT_OUT_BF16 = 0
+BAT_OUT_F32 = 1
+
+_STATUS = {
+    0: "BAT_OK", 1: "BAT_ERR_INVALID_ARG", 2: "BAT_ERR_SHAPE", 3: "BAT_ERR_ALIGN",
+    4: "BAT_ERR_SINGULAR", 5: "BAT_ERR_CUDA", 6: "BAT_ERR_UNSUPPORTED", 7: "BAT_ERR_WORKSPACE",
+    8: "BAT_ERR_DEVICE",
+}
+
+
+class BatError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_STATUS.get(status, status)}")
+
+
+class MXFP4Struct(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("k", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load ``libbat.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: run w4a4_bit_gemm_b200.build.build() first")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I64, S = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    SP = ctypes.POINTER(MXFP4Struct)
+    sig = {
+        "bat_mxfp4_codes_bytes": (ctypes.c_size_t, [I64, I64]),
+        "bat_mxfp4_scales_bytes": (ctypes.c_size_t, [I64, I64]),
+        "bat_status_string": (ctypes.c_char_p, [S]),
+        "bat_version": (S, []),
+        "bat_quantize_act": (S, [P, I64, I64, P, P, P, P, SP, P]),
+        "bat_quantize_act_trace": (S, [P, I64, I64, P, P, P, P, SP, P, P]),
+        "bat_clip_ratios": (S, [P, I64, P, P]),
+        "bat_e2m1_encode": (S, [P, I64, P, P]),
+        "bat_prepare_weight": (S, [P, I64, I64, P, P, P, P, SP, P, P]),
+        "bat_mxfp4_gemm": (S, [SP, SP, P, S, P]),
+        "bat_linear_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
+        "bat_linear": (S, [P, I64, SP, P, P, P, P, P, S, P, ctypes.c_size_t, P]),
+        "bat_device_error": (S, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def declared_functions() -> list[str]:
+    """Names of the functions ``include/bat.h`` declares."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bat_[a-z0-9_]+)\s*\(", text)))
+
+
+# ---------------------------------------------------------------- marshalling helpers
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, name: str, shape=None) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise BatError(status, where)
+
+
+@dataclass
+class MXFP4:
+    """An MXFP4 matrix: packed E2M1 codes [rows][k/2] and tiled UE8M0 scales."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    rows: int
+    k: int
+
+    @staticmethod
+    def empty(rows: int, k: int, device="cuda") -> "MXFP4":
+        cb = bat_mxfp4_codes_bytes(rows, k)
+        sb = bat_mxfp4_scales_bytes(rows, k)
+        if cb == 0 or sb == 0:
+            raise ValueError(f"invalid MXFP4 shape rows={rows} k={k}")
+        return MXFP4(torch.empty(cb, dtype=torch.uint8, device=device),
+                     torch.empty(sb, dtype=torch.uint8, device=device), rows, k)
+
+    def struct(self) -> MXFP4Struct:
+        return MXFP4Struct(self.codes.data_ptr(), self.scales.data_ptr(), self.rows, self.k)
+
+
+# ---------------------------------------------------------------- C-ABI wrappers
+def bat_mxfp4_codes_bytes(rows: int, k: int) -> int:
+    return lib().bat_mxfp4_codes_bytes(rows, k)
+
+
+def bat_mxfp4_scales_bytes(rows: int, k: int) -> int:
+    return lib().bat_mxfp4_scales_bytes(rows, k)
+
+
+def bat_status_string(status: int) -> str:
+    return lib().bat_status_string(status).decode()
+
+
+def bat_version() -> int:
+    return lib().bat_version()
+
+
+def _act_args(X, A, B, g_lo, g_hi):
+    M, K = X.shape
+    _need(X, torch.bfloat16, "X")
+    _need(A, torch.float32, "A", (8, 8))
+    _need(B, torch.float32, "B", (K // 32, 4, 4))
+    if (g_lo is None) != (g_hi is None):
+        raise ValueError("g_lo and g_hi must both be given or both be None")
+    if g_lo is not None:
+        _need(g_lo, torch.float32, "g_lo", (K // 32,))
+        _need(g_hi, torch.float32, "g_hi", (K // 32,))
+    return M, K
+
+
+def bat_quantize_act(X, A, B, g_lo=None, g_hi=None, Xq: Optional[MXFP4] = None, stream=None) -> MXFP4:
+    M, K = _act_args(X, A, B, g_lo, g_hi)
+    Xq = MXFP4.empty(M, K, X.device) if Xq is None else Xq
+    st = Xq.struct()
+    _check(lib().bat_quantize_act(_ptr(X), M, K, _ptr(A), _ptr(B), _ptr(g_lo), _ptr(g_hi),
+                                  ctypes.byref(st), _stream(stream)), "bat_quantize_act")
+    return Xq
+
+
+def bat_quantize_act_trace(X, A, B, g_lo=None, g_hi=None, Xq: Optional[MXFP4] = None,
+                           y_out: Optional[torch.Tensor] = None, stream=None):
+    M, K = _act_args(X, A, B, g_lo, g_hi)
+    Xq = MXFP4.empty(M, K, X.device) if Xq is None else Xq
+    y_out = torch.empty(M, K, dtype=torch.float32, device=X.device) if y_out is None else y_out
+    _need(y_out, torch.float32, "y_out", (M, K))
+    st = Xq.struct()
+    _check(lib().bat_quantize_act_trace(_ptr(X), M, K, _ptr(A), _ptr(B), _ptr(g_lo), _ptr(g_hi),
+                                        ctypes.byref(st), _ptr(y_out), _stream(stream)),
+           "bat_quantize_act_trace")
+    return Xq, y_out
+
+
+def bat_clip_ratios(g: Optional[torch.Tensor], n: Optional[int] = None, r=None, stream=None):
+    if g is not None:
+        _need(g, torch.float32, "g")
+        n = g.numel()
+    r = torch.empty(n, dtype=torch.float32, device="cuda") if r is None else r
+    _check(lib().bat_clip_ratios(_ptr(g), n, _ptr(r), _stream(stream)), "bat_clip_ratios")
+    return r
+
+
+def bat_e2m1_encode(v: torch.Tensor, codes=None, stream=None) -> torch.Tensor:
+    _need(v, torch.float32, "v")
+    codes = torch.empty(v.numel(), dtype=torch.uint8, device=v.device) if codes is None else codes
+    _check(lib().bat_e2m1_encode(_ptr(v), v.numel(), _ptr(codes), _stream(stream)), "bat_e2m1_encode")
+    return codes
+
+
+def bat_prepare_weight(W, A, B, gw_lo=None, gw_hi=None, Wq: Optional[MXFP4] = None,
+                       wt_out: Optional[torch.Tensor] = None, stream=None) -> MXFP4:
+    N, K = W.shape
+    _need(W, torch.bfloat16, "W")
+    _need(A, torch.float32, "A", (8, 8))
+    _need(B, torch.float32, "B", (K // 32, 4, 4))
+    if (gw_lo is None) != (gw_hi is None):
+        raise ValueError("gw_lo and gw_hi must both be given or both be None")
+    if gw_lo is not None:
+        _need(gw_lo, torch.float32, "gw_lo", (N, K // 32))
+        _need(gw_hi, torch.float32, "gw_hi", (N, K // 32))
+    if wt_out is not None:
+        _need(wt_out, torch.float32, "wt_out", (N, K))
+    Wq = MXFP4.empty(N, K, W.device) if Wq is None else Wq
+    st = Wq.struct()
+    _check(lib().bat_prepare_weight(_ptr(W), N, K, _ptr(A), _ptr(B), _ptr(gw_lo), _ptr(gw_hi),
+                                    ctypes.byref(st), _ptr(wt_out), _stream(stream)),
+           "bat_prepare_weight")
+    return Wq
+
+
+def _out_code(out_dtype: torch.dtype) -> int:
+    if out_dtype == torch.bfloat16:
+        return BAT_OUT_BF16
+    if out_dtype == torch.float32:
+        return BAT_OUT_F32
+    raise ValueError("out_dtype must be torch.bfloat16 or torch.float32")
+
+
+def bat_mxfp4_gemm(Xq: MXFP4, Wq: MXFP4, Y: Optional[torch.Tensor] = None,
+                   out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
+    code = _out_code(out_dtype)
+    Y = torch.empty(Xq.rows, Wq.rows, dtype=out_dtype, device=Xq.codes.device) if Y is None else Y
+    _need(Y, out_dtype, "Y", (Xq.rows, Wq.rows))
+    a, b = Xq.struct(), Wq.struct()
+    _check(lib().bat_mxfp4_gemm(ctypes.byref(a), ctypes.byref(b), _ptr(Y), code, _stream(stream)),
+           "bat_mxfp4_gemm")
+    return Y
+
+
+def bat_linear_workspace_bytes(M: int, K: int) -> int:
+    return lib().bat_linear_workspace_bytes(M, K)
+
+
+def bat_linear(X, Wq: MXFP4, A, B, g_lo=None, g_hi=None, Y: Optional[torch.Tensor] = None,
+               out_dtype: torch.dtype = torch.bfloat16, workspace: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    M, K = _act_args(X, A, B, g_lo, g_hi)
+    code = _out_code(out_dtype)
+    Y = torch.empty(M, Wq.rows, dtype=out_dtype, device=X.device) if Y is None else Y
+    _need(Y, out_dtype, "Y", (M, Wq.rows))
+    need = bat_linear_workspace_bytes(M, K)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    _need(workspace, torch.uint8, "workspace")
+    b = Wq.struct()
+    _check(lib().bat_linear(_ptr(X), M, ctypes.byref(b), _ptr(A), _ptr(B), _ptr(g_lo), _ptr(g_hi),
+                            _ptr(Y), code, _ptr(workspace), workspace.numel(), _stream(stream)),
+           "bat_linear")
+    return Y
+
+
+def bat_device_error() -> int:
+    return lib().bat_device_error()

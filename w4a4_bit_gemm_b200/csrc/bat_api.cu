@@ -1,0 +1,451 @@
+// C-ABI of the BATQuant W4A4 linear layer: host validation, launch
+// configuration, tensor maps and the offline fp64 inverse of the weight side.
+// Every kernel of the library is compiled in this one translation unit.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+#include "../../include/bat.h"
+#include "bat_common.cuh"
+#include "bat_gemm.cuh"
+#include "bat_prologue.cuh"
+
+namespace {
+
+constexpr int64_t kMaxK = 262144;
+constexpr double kMaxCond = 1e6;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+
+// ---------------------------------------------------------------- device facts (cached)
+struct DeviceInfo {
+  std::atomic<int> state{0};  // 0 unknown, 1 sm_100, 2 unsupported
+  std::atomic<int> sms{0};
+  std::atomic<int> gemm_attr{0};
+  std::atomic<int> pro_attr{0};
+};
+DeviceInfo g_dev[64];
+
+bat_status_t current_device(int* dev_out, int* sms_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BAT_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return BAT_ERR_UNSUPPORTED;
+  DeviceInfo& d = g_dev[dev];
+  int st = d.state.load();
+  if (st == 0) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return BAT_ERR_CUDA;
+    d.sms.store(sms);
+    st = (major == 10 && minor == 0) ? 1 : 2;
+    d.state.store(st);
+  }
+  if (st != 1) return BAT_ERR_UNSUPPORTED;
+  *dev_out = dev;
+  *sms_out = d.sms.load();
+  return BAT_OK;
+}
+
+bat_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? BAT_OK : BAT_ERR_CUDA; }
+
+// ---------------------------------------------------------------- tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::atomic<EncodeTiledFn> fn{nullptr};
+  EncodeTiledFn f = fn.load();
+  if (f) return f;
+  void* ptr = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  f = reinterpret_cast<EncodeTiledFn>(ptr);
+  fn.store(f);
+  return f;
+}
+
+// Codes of an MXFP4 matrix seen as a [rows][k/2] byte tensor, box of 128 bytes x box_rows,
+// 128-byte swizzle (the K-major operand layout of the MMA).
+bool make_code_map(CUtensorMap* map, const void* codes, int64_t rows, int64_t k, uint32_t box_rows) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(k / 2), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(k / 2)};
+  cuuint32_t box[2] = {128u, box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = f(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides,
+                 box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- fp64 inverse (host)
+// Gauss-Jordan elimination with partial pivoting on an n x n row-major matrix.
+// Returns false if a pivot vanishes or the 1-norm condition number exceeds kMaxCond.
+bool invert(int n, const double* a_in, double* inv) {
+  std::vector<double> a(a_in, a_in + n * n);
+  for (int i = 0; i < n * n; ++i) inv[i] = 0.0;
+  for (int i = 0; i < n; ++i) inv[i * n + i] = 1.0;
+  double norm_a = 0.0;
+  for (int c = 0; c < n; ++c) {
+    double s = 0.0;
+    for (int r = 0; r < n; ++r) s += std::fabs(a_in[r * n + c]);
+    norm_a = std::fmax(norm_a, s);
+  }
+  for (int c = 0; c < n; ++c) {
+    int piv = c;
+    for (int r = c + 1; r < n; ++r)
+      if (std::fabs(a[r * n + c]) > std::fabs(a[piv * n + c])) piv = r;
+    const double pv = a[piv * n + c];
+    if (!(std::fabs(pv) > 0.0) || !std::isfinite(pv)) return false;
+    if (piv != c)
+      for (int j = 0; j < n; ++j) {
+        std::swap(a[c * n + j], a[piv * n + j]);
+        std::swap(inv[c * n + j], inv[piv * n + j]);
+      }
+    for (int j = 0; j < n; ++j) {
+      a[c * n + j] /= pv;
+      inv[c * n + j] /= pv;
+    }
+    for (int r = 0; r < n; ++r) {
+      if (r == c) continue;
+      const double f = a[r * n + c];
+      if (f == 0.0) continue;
+      for (int j = 0; j < n; ++j) {
+        a[r * n + j] -= f * a[c * n + j];
+        inv[r * n + j] -= f * inv[c * n + j];
+      }
+    }
+  }
+  double norm_inv = 0.0;
+  for (int c = 0; c < n; ++c) {
+    double s = 0.0;
+    for (int r = 0; r < n; ++r) s += std::fabs(inv[r * n + c]);
+    norm_inv = std::fmax(norm_inv, s);
+  }
+  const double cond = norm_a * norm_inv;
+  return std::isfinite(cond) && cond <= kMaxCond;
+}
+
+// ---------------------------------------------------------------- prologue launch
+bat_status_t check_mxfp4(const bat_mxfp4_t* q, int64_t rows, int64_t k) {
+  if (!q || !q->codes || !q->scales) return BAT_ERR_INVALID_ARG;
+  if (q->rows != rows || q->k != k) return BAT_ERR_SHAPE;
+  if (!aligned16(q->codes) || !aligned16(q->scales)) return BAT_ERR_ALIGN;
+  return BAT_OK;
+}
+
+bat_status_t check_act_args(const void* X, int64_t M, int64_t K, const float* A, const float* B,
+                            const float* g_lo, const float* g_hi, const bat_mxfp4_t* Xq) {
+  if (!X || !A || !B || !Xq) return BAT_ERR_INVALID_ARG;
+  if ((g_lo == nullptr) != (g_hi == nullptr)) return BAT_ERR_INVALID_ARG;
+  if (M < 1 || K < 32) return BAT_ERR_INVALID_ARG;
+  if (K % 32 != 0 || K > kMaxK) return BAT_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B)) return BAT_ERR_ALIGN;
+  return check_mxfp4(Xq, M, K);
+}
+
+bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float* A,
+                             const float* B, const float* g_lo, const float* g_hi, bool per_row,
+                             const bat_mxfp4_t* out, float* y_out, cudaStream_t stream) {
+  int dev = 0, sms = 0;
+  bat_status_t st = current_device(&dev, &sms);
+  if (st != BAT_OK) return st;
+  bat::PrologueParams p;
+  p.x = static_cast<const uint16_t*>(X);
+  p.a = A;
+  p.b = B;
+  p.g_lo = g_lo;
+  p.g_hi = g_hi;
+  p.codes = static_cast<uint8_t*>(out->codes);
+  p.scales = static_cast<uint8_t*>(out->scales);
+  p.y_out = y_out;
+  p.rows = rows;
+  p.K = K;
+  p.nb = static_cast<int>(K / 32);
+  p.nseg = (p.nb + 31) / 32;
+  p.nbp4 = (p.nb + 3) / 4;
+  const size_t smem = per_row ? 0 : static_cast<size_t>(2 * p.nb) * sizeof(float);
+  const int threads = 256;
+  void (*kern)(bat::PrologueParams);
+  if (per_row)
+    kern = y_out ? bat::bat_prologue_kernel<true, true> : bat::bat_prologue_kernel<false, true>;
+  else
+    kern = y_out ? bat::bat_prologue_kernel<true, false> : bat::bat_prologue_kernel<false, false>;
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return BAT_ERR_CUDA;
+  }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess)
+    return BAT_ERR_CUDA;
+  per_sm = per_sm < 1 ? 1 : per_sm;
+  const int64_t units = rows * p.nseg;
+  const int64_t need = (units + (threads / 32) - 1) / (threads / 32);
+  int64_t grid = static_cast<int64_t>(sms) * per_sm;
+  if (need < grid) grid = need;
+  if (grid < 1) grid = 1;
+  kern<<<static_cast<unsigned>(grid), threads, smem, stream>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
+bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
+                         bat_out_dtype_t out_dtype, cudaStream_t stream) {
+  int dev = 0, sms = 0;
+  bat_status_t st = current_device(&dev, &sms);
+  if (st != BAT_OK) return st;
+  CUtensorMap ta, tb;
+  if (!make_code_map(&ta, Xq->codes, Xq->rows, Xq->k, bat::gemm::kBM)) return BAT_ERR_CUDA;
+  if (!make_code_map(&tb, Wq->codes, Wq->rows, Wq->k, bat::gemm::kBN)) return BAT_ERR_CUDA;
+  bat::GemmParams p;
+  p.sfa = static_cast<const uint8_t*>(Xq->scales);
+  p.sfb = static_cast<const uint8_t*>(Wq->scales);
+  p.y = Y;
+  p.M = Xq->rows;
+  p.N = Wq->rows;
+  p.K = Xq->k;
+  p.nbp4 = static_cast<int>((Xq->k / 32 + 3) / 4);
+  p.out_f32 = out_dtype == BAT_OUT_F32 ? 1 : 0;
+  p.vec_ok = (p.N % (p.out_f32 ? 4 : 8)) == 0 ? 1 : 0;
+  DeviceInfo& d = g_dev[dev];
+  if (!d.gemm_attr.load()) {
+    if (cudaFuncSetAttribute(bat::bat_mxf4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bat::gemm::kSmemBytes) != cudaSuccess)
+      return BAT_ERR_CUDA;
+    d.gemm_attr.store(1);
+  }
+  const int64_t tiles = ((p.M + bat::gemm::kBM - 1) / bat::gemm::kBM) *
+                        ((p.N + bat::gemm::kBN - 1) / bat::gemm::kBN);
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  bat::bat_mxf4_gemm_kernel<<<grid, bat::gemm::kThreads, bat::gemm::kSmemBytes, stream>>>(ta, tb, p);
+  return cuda_status(cudaGetLastError());
+}
+
+bat_status_t check_gemm_args(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, const void* Y,
+                             bat_out_dtype_t out_dtype) {
+  if (!Xq || !Wq || !Y) return BAT_ERR_INVALID_ARG;
+  if (out_dtype != BAT_OUT_BF16 && out_dtype != BAT_OUT_F32) return BAT_ERR_INVALID_ARG;
+  if (Xq->rows < 1 || Wq->rows < 1 || Xq->k < 32) return BAT_ERR_INVALID_ARG;
+  if (Xq->k != Wq->k || Xq->k % 32 != 0 || Xq->k > kMaxK) return BAT_ERR_SHAPE;
+  bat_status_t st = check_mxfp4(Xq, Xq->rows, Xq->k);
+  if (st != BAT_OK) return st;
+  st = check_mxfp4(Wq, Wq->rows, Wq->k);
+  if (st != BAT_OK) return st;
+  if (!aligned16(Y)) return BAT_ERR_ALIGN;
+  return BAT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int bat_version(void) { return 100; }
+
+const char* bat_status_string(bat_status_t s) {
+  switch (s) {
+    case BAT_OK: return "BAT_OK";
+    case BAT_ERR_INVALID_ARG: return "BAT_ERR_INVALID_ARG";
+    case BAT_ERR_SHAPE: return "BAT_ERR_SHAPE";
+    case BAT_ERR_ALIGN: return "BAT_ERR_ALIGN";
+    case BAT_ERR_SINGULAR: return "BAT_ERR_SINGULAR";
+    case BAT_ERR_CUDA: return "BAT_ERR_CUDA";
+    case BAT_ERR_UNSUPPORTED: return "BAT_ERR_UNSUPPORTED";
+    case BAT_ERR_WORKSPACE: return "BAT_ERR_WORKSPACE";
+    case BAT_ERR_DEVICE: return "BAT_ERR_DEVICE";
+  }
+  return "BAT_ERR_UNKNOWN";
+}
+
+size_t bat_mxfp4_codes_bytes(int64_t rows, int64_t k) {
+  if (rows < 1 || k < 32 || k % 32 != 0) return 0;
+  return static_cast<size_t>(rows) * static_cast<size_t>(k / 2);
+}
+
+size_t bat_mxfp4_scales_bytes(int64_t rows, int64_t k) {
+  if (rows < 1 || k < 32 || k % 32 != 0) return 0;
+  const int64_t nbp4 = (k / 32 + 3) / 4;
+  return static_cast<size_t>(round_up(rows, 128) / 128) * static_cast<size_t>(nbp4) * 512u;
+}
+
+bat_status_t bat_quantize_act(const void* X, int64_t M, int64_t K, const float* A, const float* B,
+                              const float* g_lo, const float* g_hi, const bat_mxfp4_t* Xq,
+                              void* stream) {
+  bat_status_t st = check_act_args(X, M, K, A, B, g_lo, g_hi, Xq);
+  if (st != BAT_OK) return st;
+  return launch_prologue(X, M, K, A, B, g_lo, g_hi, false, Xq, nullptr,
+                         static_cast<cudaStream_t>(stream));
+}
+
+bat_status_t bat_quantize_act_trace(const void* X, int64_t M, int64_t K, const float* A,
+                                    const float* B, const float* g_lo, const float* g_hi,
+                                    const bat_mxfp4_t* Xq, float* y_out, void* stream) {
+  bat_status_t st = check_act_args(X, M, K, A, B, g_lo, g_hi, Xq);
+  if (st != BAT_OK) return st;
+  if (!y_out) return BAT_ERR_INVALID_ARG;
+  if (!aligned16(y_out)) return BAT_ERR_ALIGN;
+  return launch_prologue(X, M, K, A, B, g_lo, g_hi, false, Xq, y_out,
+                         static_cast<cudaStream_t>(stream));
+}
+
+bat_status_t bat_clip_ratios(const float* g, int64_t n, float* r, void* stream) {
+  if (!r || n < 1) return BAT_ERR_INVALID_ARG;
+  int dev = 0, sms = 0;
+  bat_status_t st = current_device(&dev, &sms);
+  if (st != BAT_OK) return st;
+  const int64_t blocks = (n + 255) / 256;
+  bat::bat_clip_ratio_kernel<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), 256, 0,
+                               static_cast<cudaStream_t>(stream)>>>(g, n, r);
+  return cuda_status(cudaGetLastError());
+}
+
+bat_status_t bat_e2m1_encode(const float* v, int64_t n, uint8_t* codes, void* stream);
+
+bat_status_t bat_prepare_weight(const void* W, int64_t N, int64_t K, const float* A,
+                                const float* B, const float* gw_lo, const float* gw_hi,
+                                const bat_mxfp4_t* Wq, float* wt_out, void* stream) {
+  if (!W || !A || !B || !Wq) return BAT_ERR_INVALID_ARG;
+  if ((gw_lo == nullptr) != (gw_hi == nullptr)) return BAT_ERR_INVALID_ARG;
+  if (N < 1 || K < 32) return BAT_ERR_INVALID_ARG;
+  if (K % 32 != 0 || K > kMaxK) return BAT_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(A) || !aligned16(B)) return BAT_ERR_ALIGN;
+  if (wt_out && !aligned16(wt_out)) return BAT_ERR_ALIGN;
+  bat_status_t st = check_mxfp4(Wq, N, K);
+  if (st != BAT_OK) return st;
+  int dev = 0, sms = 0;
+  st = current_device(&dev, &sms);
+  if (st != BAT_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t nb = K / 32;
+  std::vector<float> ha(64), hb(static_cast<size_t>(nb) * 16);
+  if (cudaMemcpyAsync(ha.data(), A, 64 * sizeof(float), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemcpyAsync(hb.data(), B, hb.size() * sizeof(float), cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return BAT_ERR_CUDA;
+  // Inverse-transposed factors: w_b (B_b^-T (x) A^-T) = vec_row(B_b^-1 W_r A^-T), which the
+  // prologue computes as vec_row(F_b^T W_r G) with G = A^-T and F_b = B_b^-T.
+  std::vector<float> fac(64 + static_cast<size_t>(nb) * 16);
+  {
+    double a[64], inv[64];
+    for (int i = 0; i < 64; ++i) a[i] = ha[i];
+    if (!invert(8, a, inv)) return BAT_ERR_SINGULAR;
+    for (int p = 0; p < 8; ++p)
+      for (int q = 0; q < 8; ++q) fac[p * 8 + q] = static_cast<float>(inv[q * 8 + p]);
+  }
+  for (int64_t b = 0; b < nb; ++b) {
+    double m[16], inv[16];
+    for (int i = 0; i < 16; ++i) m[i] = hb[b * 16 + i];
+    if (!invert(4, m, inv)) return BAT_ERR_SINGULAR;
+    for (int i = 0; i < 4; ++i)
+      for (int j = 0; j < 4; ++j) fac[64 + b * 16 + i * 4 + j] = static_cast<float>(inv[j * 4 + i]);
+  }
+  // Offline only: one temporary device buffer for the inverse factors (stream-ordered).
+  void* dfac = nullptr;
+  if (cudaMallocAsync(&dfac, fac.size() * sizeof(float), s) != cudaSuccess) return BAT_ERR_CUDA;
+  st = cuda_status(cudaMemcpyAsync(dfac, fac.data(), fac.size() * sizeof(float),
+                                   cudaMemcpyHostToDevice, s));
+  if (st == BAT_OK) {
+    const float* da = static_cast<const float*>(dfac);
+    st = launch_prologue(W, N, K, da, da + 64, gw_lo, gw_hi, true, Wq, wt_out, s);
+  }
+  cudaFreeAsync(dfac, s);
+  // `fac` is read by the async copy: wait before it goes out of scope.
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BAT_ERR_CUDA;
+  return st;
+}
+
+bat_status_t bat_mxfp4_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
+                            bat_out_dtype_t out_dtype, void* stream) {
+  bat_status_t st = check_gemm_args(Xq, Wq, Y, out_dtype);
+  if (st != BAT_OK) return st;
+  return launch_gemm(Xq, Wq, Y, out_dtype, static_cast<cudaStream_t>(stream));
+}
+
+size_t bat_linear_workspace_bytes(int64_t M, int64_t K) {
+  const size_t c = bat_mxfp4_codes_bytes(M, K);
+  const size_t s = bat_mxfp4_scales_bytes(M, K);
+  if (!c || !s) return 0;
+  return static_cast<size_t>(round_up(static_cast<int64_t>(c), 256)) + s;
+}
+
+bat_status_t bat_linear(const void* X, int64_t M, const bat_mxfp4_t* Wq, const float* A,
+                        const float* B, const float* g_lo, const float* g_hi, void* Y,
+                        bat_out_dtype_t out_dtype, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  if (!Wq) return BAT_ERR_INVALID_ARG;
+  const int64_t K = Wq->k;
+  if (M < 1 || K < 32) return BAT_ERR_INVALID_ARG;
+  if (K % 32 != 0 || K > kMaxK) return BAT_ERR_SHAPE;
+  const size_t need = bat_linear_workspace_bytes(M, K);
+  if (!workspace || workspace_bytes < need) return BAT_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BAT_ERR_ALIGN;
+  bat_mxfp4_t xq;
+  xq.codes = workspace;
+  xq.scales = static_cast<uint8_t*>(workspace) + round_up(static_cast<int64_t>(bat_mxfp4_codes_bytes(M, K)), 256);
+  xq.rows = M;
+  xq.k = K;
+  bat_status_t st = check_act_args(X, M, K, A, B, g_lo, g_hi, &xq);
+  if (st != BAT_OK) return st;
+  st = check_gemm_args(&xq, Wq, Y, out_dtype);
+  if (st != BAT_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_prologue(X, M, K, A, B, g_lo, g_hi, false, &xq, nullptr, s);
+  if (st != BAT_OK) return st;
+  return launch_gemm(&xq, Wq, Y, out_dtype, s);
+}
+
+int bat_device_error(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, bat::g_dev_error, sizeof(v)) != cudaSuccess) return -1;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(bat::g_dev_error, &zero, sizeof(zero)) != cudaSuccess) return -1;
+  return static_cast<int>(v);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- element conversion
+namespace bat {
+__global__ void bat_e2m1_encode_kernel(const float* v, int64_t n, uint8_t* codes) {
+  // Pairs (2t, 2t+1) go through the same conversion as the prologue (2t in the
+  // low nibble); each code is returned in its own byte (sign in bit 3).
+  const int64_t pairs = (n + 1) / 2;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < pairs;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float lo = v[2 * t];
+    const float hi = (2 * t + 1 < n) ? v[2 * t + 1] : 0.0f;
+    const uint32_t byte = e2m1x2(lo, hi);
+    codes[2 * t] = static_cast<uint8_t>(byte & 0xFu);
+    if (2 * t + 1 < n) codes[2 * t + 1] = static_cast<uint8_t>(byte >> 4);
+  }
+}
+}  // namespace bat
+
+extern "C" bat_status_t bat_e2m1_encode(const float* v, int64_t n, uint8_t* codes, void* stream) {
+  if (!v || !codes || n < 1) return BAT_ERR_INVALID_ARG;
+  int dev = 0, sms = 0;
+  bat_status_t st = current_device(&dev, &sms);
+  if (st != BAT_OK) return st;
+  int64_t blocks = ((n + 1) / 2 + 255) / 256;
+  if (blocks > static_cast<int64_t>(sms) * 32) blocks = static_cast<int64_t>(sms) * 32;
+  bat::bat_e2m1_encode_kernel<<<static_cast<unsigned>(blocks), 256, 0,
+                                static_cast<cudaStream_t>(stream)>>>(v, n, codes);
+  return cuda_status(cudaGetLastError());
+}
