@@ -178,6 +178,40 @@ BAT_API bat_status_t bat_linear(const void* X, int64_t M, const bat_mxfp4_t* Wq,
                         void* stream);
 
 /*
+ * Allocation-free variant of bat_linear. There is no counterpart on the pages:
+ * the method's linear layer is bat_linear; this entry point exists only for
+ * callers that cannot hand the library a workspace.
+ *
+ * Who needs it: code that may not call cudaMalloc, and cannot get a device
+ * buffer from its host framework either. Examples are plugins run under an
+ * allocator that has already reserved all device memory, and serving loops
+ * that must not allocate (or make the implicit device synchronization an
+ * allocation can cause) once they are running.
+ *
+ * Instead of a caller workspace, the quantized activations go into a scratch
+ * array of BAT_NOALLOC_SCRATCH_BYTES that the library defines in device memory
+ * (a static __device__ array). Every GPU that loads the library holds that
+ * array until the process exits. Nothing here calls cudaMalloc, cudaFree or any
+ * other allocating routine.
+ *   - Limit: bat_linear_workspace_bytes(M, Wq->k) must be at most
+ *     BAT_NOALLOC_SCRATCH_BYTES (for example M = 2048 at K = 4096, M = 512 at
+ *     K = 12288); larger calls return BAT_ERR_WORKSPACE and launch nothing.
+ *   - The first call on each device looks up the array's device address with
+ *     that device current (cudaGetSymbolAddress) and caches it. Make that first
+ *     call before any stream capture.
+ *   - All calls share the one array, and it keeps the last call's contents.
+ *     Every byte a call reads is written by that same call first, so nothing
+ *     needs clearing. Calls that overlap on the GPU (other streams, other host
+ *     threads) race on the array: the caller must order them.
+ * Other arguments, results and errors are exactly those of bat_linear.
+ */
+#define BAT_NOALLOC_SCRATCH_BYTES (8u << 20)
+BAT_API bat_status_t bat_linear_noalloc(const void* X, int64_t M, const bat_mxfp4_t* Wq,
+                                        const float* A, const float* B, const float* g_lo,
+                                        const float* g_hi, void* Y, bat_out_dtype_t out_dtype,
+                                        void* stream);
+
+/*
  * Reads and clears the sticky device error word the kernels set when a bounded
  * wait runs out (a pipeline stall that should never happen). Returns 0 if no
  * kernel reported a failure since the last call; synchronizes the device.

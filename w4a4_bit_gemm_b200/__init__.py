@@ -67,6 +67,7 @@ def lib() -> ctypes.CDLL:
         "bat_mxfp4_gemm": (S, [SP, SP, P, S, P]),
         "bat_linear_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
         "bat_linear": (S, [P, I64, SP, P, P, P, P, P, S, P, ctypes.c_size_t, P]),
+        "bat_linear_noalloc": (S, [P, I64, SP, P, P, P, P, P, S, P]),
         "bat_device_error": (S, []),
     }
     for name, (res, args) in sig.items():
@@ -262,6 +263,24 @@ def bat_linear(X, Wq: MXFP4, A, B, g_lo=None, g_hi=None, Y: Optional[torch.Tenso
     _check(lib().bat_linear(_ptr(X), M, ctypes.byref(b), _ptr(A), _ptr(B), _ptr(g_lo), _ptr(g_hi),
                             _ptr(Y), code, _ptr(workspace), workspace.numel(), _stream(stream)),
            "bat_linear")
+    return Y
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20  # BAT_NOALLOC_SCRATCH_BYTES in include/bat.h
+
+
+def bat_linear_noalloc(X, Wq: MXFP4, A, B, g_lo=None, g_hi=None, Y: Optional[torch.Tensor] = None,
+                       out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
+    """bat_linear without a workspace: the library's own static device scratch holds
+    the quantized activations (for callers that cannot allocate device memory)."""
+    M, K = _act_args(X, A, B, g_lo, g_hi)
+    code = _out_code(out_dtype)
+    Y = torch.empty(M, Wq.rows, dtype=out_dtype, device=X.device) if Y is None else Y
+    _need(Y, out_dtype, "Y", (M, Wq.rows))
+    b = Wq.struct()
+    _check(lib().bat_linear_noalloc(_ptr(X), M, ctypes.byref(b), _ptr(A), _ptr(B), _ptr(g_lo),
+                                    _ptr(g_hi), _ptr(Y), code, _stream(stream)),
+           "bat_linear_noalloc")
     return Y
 
 

@@ -449,3 +449,63 @@ extern "C" bat_status_t bat_e2m1_encode(const float* v, int64_t n, uint8_t* code
                                 static_cast<cudaStream_t>(stream)>>>(v, n, codes);
   return cuda_status(cudaGetLastError());
 }
+
+// ---------------------------------------------------------------- allocation-free linear
+// Scratch for bat_linear_noalloc: holds the quantized activations (codes, then
+// tiled scales at a 256-byte boundary). Host code must not use this name as an
+// address; the device address comes from cudaGetSymbolAddress per device.
+static __device__ __align__(256) uint8_t bat_noalloc_scratch[BAT_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::atomic<void*> g_noalloc_addr[64];
+
+// Device address of the scratch array on the current device `dev` (looked up once).
+bat_status_t noalloc_scratch(int dev, void** out) {
+  void* p = g_noalloc_addr[dev].load();
+  if (p == nullptr) {
+    if (cudaGetSymbolAddress(&p, bat_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return BAT_ERR_CUDA;
+    g_noalloc_addr[dev].store(p);
+  }
+  *out = p;
+  return BAT_OK;
+}
+}  // namespace
+
+extern "C" bat_status_t bat_linear_noalloc(const void* X, int64_t M, const bat_mxfp4_t* Wq,
+                                           const float* A, const float* B, const float* g_lo,
+                                           const float* g_hi, void* Y, bat_out_dtype_t out_dtype,
+                                           void* stream) {
+  if (!Wq) return BAT_ERR_INVALID_ARG;
+  const int64_t K = Wq->k;
+  if (M < 1 || K < 32) return BAT_ERR_INVALID_ARG;
+  if (K % 32 != 0 || K > kMaxK) return BAT_ERR_SHAPE;
+  const size_t need = bat_linear_workspace_bytes(M, K);
+  if (need == 0 || need > BAT_NOALLOC_SCRATCH_BYTES) return BAT_ERR_WORKSPACE;
+  bat_mxfp4_t xq;
+  xq.codes = nullptr;  // placeholder until the device address is known
+  xq.scales = nullptr;
+  xq.rows = M;
+  xq.k = K;
+  // Validate with stand-in aligned addresses first, so bad arguments launch nothing.
+  bat_mxfp4_t probe = xq;
+  probe.codes = reinterpret_cast<void*>(static_cast<uintptr_t>(256));
+  probe.scales = reinterpret_cast<void*>(static_cast<uintptr_t>(512));
+  bat_status_t st = check_act_args(X, M, K, A, B, g_lo, g_hi, &probe);
+  if (st != BAT_OK) return st;
+  st = check_gemm_args(&probe, Wq, Y, out_dtype);
+  if (st != BAT_OK) return st;
+  int dev = 0, sms = 0;
+  st = current_device(&dev, &sms);
+  if (st != BAT_OK) return st;
+  void* scratch = nullptr;
+  st = noalloc_scratch(dev, &scratch);
+  if (st != BAT_OK) return st;
+  xq.codes = scratch;
+  xq.scales = static_cast<uint8_t*>(scratch) +
+              round_up(static_cast<int64_t>(bat_mxfp4_codes_bytes(M, K)), 256);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_prologue(X, M, K, A, B, g_lo, g_hi, false, &xq, nullptr, s);
+  if (st != BAT_OK) return st;
+  return launch_gemm(&xq, Wq, Y, out_dtype, s);
+}
