@@ -30,7 +30,8 @@ struct DeviceInfo {
   std::atomic<int> state{0};  // 0 unknown, 1 sm_100, 2 unsupported
   std::atomic<int> sms{0};
   std::atomic<int> gemm_attr{0};
-  std::atomic<int> pro_attr{0};
+  std::atomic<int> pro_attr{0};     // bit t: the prologue variant t has its smem attribute set
+  std::atomic<int> pro_per_sm{0};   // resident prologue CTAs per SM
 };
 DeviceInfo g_dev[64];
 
@@ -90,6 +91,21 @@ bool make_code_map(CUtensorMap* map, const void* codes, int64_t rows, int64_t k,
   cuuint32_t estr[2] = {1u, 1u};
   CUresult r = f(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides,
                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// bf16 Y [M][N] for the GEMM's TMA store: box of 64 columns (128 bytes) x 128 rows,
+// 128-byte swizzle, matching the epilogue's staging layout. Needs N % 8 == 0.
+bool make_out_map(CUtensorMap* map, void* y, int64_t M, int64_t N) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(N * 2)};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(bat::gemm::kBM)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = f(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -180,28 +196,38 @@ bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float
   p.nb = static_cast<int>(K / 32);
   p.nseg = (p.nb + 31) / 32;
   p.nbp4 = (p.nb + 3) / 4;
-  const size_t smem = per_row ? 0 : static_cast<size_t>(2 * p.nb) * sizeof(float);
-  const int threads = 256;
   void (*kern)(bat::PrologueParams);
   if (per_row)
     kern = y_out ? bat::bat_prologue_kernel<true, true> : bat::bat_prologue_kernel<false, true>;
   else
     kern = y_out ? bat::bat_prologue_kernel<true, false> : bat::bat_prologue_kernel<false, false>;
-  if (smem > 48 * 1024) {
+  DeviceInfo& d = g_dev[dev];
+  const int variant_bit = 1 << ((per_row ? 2 : 0) + (y_out ? 1 : 0));
+  if (!(d.pro_attr.load() & variant_bit)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
+                             bat::pro::kSmemBytes) != cudaSuccess)
       return BAT_ERR_CUDA;
+    d.pro_attr.fetch_or(variant_bit);
   }
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess)
-    return BAT_ERR_CUDA;
-  per_sm = per_sm < 1 ? 1 : per_sm;
-  const int64_t units = rows * p.nseg;
-  const int64_t need = (units + (threads / 32) - 1) / (threads / 32);
-  int64_t grid = static_cast<int64_t>(sms) * per_sm;
-  if (need < grid) grid = need;
-  if (grid < 1) grid = 1;
-  kern<<<static_cast<unsigned>(grid), threads, smem, stream>>>(p);
+  int per_sm = d.pro_per_sm.load();
+  if (per_sm == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bat::bat_prologue_kernel<false, false>,
+                                                      bat::pro::kThreads, bat::pro::kSmemBytes) != cudaSuccess)
+      return BAT_ERR_CUDA;
+    per_sm = per_sm < 1 ? 1 : per_sm;
+    d.pro_per_sm.store(per_sm);
+  }
+  // One CTA per (segment of 32 blocks, range of rows); about one CTA per SM slot.
+  const int64_t slots = static_cast<int64_t>(sms) * per_sm;
+  const int64_t max_parts = (rows + bat::pro::kRowsPerStage - 1) / bat::pro::kRowsPerStage;
+  int64_t parts = slots / p.nseg;
+  if (parts > max_parts) parts = max_parts;
+  if (parts < 1) parts = 1;
+  p.rows_per_cta = (rows + parts - 1) / parts;
+  parts = (rows + p.rows_per_cta - 1) / p.rows_per_cta;
+  const int64_t grid = parts * p.nseg;
+  if (grid > 0x7FFFFFFF) return BAT_ERR_SHAPE;
+  kern<<<static_cast<unsigned>(grid), bat::pro::kThreads, bat::pro::kSmemBytes, stream>>>(p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -210,9 +236,10 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
   int dev = 0, sms = 0;
   bat_status_t st = current_device(&dev, &sms);
   if (st != BAT_OK) return st;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, ty;
   if (!make_code_map(&ta, Xq->codes, Xq->rows, Xq->k, bat::gemm::kBM)) return BAT_ERR_CUDA;
   if (!make_code_map(&tb, Wq->codes, Wq->rows, Wq->k, bat::gemm::kBN)) return BAT_ERR_CUDA;
+  std::memset(&ty, 0, sizeof(ty));
   bat::GemmParams p;
   p.sfa = static_cast<const uint8_t*>(Xq->scales);
   p.sfb = static_cast<const uint8_t*>(Wq->scales);
@@ -223,6 +250,9 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
   p.nbp4 = static_cast<int>((Xq->k / 32 + 3) / 4);
   p.out_f32 = out_dtype == BAT_OUT_F32 ? 1 : 0;
   p.vec_ok = (p.N % (p.out_f32 ? 4 : 8)) == 0 ? 1 : 0;
+  // bf16 output with 16-byte rows goes through shared-memory staging and TMA stores
+  p.tma_store = (!p.out_f32 && p.vec_ok) ? 1 : 0;
+  if (p.tma_store && !make_out_map(&ty, Y, p.M, p.N)) return BAT_ERR_CUDA;
   DeviceInfo& d = g_dev[dev];
   if (!d.gemm_attr.load()) {
     if (cudaFuncSetAttribute(bat::bat_mxf4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -233,7 +263,7 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
   const int64_t tiles = ((p.M + bat::gemm::kBM - 1) / bat::gemm::kBM) *
                         ((p.N + bat::gemm::kBN - 1) / bat::gemm::kBN);
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  bat::bat_mxf4_gemm_kernel<<<grid, bat::gemm::kThreads, bat::gemm::kSmemBytes, stream>>>(ta, tb, p);
+  bat::bat_mxf4_gemm_kernel<<<grid, bat::gemm::kThreads, bat::gemm::kSmemBytes, stream>>>(ta, tb, ty, p);
   return cuda_status(cudaGetLastError());
 }
 

@@ -32,7 +32,12 @@ constexpr int kSfaBytes = (kBM / 128) * kChunksPerStage * kChunk;  // 1 KB
 constexpr int kSfbBytes = (kBN / 128) * kChunksPerStage * kChunk;  // 2 KB
 constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
 constexpr int kThreads = 192;
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+// bf16 output staging for the TMA store: one box of 128 rows x 64 columns (128 bytes,
+// 128-byte swizzle); the epilogue holds its whole bf16 tile in registers and
+// streams it through this box one 64-column slice at a time.
+constexpr int kEpiBoxBytes = kBM * 128;
+constexpr int kEpiBytes = kEpiBoxBytes;  // 16 KB
+constexpr int kSmemBytes = kStages * kStageBytes + kEpiBytes + 1024 /*align*/ + 256 /*barriers*/;
 // TMEM columns: accumulator [0, 256), A scales [256, 264), B scales [264, 280).
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfaCol = 256;
@@ -47,7 +52,46 @@ struct GemmParams {
   int nbp4;            // ceil(K/32 / 4): scale chunks per 128-row group
   int out_f32;         // 1: fp32 output, 0: bf16
   int vec_ok;          // rows of Y are 16-byte aligned for vector stores
+  int tma_store;       // bf16 output written through the staged TMA store
 };
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int32_t x,
+                                             int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void epi_bar_sync() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
+}
+// Barrier over the four epilogue warps that also ANDs a flag across them, so that
+// all of them take the same branch after a bounded wait (none is left at a barrier).
+__device__ __forceinline__ bool epi_bar_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 
 __device__ __forceinline__ void store_chunk(const GemmParams& p, int64_t row, int64_t col0,
                                             const uint32_t (&r)[32]) {
@@ -88,14 +132,16 @@ __device__ __forceinline__ void store_chunk(const GemmParams& p, int64_t row, in
 
 __global__ void __launch_bounds__(gemm::kThreads, 1)
     bat_mxf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                         const __grid_constant__ CUtensorMap tmap_b, const GemmParams p) {
+                         const __grid_constant__ CUtensorMap tmap_b,
+                         const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
   using namespace gemm;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t base = (raw_u32 + 1023u) & ~1023u;
   uint8_t* base_ptr = smem_raw + (base - raw_u32);
-  // stage s: [A 16K][B 32K][SFA 1K][SFB 2K]
-  const uint32_t bars = base + kStages * kStageBytes;
+  // stage s: [A 16K][B 32K][SFA 1K][SFB 2K]; then the epilogue staging; then barriers
+  const uint32_t stg = base + kStages * kStageBytes;
+  const uint32_t bars = stg + kEpiBytes;
   auto full_bar = [&](int s) { return bars + 8u * s; };
   auto empty_bar = [&](int s) { return bars + 8u * (kStages + s); };
   const uint32_t tmem_full = bars + 8u * (2 * kStages);
@@ -118,6 +164,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
+    if (p.tma_store) prefetch_tmap(&tmap_y);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -143,12 +190,11 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
         const int64_t mt = tile % m_tiles;
         const int64_t nt = tile / m_tiles;
+        const int ngb = (nt * 2 + 1 < sf_groups_b) ? 2 : 1;  // 128-row scale groups of this W tile
         for (int ks = 0; ks < k_stages; ++ks) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, kErrWaitEmpty)) { ok = false; break; }
           const int c0 = ks * kChunksPerStage;
           const int nch = min(kChunksPerStage, p.nbp4 - c0);
-          int ngb = 0;
-          for (int g = 0; g < kBN / 128; ++g) ngb += (nt * 2 + g < sf_groups_b) ? 1 : 0;
           const uint32_t bytes = kABytes + kBBytes + static_cast<uint32_t>(nch) * kChunk * (1 + ngb);
           const uint32_t sa = base + stage * kStageBytes;
           mbar_expect_tx(full_bar(stage), bytes);
@@ -157,12 +203,9 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
                       static_cast<int32_t>(nt * kBN));
           bulk_load(sa + kABytes + kBBytes, p.sfa + (mt * p.nbp4 + c0) * kChunk, nch * kChunk,
                     full_bar(stage));
-          for (int g = 0; g < kBN / 128; ++g) {
-            const int64_t grp = nt * 2 + g;
-            if (grp < sf_groups_b)
-              bulk_load(sa + kABytes + kBBytes + kSfaBytes + g * (kChunksPerStage * kChunk),
-                        p.sfb + (grp * p.nbp4 + c0) * kChunk, nch * kChunk, full_bar(stage));
-          }
+          for (int g = 0; g < ngb; ++g)
+            bulk_load(sa + kABytes + kBBytes + kSfaBytes + g * (kChunksPerStage * kChunk),
+                      p.sfb + ((nt * 2 + g) * p.nbp4 + c0) * kChunk, nch * kChunk, full_bar(stage));
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
       }
@@ -170,40 +213,60 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      // Descriptors of stage 0; other stages and K sub-blocks only move the start
+      // address field (bits 0-13, in 16-byte units), so a plain add suffices.
+      const uint64_t adesc0 = smem_desc(base, 16, 1024, 2);
+      const uint64_t bdesc0 = smem_desc(base + kABytes, 16, 1024, 2);
+      const uint64_t sfdesc0 = smem_desc(base + kABytes + kBBytes, 0, 128, 0);
+      constexpr uint32_t kStageU = kStageBytes >> 4;
+      constexpr uint32_t kChunkU = kChunk >> 4;
+      constexpr uint32_t kSfbU = kSfaBytes >> 4;
+      constexpr uint32_t kGroupU = (kChunksPerStage * kChunk) >> 4;
+      const uint32_t id_lo = idesc_mxf4(kBM, kBN, 0, 0);  // scale bytes 0-1 of each word
+      const uint32_t id_hi = idesc_mxf4(kBM, kBN, 2, 2);  // scale bytes 2-3
+      const uint32_t t_sfa = tmem_base + kSfaCol;
+      const uint32_t t_sfb = tmem_base + kSfbCol;
       int stage = 0;
       uint32_t phase = 0;
       uint32_t acc_phase = 0;
       for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
         const int64_t nt = tile / m_tiles;
+        const bool g1 = nt * 2 + 1 < sf_groups_b;
         if (!mbar_wait(tmem_empty, acc_phase ^ 1u, kErrWaitTmemEmpty)) { ok = false; break; }
         tc_fence_after();
         for (int ks = 0; ks < k_stages; ++ks) {
           if (!mbar_wait(full_bar(stage), phase, kErrWaitFull)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = base + stage * kStageBytes;
-          const uint32_t sb = sa + kABytes;
-          const uint32_t ssfa = sb + kBBytes;
-          const uint32_t ssfb = ssfa + kSfaBytes;
-          const int c0 = ks * kChunksPerStage;
-          const int nch = min(kChunksPerStage, p.nbp4 - c0);
-          for (int c = 0; c < nch; ++c) {
-            tmem_cp_32x128b_x4(tmem_base + kSfaCol + 4 * c, smem_desc(ssfa + c * kChunk, 0, 128, 0));
-            for (int g = 0; g < kBN / 128; ++g)
-              if (nt * 2 + g < sf_groups_b)
-                tmem_cp_32x128b_x4(tmem_base + kSfbCol + 8 * c + 4 * g,
-                                   smem_desc(ssfb + g * (kChunksPerStage * kChunk) + c * kChunk, 0, 128, 0));
+          const uint64_t so = static_cast<uint64_t>(stage) * kStageU;
+          const int nch = min(kChunksPerStage, p.nbp4 - ks * kChunksPerStage);
+          // scale chunks -> TMEM: A at words [4c, 4c+4), B group g at words [8c + 4g, 8c + 4g + 4)
+          tmem_cp_32x128b_x4(t_sfa, sfdesc0 + so);
+          tmem_cp_32x128b_x4(t_sfb, sfdesc0 + so + kSfbU);
+          if (g1) tmem_cp_32x128b_x4(t_sfb + 4, sfdesc0 + so + kSfbU + kGroupU);
+          if (nch > 1) {
+            tmem_cp_32x128b_x4(t_sfa + 4, sfdesc0 + so + kChunkU);
+            tmem_cp_32x128b_x4(t_sfb + 8, sfdesc0 + so + kSfbU + kChunkU);
+            if (g1) tmem_cp_32x128b_x4(t_sfb + 12, sfdesc0 + so + kSfbU + kGroupU + kChunkU);
           }
           const int64_t krem = p.K - static_cast<int64_t>(ks) * kBK;
-          const int nkb = krem >= 256 ? 4 : static_cast<int>((krem + 63) / 64);
-          for (int kb = 0; kb < nkb; ++kb) {
-            const uint32_t sf_id = (kb & 1) * 2;
-            const uint32_t c = kb >> 1;
-            const uint64_t adesc = smem_desc(sa + kb * 32, 16, 1024, 2);
-            const uint64_t bdesc = smem_desc(sb + kb * 32, 16, 1024, 2);
-            const uint32_t idesc = idesc_mxf4(kBM, kBN, sf_id, sf_id);
-            const uint32_t sfa_addr = (tmem_base + kSfaCol + 4 * c) | (sf_id << 30);
-            const uint32_t sfb_addr = (tmem_base + kSfbCol + 8 * c) | (sf_id << 30);
-            mma_mxf4(tmem_base, adesc, bdesc, idesc, sfa_addr, sfb_addr, (ks | kb) != 0);
+          const uint32_t acc0 = (ks != 0) ? 1u : 0u;
+          if (krem >= kBK) {
+            // four K=64 MMAs; 32 bytes of codes each; scale byte pair 0-1 then 2-3 of each chunk
+            mma_mxf4(tmem_base, adesc0 + so, bdesc0 + so, id_lo, t_sfa, t_sfb, acc0);
+            mma_mxf4(tmem_base, adesc0 + so + 2, bdesc0 + so + 2, id_hi, t_sfa | (2u << 30),
+                     t_sfb | (2u << 30), 1u);
+            mma_mxf4(tmem_base, adesc0 + so + 4, bdesc0 + so + 4, id_lo, t_sfa + 4, t_sfb + 8, 1u);
+            mma_mxf4(tmem_base, adesc0 + so + 6, bdesc0 + so + 6, id_hi, (t_sfa + 4) | (2u << 30),
+                     (t_sfb + 8) | (2u << 30), 1u);
+          } else {
+            const int nkb = static_cast<int>((krem + 63) / 64);
+            for (int kb = 0; kb < nkb; ++kb) {
+              const uint32_t hi = static_cast<uint32_t>(kb & 1);
+              const uint32_t c = static_cast<uint32_t>(kb >> 1);
+              mma_mxf4(tmem_base, adesc0 + so + 2 * kb, bdesc0 + so + 2 * kb, hi ? id_hi : id_lo,
+                       (t_sfa + 4 * c) | (hi << 31), (t_sfb + 8 * c) | (hi << 31),
+                       (acc0 | static_cast<uint32_t>(kb)) != 0 ? 1u : 0u);
+            }
           }
           tc_commit(empty_bar(stage));
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -215,24 +278,68 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int rl = 32 * q + lane;  // row within the tile
+    const bool leader = (warp == 2 && lane == 0);
     uint32_t acc_phase = 0;
     for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
       const int64_t mt = tile % m_tiles;
       const int64_t nt = tile / m_tiles;
-      if (!mbar_wait(tmem_full, acc_phase, kErrWaitTmemFull)) { ok = false; break; }
+      bool got = mbar_wait(tmem_full, acc_phase, kErrWaitTmemFull);
+      if (p.tma_store) got = epi_bar_and(got);
+      if (!got) { ok = false; break; }
       tc_fence_after();
-      const int64_t row = mt * kBM + 32 * q + lane;
-      for (int cc = 0; cc < kBN / 32; ++cc) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + cc * 32, r);
-        tmem_wait_ld();
-        store_chunk(p, row, nt * kBN + cc * 32, r);
+      const uint32_t trow = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+      if (p.tma_store) {
+        // 1) drain the accumulator into registers as bf16 pairs and release TMEM at once
+        uint32_t h[kBN / 2];
+#pragma unroll
+        for (int cc = 0; cc < kBN / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(trow + cc * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1]));
+            h[cc * 16 + c] = *reinterpret_cast<uint32_t*>(&v);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tmem_empty);  // accumulator free: next tile's MMAs may start
+        // 2) stream 64-column slices through the staging box; 16-byte chunk j of row rl
+        //    sits at chunk (j ^ (rl % 8)) (the 128-byte swizzle of the store's tensor map)
+        const uint32_t rowb = stg + rl * 128;
+#pragma unroll
+        for (int b = 0; b < kBN / 64; ++b) {
+          if (leader) bulk_wait_read0();  // the previous slice has left the box
+          epi_bar_sync();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(rowb + ((j ^ (rl & 7)) << 4), h[b * 32 + 4 * j], h[b * 32 + 4 * j + 1],
+                         h[b * 32 + 4 * j + 2], h[b * 32 + 4 * j + 3]);
+          fence_async_smem();
+          epi_bar_sync();
+          const int64_t col = nt * kBN + 64 * b;
+          if (leader && col < p.N) {
+            tma_store_2d(&tmap_y, stg, static_cast<int32_t>(col), static_cast<int32_t>(mt * kBM));
+            bulk_commit();
+          }
+        }
+      } else {
+        const int64_t row = mt * kBM + rl;
+        for (int cc = 0; cc < kBN / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(trow + cc * 32, r);
+          tmem_wait_ld();
+          store_chunk(p, row, nt * kBN + cc * 32, r);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tmem_empty);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tmem_empty);
       acc_phase ^= 1u;
     }
+    if (leader) bulk_wait0();
   }
 
   tc_fence_before();
