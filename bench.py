@@ -45,6 +45,24 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu record, if it still describes
+    the current kernel source (hash match) and this workload; else None."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)[kernel]
+        h = hashlib.sha256()
+        for fn in rec["files"]:
+            with open(os.path.join(ROOT, fn), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest()[:16] != rec["source_sha256_16"] or rec["workload"] != workload:
+            return None
+        return int(rec["traffic_bytes"])
+    except Exception:
+        return None
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -133,18 +151,21 @@ def oracle_sample(inp, w, budget_s: float, seed: int = 0):
         return time.perf_counter() - t0
 
     cols = np.arange(w.N)
-    t1 = run(rng.integers(0, w.M, size=1), cols)
-    nrows = int(max(1, min(w.M, budget_s / max(t1, 1e-6))))
+    run(rng.integers(0, w.M, size=1), cols)  # first call: page in the dequantized weights
+    t1 = run(rng.integers(0, w.M, size=4), cols) / 4
     ncols = w.N
+    per = int(max(1, min(w.M, 0.5 * budget_s / max(t1, 1e-6) / 4)))  # rows per timed batch
     if t1 > budget_s:  # a single full row is already over budget: sample columns too
-        nrows = 1
-        ncols = int(max(1, w.N * budget_s / t1))
-    rows = rng.choice(w.M, size=nrows, replace=False)
-    cols = np.sort(rng.choice(w.N, size=ncols, replace=False))
-    dt = run(rows, cols)
+        per, ncols = 1, int(max(1, w.N * budget_s / t1))
+    sel = np.sort(rng.choice(w.N, size=ncols, replace=False))
+    dt, nrows = 0.0, 0
+    while dt < budget_s and nrows < w.M:  # repeat batches until the time budget is used
+        rows = rng.choice(w.M, size=per, replace=False)
+        dt += run(rows, sel)
+        nrows += per
     flops = 2.0 * nrows * ncols * w.K
     desc = (f"{nrows} random token rows x {ncols} weight rows of {w.name} "
-            f"(K={w.K}): transform+clip+quantize, dequantize, fp64 dot products")
+            f"(K={w.K}) in batches of {per}: transform+clip+quantize, dequantize, fp64 dot products")
     return flops / dt, dt, desc, oracle.num_threads()
 
 
@@ -260,8 +281,15 @@ def main():
         bat.bat_quantize_act(X, A, B, gl, gh, Xq=Xq, stream=stream)
         bat.bat_mxfp4_gemm(Xq, Wq, Y=Y, out_dtype=torch.bfloat16, stream=stream)
 
-    for _ in range(args.warmup):
-        flush.fill_(1)
+    def flush_l2(i):
+        # write, then read, a buffer twice the L2: the next kernel starts with a cold L2
+        # holding only clean lines of unrelated data (no write-back lands on it)
+        flush.fill_(i & 0xFF)
+        flush_view.sum(dtype=torch.int64)
+
+    flush_view = flush.view(torch.int32)
+    for i in range(args.warmup):
+        flush_l2(i)
         step()
     torch.cuda.synchronize()
 
@@ -274,7 +302,7 @@ def main():
         pg.barrier()
     torch.cuda.synchronize()
     for i in range(K_):
-        flush.fill_(i & 0xFF)  # evict L2 between steps (outside the timed events)
+        flush_l2(i)  # evict L2 between steps (outside the timed events)
         ev[i][0].record(stream)
         bat.bat_quantize_act(X, A, B, gl, gh, Xq=Xq, stream=stream)
         ev[i][1].record(stream)
@@ -349,16 +377,18 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "mxfp4", "data": "synthetic",
             "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "out": "bf16",
-                       "l2": "flushed between steps (256 MiB write outside the timed events)",
+                       "l2": "flushed between steps (256 MiB write + read outside the timed events)",
                        "parallelism": f"replicas x{world} (independent token batches)"},
             "gpu_launches": 2 * K_ * world,
             "roofline": {"bound": "tensor", "achieved": gemm_tf, "peak": fp4_peak,
-                         "unit": "TFLOP/s", "frac": gemm_tf / fp4_peak, "traffic": None,
+                         "unit": "TFLOP/s", "frac": gemm_tf / fp4_peak,
+                         "traffic": recorded_traffic("bat_mxf4_gemm_kernel", w.name),
                          "kernel": "bat_mxf4_gemm_kernel",
                          "peak_source": f"{peak_src} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/BF16)"},
             "prologue": {"bound": "hbm", "achieved": pro_gbs, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": pro_gbs / peaks["hbm_gbs"],
-                         "us_per_launch": 1e6 * sp / K_, "traffic": None,
+                         "us_per_launch": 1e6 * sp / K_,
+                         "traffic": recorded_traffic("bat_prologue_kernel", w.name),
                          "kernel": "bat_prologue_kernel", "peak_source": peak_src},
             "gemm_us_per_launch": 1e6 * sg / K_,
             "prepare_weight_ms": prep_ms,

@@ -212,6 +212,12 @@ BAT_API bat_status_t bat_linear_noalloc(const void* X, int64_t M, const bat_mxfp
                                         void* stream);
 
 /*
+ * Text of the last CUDA error that made a call on this host thread return
+ * BAT_ERR_CUDA ("no CUDA error" if none). Static storage; per thread.
+ */
+BAT_API const char* bat_last_cuda_error(void);
+
+/*
  * Reads and clears the sticky device error word the kernels set when a bounded
  * wait runs out (a pipeline stall that should never happen). Returns 0 if no
  * kernel reported a failure since the last call; synchronizes the device.

@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
         "bat_linear": (S, [P, I64, SP, P, P, P, P, P, S, P, ctypes.c_size_t, P]),
         "bat_linear_noalloc": (S, [P, I64, SP, P, P, P, P, P, S, P]),
         "bat_device_error": (S, []),
+        "bat_last_cuda_error": (ctypes.c_char_p, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -112,7 +113,10 @@ def _need(t: torch.Tensor, dtype: torch.dtype, name: str, shape=None) -> torch.T
 
 def _check(status: int, where: str) -> None:
     if status != 0:
-        raise BatError(status, where)
+        err = BatError(status, where)
+        if status == 5:  # BAT_ERR_CUDA: attach the CUDA error text
+            err.args = (f"{err.args[0]} ({lib().bat_last_cuda_error().decode()})",)
+        raise err
 
 
 @dataclass

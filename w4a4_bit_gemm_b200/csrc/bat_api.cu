@@ -57,7 +57,13 @@ bat_status_t current_device(int* dev_out, int* sms_out) {
   return BAT_OK;
 }
 
-bat_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? BAT_OK : BAT_ERR_CUDA; }
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+bat_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return BAT_OK;
+  t_last_cuda_error = e;
+  return BAT_ERR_CUDA;
+}
 
 // ---------------------------------------------------------------- tensor maps
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -255,9 +261,10 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
   if (p.tma_store && !make_out_map(&ty, Y, p.M, p.N)) return BAT_ERR_CUDA;
   DeviceInfo& d = g_dev[dev];
   if (!d.gemm_attr.load()) {
-    if (cudaFuncSetAttribute(bat::bat_mxf4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             bat::gemm::kSmemBytes) != cudaSuccess)
-      return BAT_ERR_CUDA;
+    const cudaError_t ae = cudaFuncSetAttribute(bat::bat_mxf4_gemm_kernel,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                bat::gemm::kSmemBytes);
+    if (ae != cudaSuccess) return cuda_status(ae);
     d.gemm_attr.store(1);
   }
   const int64_t tiles = ((p.M + bat::gemm::kBM - 1) / bat::gemm::kBM) *
@@ -438,6 +445,10 @@ bat_status_t bat_linear(const void* X, int64_t M, const bat_mxfp4_t* Wq, const f
   st = launch_prologue(X, M, K, A, B, g_lo, g_hi, false, &xq, nullptr, s);
   if (st != BAT_OK) return st;
   return launch_gemm(&xq, Wq, Y, out_dtype, s);
+}
+
+const char* bat_last_cuda_error(void) {
+  return t_last_cuda_error == cudaSuccess ? "no CUDA error" : cudaGetErrorString(t_last_cuda_error);
 }
 
 int bat_device_error(void) {

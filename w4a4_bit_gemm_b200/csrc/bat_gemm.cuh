@@ -2,16 +2,22 @@
 // elements along K, the low-bit product Q(XP) . Q(P^-1 W^T) of the BATQuant
 // linear layer (BATQuant note, en.papernotes.org, Method > Key Designs 1).
 //
-// One persistent CTA per SM walks 128 x 256 output tiles. Warp roles:
-//   warp 0      TMA producer: code tiles through 2-D tensor maps (128-byte
+// One persistent CTA per SM walks 128 x 256 output tiles. Warp roles (three
+// warpgroups; registers are moved to the epilogue with setmaxnreg):
+//   warps 0..3  epilogue: tcgen05.ld of the fp32 accumulator, conversion,
+//               staged TMA stores of Y (holds a whole bf16 tile row in registers);
+//   warps 4..7  scale-factor writers, one per TMEM lane quarter: each stage's
+//               scale chunks go shared -> registers -> TMEM (tcgen05.st) into a
+//               per-stage TMEM buffer, in the layout the block-scaled MMA reads
+//               (each 128-row chunk replicated over the four lane quarters).
+//               Writing them from registers keeps the copies off the tensor
+//               pipe, where tcgen05.cp would queue behind the MMAs;
+//   warp 8      TMA producer: code tiles through 2-D tensor maps (128-byte
 //               swizzle), scale tiles through 1-D bulk copies, into a ring of
 //               kStages shared-memory stages guarded by mbarriers;
-//   warp 1      TMEM owner and MMA issuer: copies each stage's scale factors
-//               shared -> TMEM (tcgen05.cp, replicated over the four lane
-//               quarters) and issues tcgen05.mma kind::mxf4.block_scale
+//   warp 9      TMEM owner and MMA issuer: tcgen05.mma kind::mxf4.block_scale
 //               (M=128, N=256, K=64) accumulating in TMEM;
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator, conversion,
-//               stores of Y.
+//   warps 10,11 idle (they complete the third warpgroup).
 // Every wait is bounded (see mbar_wait) and reports through the error word.
 #pragma once
 
@@ -31,17 +37,21 @@ constexpr int kChunksPerStage = kBK / 128;   // 2
 constexpr int kSfaBytes = (kBM / 128) * kChunksPerStage * kChunk;  // 1 KB
 constexpr int kSfbBytes = (kBN / 128) * kChunksPerStage * kChunk;  // 2 KB
 constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;
+constexpr uint32_t kRegsEpi = 248;   // after setmaxnreg: 128 x 248 + 256 x 56 <= 384 x 168
+constexpr uint32_t kRegsOther = 56;
 // bf16 output staging for the TMA store: one box of 128 rows x 64 columns (128 bytes,
 // 128-byte swizzle); the epilogue holds its whole bf16 tile in registers and
 // streams it through this box one 64-column slice at a time.
 constexpr int kEpiBoxBytes = kBM * 128;
 constexpr int kEpiBytes = kEpiBoxBytes;  // 16 KB
 constexpr int kSmemBytes = kStages * kStageBytes + kEpiBytes + 1024 /*align*/ + 256 /*barriers*/;
-// TMEM columns: accumulator [0, 256), A scales [256, 264), B scales [264, 280).
+// TMEM columns: accumulator [0, 256); stage s's scales at 256 + 24 s: A words
+// [0, 8) (two 128-K chunks x 4), B words [8, 24) (two chunks x two 128-row groups x 4).
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSfaCol = 256;
-constexpr uint32_t kSfbCol = 264;
+constexpr uint32_t kSfCol0 = 256;
+constexpr uint32_t kSfStageCols = 24;
+static_assert(kSfCol0 + kStages * kSfStageCols <= kTmemCols, "TMEM columns");
 }  // namespace gemm
 
 struct GemmParams {
@@ -55,6 +65,13 @@ struct GemmParams {
   int tma_store;       // bf16 output written through the staged TMA store
 };
 
+__device__ __forceinline__ uint4 lds_v4_u32(uint32_t addr) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(addr));
+  return r;
+}
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
@@ -147,6 +164,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   const uint32_t tmem_full = bars + 8u * (2 * kStages);
   const uint32_t tmem_empty = tmem_full + 8u;
   const uint32_t tmem_slot = tmem_empty + 8u;
+  auto sf_bar = [&](int s) { return tmem_slot + 8u + 8u * s; };  // scales of stage s in TMEM
   volatile uint32_t* tmem_slot_ptr =
       reinterpret_cast<volatile uint32_t*>(base_ptr + (tmem_slot - base));
 
@@ -160,13 +178,14 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     }
     mbar_init(tmem_full, 1);
     mbar_init(tmem_empty, 4);
+    for (int s = 0; s < kStages; ++s) mbar_init(sf_bar(s), 4);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
     if (p.tma_store) prefetch_tmap(&tmap_y);
   }
-  if (warp == 1) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -182,7 +201,10 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   const int64_t sf_groups_b = (p.N + 127) / 128;
   bool ok = true;
 
-  if (warp == 0) {
+  if (warp >= 8) {
+    setmaxnreg_dec<kRegsOther>();  // warpgroup 2: producer, MMA issuer, two idle warps
+  }
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int stage = 0;
@@ -210,44 +232,29 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       // Descriptors of stage 0; other stages and K sub-blocks only move the start
       // address field (bits 0-13, in 16-byte units), so a plain add suffices.
       const uint64_t adesc0 = smem_desc(base, 16, 1024, 2);
       const uint64_t bdesc0 = smem_desc(base + kABytes, 16, 1024, 2);
-      const uint64_t sfdesc0 = smem_desc(base + kABytes + kBBytes, 0, 128, 0);
       constexpr uint32_t kStageU = kStageBytes >> 4;
-      constexpr uint32_t kChunkU = kChunk >> 4;
-      constexpr uint32_t kSfbU = kSfaBytes >> 4;
-      constexpr uint32_t kGroupU = (kChunksPerStage * kChunk) >> 4;
       const uint32_t id_lo = idesc_mxf4(kBM, kBN, 0, 0);  // scale bytes 0-1 of each word
       const uint32_t id_hi = idesc_mxf4(kBM, kBN, 2, 2);  // scale bytes 2-3
-      const uint32_t t_sfa = tmem_base + kSfaCol;
-      const uint32_t t_sfb = tmem_base + kSfbCol;
       int stage = 0;
       uint32_t phase = 0;
       uint32_t acc_phase = 0;
       for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-        const int64_t nt = tile / m_tiles;
-        const bool g1 = nt * 2 + 1 < sf_groups_b;
         if (!mbar_wait(tmem_empty, acc_phase ^ 1u, kErrWaitTmemEmpty)) { ok = false; break; }
         tc_fence_after();
         for (int ks = 0; ks < k_stages; ++ks) {
-          if (!mbar_wait(full_bar(stage), phase, kErrWaitFull)) { ok = false; break; }
+          if (!mbar_wait(full_bar(stage), phase, kErrWaitFull) ||
+              !mbar_wait(sf_bar(stage), phase, kErrWaitFull)) { ok = false; break; }
           tc_fence_after();
           const uint64_t so = static_cast<uint64_t>(stage) * kStageU;
-          const int nch = min(kChunksPerStage, p.nbp4 - ks * kChunksPerStage);
-          // scale chunks -> TMEM: A at words [4c, 4c+4), B group g at words [8c + 4g, 8c + 4g + 4)
-          tmem_cp_32x128b_x4(t_sfa, sfdesc0 + so);
-          tmem_cp_32x128b_x4(t_sfb, sfdesc0 + so + kSfbU);
-          if (g1) tmem_cp_32x128b_x4(t_sfb + 4, sfdesc0 + so + kSfbU + kGroupU);
-          if (nch > 1) {
-            tmem_cp_32x128b_x4(t_sfa + 4, sfdesc0 + so + kChunkU);
-            tmem_cp_32x128b_x4(t_sfb + 8, sfdesc0 + so + kSfbU + kChunkU);
-            if (g1) tmem_cp_32x128b_x4(t_sfb + 12, sfdesc0 + so + kSfbU + kGroupU + kChunkU);
-          }
+          const uint32_t t_sfa = tmem_base + kSfCol0 + kSfStageCols * stage;
+          const uint32_t t_sfb = t_sfa + 8;
           const int64_t krem = p.K - static_cast<int64_t>(ks) * kBK;
           const uint32_t acc0 = (ks != 0) ? 1u : 0u;
           if (krem >= kBK) {
@@ -275,11 +282,50 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         acc_phase ^= 1u;
       }
     }
-  } else {
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ scale-factor writers
+    setmaxnreg_dec<kRegsOther>();
+    // Warp w writes TMEM lane quarter q = w % 4. Lane l of it holds TMEM lane 32q + l,
+    // which takes 16-byte row l of every 512-byte chunk (the scales of rows l, l+32,
+    // l+64, l+96 of that chunk's 128-row group) at the chunk's four words.
+    const int q = warp & 3;
+    const uint32_t tlane = static_cast<uint32_t>(32 * q) << 16;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+      for (int ks = 0; ks < k_stages; ++ks) {
+        if (!mbar_wait(full_bar(stage), phase, kErrWaitFull)) { ok = false; break; }
+        const uint32_t ssf = base + stage * kStageBytes + kABytes + kBBytes + lane * 16;
+        uint32_t fa[8], fb[16];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uint4 v = lds_v4_u32(ssf + c * kChunk);
+          fa[4 * c] = v.x; fa[4 * c + 1] = v.y; fa[4 * c + 2] = v.z; fa[4 * c + 3] = v.w;
+        }
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            const uint4 v = lds_v4_u32(ssf + kSfaBytes + g * (kChunksPerStage * kChunk) + c * kChunk);
+            const int w = 8 * c + 4 * g;
+            fb[w] = v.x; fb[w + 1] = v.y; fb[w + 2] = v.z; fb[w + 3] = v.w;
+          }
+        const uint32_t tcol = tmem_base + tlane + kSfCol0 + kSfStageCols * stage;
+        tmem_st_32x32b_x8(tcol, fa);
+        tmem_st_32x32b_x16(tcol + 8, fb);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sf_bar(stage));
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else if (warp < 4) {
     // ------------------------------------------------------------ epilogue
+    setmaxnreg_inc<kRegsEpi>();
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int rl = 32 * q + lane;  // row within the tile
-    const bool leader = (warp == 2 && lane == 0);
+    const bool leader = (warp == 0 && lane == 0);
     uint32_t acc_phase = 0;
     for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
       const int64_t mt = tile % m_tiles;
@@ -345,7 +391,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+  if (warp == 9) tmem_dealloc(tmem_base, kTmemCols);
 }
 
 }  // namespace bat
