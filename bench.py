@@ -63,6 +63,35 @@ def recorded_traffic(kernel: str, workload: str):
         return None
 
 
+def max_over_ranks(dist_mod, values, device):
+    """Element-wise max of per-rank timings (every rank gets the result)."""
+    import torch
+    if dist_mod is None:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(units_per_step: float, steps: int, world: int, seconds: float) -> float:
+    """Whole-job rate: the units every rank processed over the slowest rank's time."""
+    return units_per_step * steps * world / seconds
+
+
+def rank_batch_seed(rank: int) -> int:
+    """Token batch of rank r: seed r (rank 0 uses the workload's own seed 0)."""
+    return rank
+
+
+def rank_inputs(name: str, rank: int):
+    """The workload for one rank: weights, factors and clip logits from seed 0 (shared
+    by every rank), the token batch X from the rank's own seed."""
+    inp = wl.make_inputs(name, seed=0)
+    seed = rank_batch_seed(rank)
+    x = inp.X if seed == 0 else wl.make_inputs(name, seed=seed, with_weight=False).X
+    return inp, x
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -178,14 +207,17 @@ def run_reference(args, w, inp):
     Wd = oracle.dequantize(wc, ws)
     rng = np.random.default_rng(1)
 
+    nrows = max(1, min(w.M, oracle.num_threads()))  # one token row per oracle thread
+
     def step(ncols):
-        rows = rng.integers(0, w.M, size=1)
+        rows = rng.choice(w.M, size=nrows, replace=False)
         cols = np.sort(rng.choice(w.N, size=ncols, replace=False))
         t0 = time.perf_counter()
         _, xc, xs = oracle.quantize_act(inp.X[rows], inp.A, inp.B, inp.g_lo, inp.g_hi)
         oracle.gemm_sampled(oracle.dequantize(xc, xs), Wd, None, cols)
         return time.perf_counter() - t0
 
+    step(w.N)  # page in the dequantized weights
     t_full = step(w.N)
     ncols = int(max(1, min(w.N, w.N * per_step / max(t_full, 1e-6))))
     for _ in range(warm):
@@ -193,9 +225,9 @@ def run_reference(args, w, inp):
     total = 0.0
     for _ in range(steps):
         total += step(ncols)
-    flops = 2.0 * ncols * w.K * steps
+    flops = 2.0 * nrows * ncols * w.K * steps
     value = flops / total / 1e12
-    desc = f"per step: 1 random token row x {ncols} weight rows of {w.name} (K={w.K})"
+    desc = f"per step: {nrows} random token rows x {ncols} weight rows of {w.name} (K={w.K})"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": steps, "warmup": warm,
@@ -250,8 +282,7 @@ def main():
         pg = dist
 
     # rank r draws its own token batch; weights and transform factors are shared
-    inp = wl.make_inputs(w.name, seed=0)
-    X_host = inp.X if rank == 0 else wl.make_inputs(w.name, seed=rank, with_weight=False).X
+    inp, X_host = rank_inputs(w.name, rank)
 
     def bf16(bits):
         return torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(dev)
@@ -314,17 +345,11 @@ def main():
     clocks = sampler.stop() if (not args.no_clocks and rank == 0) else None
     t_pro = [ev[i][0].elapsed_time(ev[i][1]) * 1e-3 for i in range(K_)]
     t_gemm = [ev[i][1].elapsed_time(ev[i][2]) * 1e-3 for i in range(K_)]
-    t_step = sum(t_pro) + sum(t_gemm)
-    if pg:
-        t = torch.tensor([t_step, sum(t_pro), sum(t_gemm)], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        t_step, sp, sg = t.tolist()
-    else:
-        sp, sg = sum(t_pro), sum(t_gemm)
+    t_step, sp, sg = max_over_ranks(pg, [sum(t_pro) + sum(t_gemm), sum(t_pro), sum(t_gemm)], dev)
     assert bat.bat_device_error() == 0, "a kernel reported a stalled wait"
 
     flop = 2.0 * w.M * w.N * w.K
-    value = flop * K_ * world / t_step / 1e12
+    value = job_throughput(flop, K_, world, t_step) / 1e12
     peaks, peak_src = load_peaks()
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
     gemm_tf = flop / (sg / K_) / 1e12
@@ -356,12 +381,8 @@ def main():
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        te = e0.elapsed_time(e1) * 1e-3
-        if pg:
-            t = torch.tensor([te], dtype=torch.float64, device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            te = t.item()
-        e2e = {"value": flop * args.e2e_steps * world / te / 1e12, "unit": "TFLOP/s",
+        te = max_over_ranks(pg, [e0.elapsed_time(e1) * 1e-3], dev)[0]
+        e2e = {"value": job_throughput(flop, args.e2e_steps, world, te) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(X.numel() * 2), "d2h_bytes_per_step": int(Y.numel() * 2)}
 
     cpu = None
