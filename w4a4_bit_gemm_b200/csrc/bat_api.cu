@@ -31,7 +31,6 @@ struct DeviceInfo {
   std::atomic<int> sms{0};
   std::atomic<int> gemm_attr{0};
   std::atomic<int> pro_attr{0};     // bit t: the prologue variant t has its smem attribute set
-  std::atomic<int> pro_per_sm{0};   // resident prologue CTAs per SM
 };
 DeviceInfo g_dev[64];
 
@@ -116,6 +115,21 @@ bool make_out_map(CUtensorMap* map, void* y, int64_t M, int64_t N) {
   return r == CUDA_SUCCESS;
 }
 
+// bf16 X [rows][K] for the prologue: box of 64 columns (128 bytes) x 128 rows, 128-byte
+// swizzle (the K-major A-operand layout of the transform MMA); rows past the end read 0.
+bool make_act_map(CUtensorMap* map, const void* x, int64_t rows, int64_t K) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K * 2)};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(bat::pro::kTok)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = f(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box,
+                 estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------- fp64 inverse (host)
 // Gauss-Jordan elimination with partial pivoting on an n x n row-major matrix.
 // Returns false if a pivot vanishes or the 1-norm condition number exceeds kMaxCond.
@@ -188,8 +202,10 @@ bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float
   int dev = 0, sms = 0;
   bat_status_t st = current_device(&dev, &sms);
   if (st != BAT_OK) return st;
+  if (rows >= (int64_t{1} << 31)) return BAT_ERR_SHAPE;  // TMA row coordinates are int32
+  CUtensorMap tx;
+  if (!make_act_map(&tx, X, rows, K)) return BAT_ERR_CUDA;
   bat::PrologueParams p;
-  p.x = static_cast<const uint16_t*>(X);
   p.a = A;
   p.b = B;
   p.g_lo = g_lo;
@@ -200,9 +216,11 @@ bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float
   p.rows = rows;
   p.K = K;
   p.nb = static_cast<int>(K / 32);
-  p.nseg = (p.nb + 31) / 32;
+  p.nbp2 = (p.nb + 1) / 2;
   p.nbp4 = (p.nb + 3) / 4;
-  void (*kern)(bat::PrologueParams);
+  p.mtiles = (rows + bat::pro::kTok - 1) / bat::pro::kTok;
+  p.units = p.mtiles * p.nbp2;
+  void (*kern)(CUtensorMap, bat::PrologueParams);
   if (per_row)
     kern = y_out ? bat::bat_prologue_kernel<true, true> : bat::bat_prologue_kernel<false, true>;
   else
@@ -215,25 +233,9 @@ bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float
       return BAT_ERR_CUDA;
     d.pro_attr.fetch_or(variant_bit);
   }
-  int per_sm = d.pro_per_sm.load();
-  if (per_sm == 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bat::bat_prologue_kernel<false, false>,
-                                                      bat::pro::kThreads, bat::pro::kSmemBytes) != cudaSuccess)
-      return BAT_ERR_CUDA;
-    per_sm = per_sm < 1 ? 1 : per_sm;
-    d.pro_per_sm.store(per_sm);
-  }
-  // One CTA per (segment of 32 blocks, range of rows); about one CTA per SM slot.
-  const int64_t slots = static_cast<int64_t>(sms) * per_sm;
-  const int64_t max_parts = (rows + bat::pro::kRowsPerStage - 1) / bat::pro::kRowsPerStage;
-  int64_t parts = slots / p.nseg;
-  if (parts > max_parts) parts = max_parts;
-  if (parts < 1) parts = 1;
-  p.rows_per_cta = (rows + parts - 1) / parts;
-  parts = (rows + p.rows_per_cta - 1) / p.rows_per_cta;
-  const int64_t grid = parts * p.nseg;
-  if (grid > 0x7FFFFFFF) return BAT_ERR_SHAPE;
-  kern<<<static_cast<unsigned>(grid), bat::pro::kThreads, bat::pro::kSmemBytes, stream>>>(p);
+  // One CTA per SM, each over a contiguous range of (block pair, token tile) units.
+  const int64_t grid = p.units < sms ? p.units : sms;
+  kern<<<static_cast<unsigned>(grid), bat::pro::kThreads, bat::pro::kSmemBytes, stream>>>(tx, p);
   return cuda_status(cudaGetLastError());
 }
 

@@ -1,27 +1,38 @@
 // Fused prologue: GPK block transform + block-wise clipping + MXFP4 quantize/pack.
 //
 // BATQuant note (en.papernotes.org), Method > Key Designs 2 and 3: each
-// 32-channel block x (a row-major 4x8 matrix X_r) becomes
-// y = vec_row(B_b^T X_r A) — two small matrix products instead of the explicit
-// 32x32 block B_b (x) A — then is clipped to [r_lo*min(y), r_hi*max(y)] and
-// quantized to E2M1 codes with one UE8M0 scale 2^e, e = floor(log2 amax) - 2.
+// 32-channel block x of a token becomes y = x (B_b (x) A) = vec_row(B_b^T X_r A),
+// then is clipped to [r_lo*min(y), r_hi*max(y)] and quantized to E2M1 codes with
+// one UE8M0 scale 2^e, e = floor(log2 amax) - 2.
 //
-// Work mapping. X is cut into segments of 32 consecutive blocks (1024 columns,
-// 2 KB of bf16 per row). A CTA owns one segment and a range of rows. One
-// producer warp streams the CTA's rows into a ring of shared-memory stages
-// with bulk copies (16 rows x 2 KB per stage); each of 16 consumer warps takes
-// one row of a stage.
-//  1. T = X_r A for all 128 rows of 8 of the segment (the shared factor is the
-//     same for every block) runs on the tensor cores: ldmatrix feeds the 16-byte
-//     rows straight from the stage to mma.sync (bf16 inputs, fp32 accumulate).
-//     x is exact in bf16; A is split into three bf16 terms A_hi + A_mid + A_lo
-//     (residual ~2^-24 |A|), so T matches an fp32 product to within fp32 rounding.
-//  2. The 16x8 accumulator fragments go to a per-warp shared buffer, swizzled
-//     so that lane b then reads block b's 4x8 T with conflict-free 16-byte loads.
-//  3. Per lane (= block): Y = B_b^T T on packed fp32x2 FMAs (B_b as broadcast
-//     pairs in registers), block min/max by 3-input min/max trees, clip bounds,
-//     scale and E2M1 codes in registers; 16 bytes of codes per lane (a warp
-//     writes 512 contiguous bytes) and one scale byte in the GEMM's tiled order.
+// All tokens share the 32x32 matrix P_b = B_b (x) A of block column b, so the
+// transform of 128 tokens is one dense product X_b (128x32) . P_b (32x32): a
+// 5th-generation tensor-core MMA (tcgen05, kind::f16, bf16 operands, fp32
+// accumulators in TMEM). x is exact in bf16; P_b (each entry the fp32 product
+// B_b[i][j] * A[p][q]) is split into three bf16 terms P_hi + P_mid + P_lo
+// (residual ~2^-24 |P_b|). The three terms sit side by side as one N=96 operand,
+// so one MMA per 16-wide K-step reads the X tile once and yields the three
+// partial products, which the quantizer adds in fp32: y matches an fp32 product
+// to within fp32 rounding. The accumulator puts token m in TMEM lane m, so a
+// thread holds the whole 32-element block of one token: block min/max, clip,
+// scale and E2M1 codes need no exchange between threads.
+//
+// Work unit: 128 tokens x one pair of blocks (a 128-row x 128-byte box of X).
+//   warp 0      producer: TMA copies of the units' boxes into a ring of kStages
+//               shared-memory stages (lane 0), and, with all 32 lanes, the P
+//               terms of each new block pair before its first copy;
+//   warp 1      TMEM owner and MMA issuer: per unit, two blocks x two K-steps of
+//               M=128, N=96, K=16 into one of two 192-column accumulators;
+//   warps 2-17  two quantizer sets of eight warps; set s takes the units whose
+//               index within the CTA is s mod 2, warp (s, j, q) block j of the
+//               pair for the 32 tokens of TMEM lane quarter q.
+// The issuer waits once per unit for its copy and once for its accumulator, so
+// its chain of waits, MMAs and commits stays well inside the copy's time, and
+// each quantizer set has two units' time for one block.
+// A CTA walks a contiguous range of units ordered by block pair, so it needs the
+// terms of only a few pairs. They sit in two shared-memory buffers (pair i of
+// the CTA's range in buffer i%2); the producer refills a buffer only after the
+// issuer has signalled that the MMAs of the pair that used it have finished.
 #pragma once
 
 #include "bat_common.cuh"
@@ -29,17 +40,24 @@
 namespace bat {
 
 namespace pro {
-constexpr int kRowsPerStage = 16;                // = consumer warps
-constexpr int kStages = 5;
-constexpr int kSegBytes = 32 * kG * 2;           // 2 KB: 32 blocks of 32 bf16
-constexpr int kStageBytes = kRowsPerStage * kSegBytes;
-constexpr int kTBytes = 32 * 32 * 4;             // per-warp fp32 T of one segment: 4 KB
-constexpr int kThreads = 32 * (kRowsPerStage + 1);
-constexpr int kSmemBytes = kStages * kStageBytes + kRowsPerStage * kTBytes + 256;
+constexpr int kTok = 128;                        // tokens per unit (MMA M)
+constexpr int kBlk = 2;                          // 32-element blocks per unit
+constexpr int kStages = 10;
+constexpr int kStageBytes = kTok * 128;          // 128 rows x 64 bf16: 16 KB
+constexpr int kPTermBytes = 32 * 32 * 2;         // one bf16 term of one block's P: 2 KB
+constexpr int kPBlockBytes = 3 * kPTermBytes;    // one block's three terms: 6 KB
+constexpr int kPBytes = kBlk * kPBlockBytes;     // one pair: 12 KB
+constexpr int kSets = 2;                         // quantizer sets (alternate units)
+constexpr int kSetWarps = 4 * kBlk;              // lane quarters x blocks
+constexpr int kThreads = 32 * (2 + kSets * kSetWarps);
+constexpr int kBarBytes = 256;
+constexpr int kSmemBytes = kStages * kStageBytes + 2 * kPBytes + kBarBytes + 1024;
+constexpr int kSlotCols = 96;                    // one block's accumulator: 3 terms x 32 columns
+constexpr uint32_t kAccCols = kBlk * kSlotCols;  // one unit's accumulator: 192 columns
+constexpr uint32_t kTmemCols = 512;              // allocation (power of two) holding 2 x 192
 }  // namespace pro
 
 struct PrologueParams {
-  const uint16_t* x;     // bf16 [rows][K]
   const float* a;        // fp32 [8][8]
   const float* b;        // fp32 [nb][4][4]
   const float* g_lo;     // clip logits: [nb] (shared by rows) or [rows][nb]; may be null
@@ -50,9 +68,10 @@ struct PrologueParams {
   int64_t rows;
   int64_t K;
   int nb;                // K / 32
-  int nseg;              // ceil(nb / 32)
-  int nbp4;              // ceil(nb / 4)
-  int64_t rows_per_cta;  // rows of one segment handled by one CTA
+  int nbp2;              // ceil(nb / 2): block pairs
+  int nbp4;              // ceil(nb / 4): groups of the tiled scale layout
+  int64_t mtiles;        // ceil(rows / 128)
+  int64_t units;         // nbp2 * mtiles, unit u = (pair u / mtiles, token tile u % mtiles)
 };
 
 // fp32(sigma(g)) evaluated in fp64; +inf gives exactly 1.
@@ -65,31 +84,6 @@ __device__ __forceinline__ int64_t scale_offset(int64_t m, int64_t b, int nbp4) 
   return ((m >> 7) * nbp4 + (b >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (b & 3);
 }
 
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                        uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-// D = A(16x16, rows g / g+8) . B(16x8) + C, bf16 inputs, fp32 accumulators.
-__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void mma_1688(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
-      "{%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(b0));
-}
-__device__ __forceinline__ void sts_v2(uint32_t addr, float a, float b) {
-  asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
-}
 __device__ __forceinline__ float min3f(float a, float b, float c) {
   float d;
   asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -105,227 +99,346 @@ __device__ __forceinline__ uint32_t bf16_bits(float v) {
   return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v)));
 }
 
-__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
-  uint4 r;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "r"(addr));
-  return r;
+// Instruction descriptor of kind::f16 with bf16 A and B (both K-major), fp32 accumulation.
+__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
+  return 1u << 4 |                                 // D format: fp32
+         1u << 7 |                                 // A format: bf16
+         1u << 10 |                                // B format: bf16
+         static_cast<uint32_t>(n >> 3) << 17 |     // N / 8
+         static_cast<uint32_t>(m >> 4) << 24;      // M / 16
+}
+// D[tmem] (+)= A x B^T, bf16 operands from shared memory, M=128, K=16.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
+// The three bf16 terms of P_b for block b, in the MMA's B-operand layout (N x K,
+// K-major, no swizzle: 8x8 core matrices of 128 bytes, K-adjacent ones 128 bytes
+// apart, N-adjacent ones 512 bytes apart; the terms follow one another, so the
+// three together are one N=96 operand). Operand element (n, k) is
+// P_b[k][n] = B_b[k/8][n/8] * A[k%8][n%8]; a block past nb gets 0.
+// `row` in [0, 128) picks n = row/4 and the eight k of core-matrix column row%4:
+// one 16-byte row of a core matrix per term.
+__device__ __forceinline__ void build_p_row(uint8_t* dst, const PrologueParams& p, int64_t b,
+                                            int row) {
+  const int n = row >> 2, kc = row & 3;
+  uint32_t w[3][4];
+  const float bv = b < p.nb ? p.b[b * 16 + kc * 4 + (n >> 3)] : 0.0f;  // B_b[k/8][n/8], k/8 = kc
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    uint32_t hh[2], mm[2], ll[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float prod = __fmul_rn(bv, p.a[(i + h) * 8 + (n & 7)]);  // A[k%8][n%8]
+      const uint32_t hi = bf16_bits(prod);
+      const float r1 = prod - __uint_as_float(hi << 16);
+      const uint32_t mid = bf16_bits(r1);
+      hh[h] = hi;
+      mm[h] = mid;
+      ll[h] = bf16_bits(r1 - __uint_as_float(mid << 16));
+    }
+    w[0][i >> 1] = hh[0] | (hh[1] << 16);
+    w[1][i >> 1] = mm[0] | (mm[1] << 16);
+    w[2][i >> 1] = ll[0] | (ll[1] << 16);
+  }
+  const int off = ((n >> 3) * 4 + kc) * 128 + (n & 7) * 16;
+#pragma unroll
+  for (int term = 0; term < 3; ++term)
+    *reinterpret_cast<uint4*>(dst + term * pro::kPTermBytes + off) =
+        make_uint4(w[term][0], w[term][1], w[term][2], w[term][3]);
+}
+
+// Quantize one 32-element block held by this thread: clip to [r_lo*min, r_hi*max],
+// UE8M0 scale, E2M1 codes (16 bytes into `packed`). Returns the scale byte e + 127.
+__device__ __forceinline__ uint32_t quantize_block(const float (&y)[32], float r_lo, float r_hi,
+                                                   uint32_t (&packed)[4]) {
+  float tmn[11], tmx[11];
+#pragma unroll
+  for (int k = 0; k < 10; ++k) {
+    tmn[k] = min3f(y[3 * k], y[3 * k + 1], y[3 * k + 2]);
+    tmx[k] = max3f(y[3 * k], y[3 * k + 1], y[3 * k + 2]);
+  }
+  tmn[10] = fminf(y[30], y[31]);
+  tmx[10] = fmaxf(y[30], y[31]);
+  const float mn = fminf(min3f(min3f(tmn[0], tmn[1], tmn[2]), min3f(tmn[3], tmn[4], tmn[5]),
+                               min3f(tmn[6], tmn[7], tmn[8])),
+                         fminf(tmn[9], tmn[10]));
+  const float mx = fmaxf(max3f(max3f(tmx[0], tmx[1], tmx[2]), max3f(tmx[3], tmx[4], tmx[5]),
+                               max3f(tmx[6], tmx[7], tmx[8])),
+                         fmaxf(tmx[9], tmx[10]));
+  const float lo = __fmul_rn(r_lo, mn);
+  const float hi = __fmul_rn(r_hi, mx);
+  // The clamp is monotone, so the clipped block's extremes are the clipped min/max.
+  const float amax = fmaxf(fabsf(fminf(fmaxf(mn, lo), hi)), fabsf(fminf(fmaxf(mx, lo), hi)));
+  // UE8M0 scale: e = floor(log2 amax) - 2, clamped to >= -127 (amax = 0 -> -127)
+  const int efield = static_cast<int>(__float_as_uint(amax) >> 23);
+  const int sbyte = efield > 2 ? efield - 2 : 0;  // e + 127
+  const float inv_scale = __uint_as_float(static_cast<uint32_t>(254 - sbyte) << 23);  // 2^-e
+  const uint64_t s2 = pack2(inv_scale, inv_scale);
+  // codes: v = c * 2^-e (+0 turns an exact -0 into +0), E2M1 round-to-nearest-even
+  uint32_t byte[16];
+#pragma unroll
+  for (int h = 0; h < 16; ++h) {
+    const float c0 = fminf(fmaxf(y[2 * h], lo), hi);
+    const float c1 = fminf(fmaxf(y[2 * h + 1], lo), hi);
+    float v0, v1;
+    unpack2(ffma2(pack2(c0, c1), s2, 0ull), v0, v1);
+    byte[h] = e2m1x2(v0, v1);
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    packed[c] = (byte[4 * c] | (byte[4 * c + 1] << 8)) | ((byte[4 * c + 2] << 16) | (byte[4 * c + 3] << 24));
+  return static_cast<uint32_t>(sbyte);
+}
+
+// tmap_x: bf16 X [rows][K], box 64 columns x 128 rows, 128-byte swizzle, zero fill.
 // kPerRowClip: clip logits indexed [row][block] (weight side) instead of [block].
 template <bool kTrace, bool kPerRowClip>
-__global__ void __launch_bounds__(pro::kThreads, 1) bat_prologue_kernel(const PrologueParams p) {
+__global__ void __launch_bounds__(pro::kThreads, 1)
+    bat_prologue_kernel(const __grid_constant__ CUtensorMap tmap_x, const PrologueParams p) {
   using namespace pro;
-  extern __shared__ __align__(128) uint8_t smem[];
-  const uint32_t sbase = smem_u32(smem);
-  const uint32_t bars = sbase + kStages * kStageBytes;  // full[s], empty[s]
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  const uint32_t base = (raw_u32 + 1023u) & ~1023u;  // 128-byte swizzle atoms: 1 KB aligned
+  uint8_t* base_ptr = smem_raw + (base - raw_u32);
+  const uint32_t pbase = base + kStages * kStageBytes;  // [buffer][block][term][2 KB]
+  uint8_t* pbase_ptr = base_ptr + kStages * kStageBytes;
+  const uint32_t bars = pbase + 2 * kPBytes;
+  auto full_bar = [&](int s) { return bars + 8u * s; };
+  auto empty_bar = [&](int s) { return bars + 8u * (kStages + s); };
+  auto tfull = [&](int a) { return bars + 8u * (2 * kStages + a); };
+  auto tempty = [&](int a) { return bars + 8u * (2 * kStages + 2 + a); };
+  auto pfull = [&](int buf) { return bars + 8u * (2 * kStages + 4 + buf); };
+  auto pdone = [&](int buf) { return bars + 8u * (2 * kStages + 6 + buf); };
+  const uint32_t done_bar = bars + 8u * (2 * kStages + 8);
+  const uint32_t tmem_slot = done_bar + 8u;
+  volatile uint32_t* tmem_slot_ptr =
+      reinterpret_cast<volatile uint32_t*>(base_ptr + (tmem_slot - base));
 
-  const int seg = static_cast<int>(blockIdx.x % p.nseg);
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x / p.nseg) * p.rows_per_cta;
-  const int64_t row1 = min(p.rows, row0 + p.rows_per_cta);
-  const int nblk = min(32, p.nb - seg * 32);           // blocks in this segment
-  const uint32_t seg_bytes = static_cast<uint32_t>(nblk) * kG * 2;
-  const int nst = row1 > row0 ? static_cast<int>((row1 - row0 + kRowsPerStage - 1) / kRowsPerStage) : 0;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // contiguous unit range of this CTA and the block pairs it spans
+  const int64_t u_begin = p.units * blockIdx.x / gridDim.x;
+  const int64_t u_end = p.units * (blockIdx.x + 1) / gridDim.x;
+  const int64_t pair0 = u_begin / p.mtiles;
+  const int64_t mt0 = u_begin - pair0 * p.mtiles;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(bars + 8 * s, 1);
-      mbar_init(bars + 8 * (kStages + s), kRowsPerStage);
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
     }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull(a), 1);
+      mbar_init(tempty(a), kSetWarps);
+      mbar_init(pfull(a), 32);  // the producer warp's lanes
+      mbar_init(pdone(a), 1);
+    }
+    mbar_init(done_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    prefetch_tmap(&tmap_x);
   }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot_ptr;
 
-  if (warp == kRowsPerStage) {
+  if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      for (int st = 0; st < nst; ++st) {
-        const int slot = st % kStages;
-        const uint32_t par = static_cast<uint32_t>((st / kStages) & 1);
-        if (!mbar_wait(bars + 8 * (kStages + slot), par ^ 1u, kErrWaitEmpty)) break;
-        const int64_t r0 = row0 + static_cast<int64_t>(st) * kRowsPerStage;
-        const int nrows = row1 - r0 < kRowsPerStage ? static_cast<int>(row1 - r0) : kRowsPerStage;
-        mbar_expect_tx(bars + 8 * slot, seg_bytes * nrows);
-        for (int r = 0; r < nrows; ++r)
-          bulk_load(sbase + slot * kStageBytes + r * kSegBytes,
-                    p.x + (r0 + r) * p.K + static_cast<int64_t>(seg) * 1024, seg_bytes, bars + 8 * slot);
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t inflight = 0;  // bit s: stage s was loaded; bit 16+s: parity of that load
+    int64_t pair = pair0, mt = mt0;
+    uint32_t rel = 0;       // pair index within the CTA's range
+    bool ok = true;
+    for (int64_t u = u_begin; u < u_end && ok; ++u) {
+      if (u == u_begin || mt == 0) {
+        // a new pair: its terms go to buffer rel%2 once the pair that used that
+        // buffer (rel-2) has no MMA left in flight
+        if (rel >= 2 && !mbar_wait(pdone(rel & 1u), ((rel - 2) >> 1) & 1u, kErrWaitEmpty)) break;
+        build_p_row(pbase_ptr + (rel & 1u) * kPBytes, p, 2 * pair, lane);
+        build_p_row(pbase_ptr + (rel & 1u) * kPBytes, p, 2 * pair, lane + 32);
+        build_p_row(pbase_ptr + (rel & 1u) * kPBytes, p, 2 * pair, lane + 64);
+        build_p_row(pbase_ptr + (rel & 1u) * kPBytes, p, 2 * pair, lane + 96);
+        build_p_row(pbase_ptr + (rel & 1u) * kPBytes + kPBlockBytes, p, 2 * pair + 1, lane);
+        build_p_row(pbase_ptr + (rel & 1u) * kPBytes + kPBlockBytes, p, 2 * pair + 1, lane + 32);
+        build_p_row(pbase_ptr + (rel & 1u) * kPBytes + kPBlockBytes, p, 2 * pair + 1, lane + 64);
+        build_p_row(pbase_ptr + (rel & 1u) * kPBytes + kPBlockBytes, p, 2 * pair + 1, lane + 96);
+        fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor cores
+        mbar_arrive(pfull(rel & 1u));
       }
+      if (lane == 0) {
+        if (!mbar_wait(empty_bar(stage), phase ^ 1u, kErrWaitEmpty)) {
+          ok = false;
+        } else {
+          mbar_expect_tx(full_bar(stage), kStageBytes);
+          tma_load_2d(base + stage * kStageBytes, &tmap_x, full_bar(stage),
+                      static_cast<int32_t>(pair * 64), static_cast<int32_t>(mt * kTok));
+          inflight = (inflight & ~(0x10001u << stage)) | (1u << stage) | (phase << (16 + stage));
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      if (++mt == p.mtiles) { mt = 0; ++pair; ++rel; }
+    }
+    // no copy may still be writing shared memory when the CTA exits
+    if (lane == 0)
+      for (int s = 0; s < kStages; ++s)
+        if ((inflight >> s) & 1u) mbar_wait(full_bar(s), (inflight >> (16 + s)) & 1u, kErrWaitFull);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(kTok, kSlotCols);
+      // Descriptors differ only in the start-address field (bits 0-13, address / 16).
+      const uint64_t adesc0 = smem_desc(base, 16, 1024, 2);
+      const uint64_t bdesc0 = smem_desc(pbase, 128, 512, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t rel = 0;
+      int64_t mt = mt0;
+      uint32_t n = 0;
+      for (int64_t u = u_begin; u < u_end; ++u, ++n) {
+        if (u == u_begin || mt == 0)
+          if (!mbar_wait(pfull(rel & 1u), (rel >> 1) & 1u, kErrWaitFull)) break;
+        const uint32_t a = n & 1u;
+        if (!mbar_wait(full_bar(stage), phase, kErrWaitFull)) break;
+        if (!mbar_wait(tempty(a), ((n >> 1) & 1u) ^ 1u, kErrWaitTmemEmpty)) break;
+        tc_fence_after();
+        const uint64_t ad = adesc0 + static_cast<uint32_t>(stage * (kStageBytes >> 4));
+        const uint64_t bd = bdesc0 + (rel & 1u) * static_cast<uint32_t>(kPBytes >> 4);
+        const uint32_t d = tmem_base + a * kAccCols;
+#pragma unroll
+        for (int j = 0; j < kBlk; ++j)
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks)
+            // A: block j is the j-th 64 bytes of the box's 128-byte rows, K-step 32 bytes;
+            // B: block j's three terms (96 rows), K-step 256 bytes
+            mma_bf16(d + j * kSlotCols, ad + ((j * 64 + ks * 32) >> 4),
+                     bd + ((j * kPBlockBytes + ks * 256) >> 4), idesc, static_cast<uint32_t>(ks));
+        tc_commit(tfull(a));
+        tc_commit(empty_bar(stage));
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        if (++mt == p.mtiles || u + 1 == u_end) {
+          tc_commit(pdone(rel & 1u));  // this pair's MMAs: its buffer may be refilled
+          mt = 0;
+          ++rel;
+        }
+      }
+      // every MMA issued above has finished before TMEM is released
+      tc_commit(done_bar);
+      mbar_wait(done_bar, 0, kErrWaitTmemFull);
     }
   } else {
-    // ------------------------------------------------------------ consumers
-    const int b = seg * 32 + lane;
-    const bool active = lane < nblk;
-    const int g = lane >> 2;  // mma fragment coordinates
-    const int t4 = lane & 3;
-    // Shared factor for the tensor-core stage: B-operand fragments of A split into
-    // three bf16 terms. Fragment (k = 2*t4 + {0,1}, n = g): A[2*t4 + {0,1}][g].
-    uint32_t fa_hm0, fa_hm1, fa_lo;
-    {
-      const float v0 = p.a[(2 * t4) * 8 + g], v1 = p.a[(2 * t4 + 1) * 8 + g];
-      const uint32_t h0 = bf16_bits(v0), h1 = bf16_bits(v1);
-      const float r0 = v0 - __uint_as_float(h0 << 16), r1 = v1 - __uint_as_float(h1 << 16);
-      const uint32_t m0 = bf16_bits(r0), m1 = bf16_bits(r1);
-      const float s0 = r0 - __uint_as_float(m0 << 16), s1 = r1 - __uint_as_float(m1 << 16);
-      fa_hm0 = h0 | (h1 << 16);                    // k 0-7 of the k16 MMA: A_hi
-      fa_hm1 = m0 | (m1 << 16);                    // k 8-15: A_mid
-      fa_lo = bf16_bits(s0) | (bf16_bits(s1) << 16);  // the k8 MMA: A_lo
+    // ------------------------------------------------------------ quantizer sets
+    const int w = warp - 2;
+    const int set = w / kSetWarps;       // units n with n % 2 == set
+    const int j = (w >> 2) & 1;          // block of the pair
+    const int q = warp & 3;              // TMEM lane quarter of this warp
+    const uint32_t taddr0 = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                            static_cast<uint32_t>(set) * kAccCols + j * kSlotCols;
+    // unit state: pair, token tile; per-pair: block column, clip ratios, output pointers
+    int64_t pair = pair0, mt = mt0;
+    if (set == 1 && u_begin + 1 < u_end) {
+      if (++mt == p.mtiles) { mt = 0; ++pair; }
     }
-    // Private factor as broadcast pairs: b2[i][j] = {B[i][j], B[i][j]}.
-    uint64_t b2[4][4];
+    int64_t b = 0, m = 0;
+    bool bvalid = false, pad2 = false;
     float r_lo = 1.0f, r_hi = 1.0f;
-    {
-      const float4* bp = reinterpret_cast<const float4*>(p.b + static_cast<int64_t>(active ? b : 0) * 16);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 v = __ldg(bp + i);
-        b2[i][0] = pack2(v.x, v.x);
-        b2[i][1] = pack2(v.y, v.y);
-        b2[i][2] = pack2(v.z, v.z);
-        b2[i][3] = pack2(v.w, v.w);
-      }
-      if (!kPerRowClip && active) {
+    uint8_t* cptr = nullptr;   // 16 code bytes of (m, b)
+    uint8_t* sptr = nullptr;   // scale byte of (m, b)
+    float* yptr = nullptr;     // trace of (m, b)
+    auto enter_pair = [&]() {
+      b = 2 * pair + j;
+      bvalid = b < p.nb;
+      // the last pair also writes the padding scale bytes of blocks [2*nbp2, 4*nbp4)
+      pad2 = (b & 3) < 2 && b + 2 >= 2 * static_cast<int64_t>(p.nbp2) && b + 2 < 4 * static_cast<int64_t>(p.nbp4);
+      if (!kPerRowClip && bvalid) {
         r_lo = p.g_lo ? clip_ratio(p.g_lo[b]) : 1.0f;
         r_hi = p.g_hi ? clip_ratio(p.g_hi[b]) : 1.0f;
       }
-    }
-    const uint32_t tbuf = sbase + kStages * kStageBytes + warp * kTBytes;
-
-    for (int st = 0; st < nst; ++st) {
-      const int slot = st % kStages;
-      const uint32_t par = static_cast<uint32_t>((st / kStages) & 1);
-      if (!mbar_wait(bars + 8 * slot, par, kErrWaitFull)) break;
-      const int64_t m = row0 + static_cast<int64_t>(st) * kRowsPerStage + warp;
-      const bool row_ok = m < row1;
-      if (row_ok) {
-        // ---- 1+2: T = X_r A on the tensor cores, 16 rows of 8 (4 blocks) per MMA tile
-        const uint32_t xrow = sbase + slot * kStageBytes + warp * kSegBytes;
-        __syncwarp();  // the previous row's T has been read by every lane
+    };
+    auto set_ptrs = [&]() {
+      m = mt * kTok + 32 * q + lane;
+      cptr = p.codes + m * (p.K / 2) + b * (kG / 2);
+      sptr = p.scales + scale_offset(m, b, p.nbp4);
+      if (kTrace) yptr = p.y_out + m * p.K + b * kG;
+    };
+    enter_pair();
+    set_ptrs();
+    uint32_t k = 0;  // this set's units handled so far
+    for (int64_t u = u_begin + set; u < u_end; u += kSets, ++k) {
+      if (!mbar_wait(tfull(set), k & 1u, kErrWaitTmemFull)) break;
+      tc_fence_after();
+      // the three partial products y_hi, y_mid, y_lo, summed in that order
+      uint32_t r[32], r2[32];
+      tmem_ld_32x32b_x32(taddr0, r);
+      tmem_ld_32x32b_x32(taddr0 + 32, r2);
+      tmem_wait_ld();
+      uint64_t y2[16];
 #pragma unroll
-        for (int tp = 0; tp < 4; ++tp) {
-          uint32_t x0, x1, x2, x3;  // tiles 2tp (x0, x1) and 2tp+1 (x2, x3)
-          ldsm_x4(xrow + tp * 512 + lane * 16, x0, x1, x2, x3);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t a0 = h ? x2 : x0, a1 = h ? x3 : x1;
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-            mma_16816(d, a0, a1, a0, a1, fa_hm0, fa_hm1);
-            mma_1688(d, a0, a1, fa_lo);
-            // rows c = 32tp + 16h + g and c + 8: block c/4, row i = c%4, columns 2*t4, 2*t4+1;
-            // 16-byte unit (2i + t4/2) of block blk sits at unit ^ (blk % 8)
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-              const int c = 32 * tp + 16 * h + g + 8 * r;
-              const int blk = c >> 2, i = c & 3;
-              sts_v2(tbuf + blk * 128 + ((((i << 1) | (t4 >> 1)) ^ (blk & 7)) << 4) + ((t4 & 1) << 3),
-                     d[2 * r], d[2 * r + 1]);
-            }
-          }
-        }
-      }
+      for (int c = 0; c < 16; ++c)
+        y2[c] = fadd2(pack2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])),
+                      pack2(__uint_as_float(r2[2 * c]), __uint_as_float(r2[2 * c + 1])));
+      tmem_ld_32x32b_x32(taddr0 + 64, r);
+      tmem_wait_ld();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bars + 8 * (kStages + slot));  // X row consumed
-      if (row_ok && active) {
-        if (kPerRowClip) {
-          const int64_t ri = m * p.nb + b;
-          r_lo = p.g_lo ? clip_ratio(p.g_lo[ri]) : 1.0f;
-          r_hi = p.g_hi ? clip_ratio(p.g_hi[ri]) : 1.0f;
-        }
-        // ---- 3: T rows as column pairs, t2[i][qq] = {T[i][2qq], T[i][2qq+1]}
-        uint64_t t2[4][4];
+      if (lane == 0) mbar_arrive(tempty(set));  // accumulator read: the issuer may reuse it
+      float y[32];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint4 v = lds_v4(tbuf + lane * 128 + ((u ^ (lane & 7)) << 4));
-          t2[u >> 1][(u & 1) * 2] = pack2(__uint_as_float(v.x), __uint_as_float(v.y));
-          t2[u >> 1][(u & 1) * 2 + 1] = pack2(__uint_as_float(v.z), __uint_as_float(v.w));
-        }
-        // ---- Y = B^T T  (Y[j][q] = sum_i B[i][j] T[i][q])
-        float y[32];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
-            uint64_t acc = fmul2(b2[0][j], t2[0][qq]);
-            acc = ffma2(b2[1][j], t2[1][qq], acc);
-            acc = ffma2(b2[2][j], t2[2][qq], acc);
-            acc = ffma2(b2[3][j], t2[3][qq], acc);
-            unpack2(acc, y[8 * j + 2 * qq], y[8 * j + 2 * qq + 1]);
-          }
-        }
-        const int64_t eoff = m * p.K + static_cast<int64_t>(b) * kG;  // element offset of the block
+      for (int c = 0; c < 16; ++c)
+        unpack2(fadd2(y2[c], pack2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1]))), y[2 * c],
+                y[2 * c + 1]);
+      const bool valid = bvalid && m < p.rows;
+      if (kPerRowClip && valid) {
+        const int64_t ri = m * p.nb + b;
+        r_lo = p.g_lo ? clip_ratio(p.g_lo[ri]) : 1.0f;
+        r_hi = p.g_hi ? clip_ratio(p.g_hi[ri]) : 1.0f;
+      }
+      uint32_t packed[4];
+      const uint32_t sbyte = quantize_block(y, r_lo, r_hi, packed);
+      if (valid) {
+        *reinterpret_cast<uint4*>(cptr) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
         if (kTrace) {
-          float4* dst = reinterpret_cast<float4*>(p.y_out + eoff);
+          float4* dst = reinterpret_cast<float4*>(yptr);
 #pragma unroll
           for (int c = 0; c < 8; ++c)
             dst[c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
         }
-        // ---- block clip: [r_lo * min, r_hi * max]; 3-input min/max trees
-        float tmn[11], tmx[11];
-#pragma unroll
-        for (int k = 0; k < 10; ++k) {
-          tmn[k] = min3f(y[3 * k], y[3 * k + 1], y[3 * k + 2]);
-          tmx[k] = max3f(y[3 * k], y[3 * k + 1], y[3 * k + 2]);
-        }
-        tmn[10] = fminf(y[30], y[31]);
-        tmx[10] = fmaxf(y[30], y[31]);
-        const float mn = fminf(min3f(min3f(tmn[0], tmn[1], tmn[2]), min3f(tmn[3], tmn[4], tmn[5]),
-                                     min3f(tmn[6], tmn[7], tmn[8])),
-                               fminf(tmn[9], tmn[10]));
-        const float mx = fmaxf(max3f(max3f(tmx[0], tmx[1], tmx[2]), max3f(tmx[3], tmx[4], tmx[5]),
-                                     max3f(tmx[6], tmx[7], tmx[8])),
-                               fmaxf(tmx[9], tmx[10]));
-        const float lo = __fmul_rn(r_lo, mn);
-        const float hi = __fmul_rn(r_hi, mx);
-        // The clamp is monotone, so the clipped block's extremes are the clipped min/max.
-        const float amax = fmaxf(fabsf(fminf(fmaxf(mn, lo), hi)), fabsf(fminf(fmaxf(mx, lo), hi)));
-        // ---- UE8M0 scale: e = floor(log2 amax) - 2, clamped to >= -127 (amax = 0 -> -127)
-        const int efield = static_cast<int>(__float_as_uint(amax) >> 23);
-        const int sbyte = efield > 2 ? efield - 2 : 0;  // e + 127
-        const float inv_scale = __uint_as_float(static_cast<uint32_t>(254 - sbyte) << 23);  // 2^-e
-        const uint64_t s2 = pack2(inv_scale, inv_scale);
-        // ---- codes: v = c * 2^-e (+0 turns an exact -0 into +0), E2M1 round-to-nearest-even
-        uint32_t byte[16];
-#pragma unroll
-        for (int h = 0; h < 16; ++h) {
-          const float c0 = fminf(fmaxf(y[2 * h], lo), hi);
-          const float c1 = fminf(fmaxf(y[2 * h + 1], lo), hi);
-          float v0, v1;
-          unpack2(ffma2(pack2(c0, c1), s2, 0ull), v0, v1);
-          byte[h] = e2m1x2(v0, v1);
-        }
-        uint32_t packed[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          packed[c] = (byte[4 * c] | (byte[4 * c + 1] << 8)) | ((byte[4 * c + 2] << 16) | (byte[4 * c + 3] << 24));
-        *reinterpret_cast<uint4*>(p.codes + eoff / 2) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-        p.scales[scale_offset(m, b, p.nbp4)] = static_cast<uint8_t>(sbyte);
+      }
+      // rows past M and blocks past nb are padding of the tiled scale buffer: 0
+      *sptr = static_cast<uint8_t>(valid ? sbyte : 0u);
+      if (pad2) sptr[2] = 0;
+      // next unit of this set: two token tiles on (possibly into the next pairs)
+      const int64_t old_pair = pair;
+      mt += kSets;
+      while (mt >= p.mtiles) { mt -= p.mtiles; ++pair; }
+      if (pair != old_pair) {
+        enter_pair();
+        set_ptrs();
+      } else {
+        m += kSets * kTok;
+        cptr += kSets * kTok * (p.K / 2);
+        sptr += static_cast<int64_t>(kSets) * p.nbp4 * 512;
+        if (kTrace) yptr += kSets * kTok * p.K;
       }
     }
   }
 
-  // ---- zero the padding bytes of the tiled scale buffer
-  const int64_t rows_pad = (p.rows + 127) & ~static_cast<int64_t>(127);
-  const int64_t bcols = static_cast<int64_t>(p.nbp4) * 4;
-  const int64_t pad_cols = bcols - p.nb;                // blocks past nb, rows < M
-  const int64_t n_right = p.rows * pad_cols;
-  const int64_t n_below = (rows_pad - p.rows) * bcols;  // rows past M, all blocks
-  const int64_t tstride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-       t < n_right + n_below; t += tstride) {
-    int64_t m, bb;
-    if (t < n_right) {
-      m = t / pad_cols;
-      bb = p.nb + (t - m * pad_cols);
-    } else {
-      const int64_t r = t - n_right;
-      m = p.rows + r / bcols;
-      bb = r - (m - p.rows) * bcols;
-    }
-    p.scales[scale_offset(m, bb, p.nbp4)] = 0;
-  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
 }
 
 __global__ void bat_clip_ratio_kernel(const float* g, int64_t n, float* r) {
