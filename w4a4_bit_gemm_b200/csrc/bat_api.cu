@@ -219,7 +219,15 @@ bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float
   p.nbp2 = (p.nb + 1) / 2;
   p.nbp4 = (p.nb + 3) / 4;
   p.mtiles = (rows + bat::pro::kTok - 1) / bat::pro::kTok;
-  p.units = p.mtiles * p.nbp2;
+  p.strips = (p.nbp2 + bat::pro::kStrip - 1) / bat::pro::kStrip;
+  // CTAs per strip: the SMs shared out over the strips, but no more CTAs than a
+  // strip has units
+  {
+    int cps = sms / p.strips;
+    const int64_t strip_units = p.mtiles * (p.nbp2 < bat::pro::kStrip ? p.nbp2 : bat::pro::kStrip);
+    if (cps > strip_units) cps = static_cast<int>(strip_units);
+    p.cps = cps < 1 ? 1 : cps;
+  }
   void (*kern)(CUtensorMap, bat::PrologueParams);
   if (per_row)
     kern = y_out ? bat::bat_prologue_kernel<true, true> : bat::bat_prologue_kernel<false, true>;
@@ -233,8 +241,8 @@ bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float
       return BAT_ERR_CUDA;
     d.pro_attr.fetch_or(variant_bit);
   }
-  // One CTA per SM, each over a contiguous range of (block pair, token tile) units.
-  const int64_t grid = p.units < sms ? p.units : sms;
+  // One CTA per (strip, part): about one per SM.
+  const int64_t grid = static_cast<int64_t>(p.strips) * p.cps;
   kern<<<static_cast<unsigned>(grid), bat::pro::kThreads, bat::pro::kSmemBytes, stream>>>(tx, p);
   return cuda_status(cudaGetLastError());
 }

@@ -18,21 +18,22 @@
 // scale and E2M1 codes need no exchange between threads.
 //
 // Work unit: 128 tokens x one pair of blocks (a 128-row x 128-byte box of X).
+// Block pairs are grouped into strips of kStrip pairs; each CTA owns one strip
+// (the P terms of all its blocks stay in shared memory) and a contiguous range
+// of its units, walked token tile by token tile with the strip's pairs inner, so
+// that consecutive copies read adjacent 128-byte pieces of the same 128 rows.
 //   warp 0      producer: TMA copies of the units' boxes into a ring of kStages
-//               shared-memory stages (lane 0), and, with all 32 lanes, the P
-//               terms of each new block pair before its first copy;
+//               shared-memory stages;
 //   warp 1      TMEM owner and MMA issuer: per unit, two blocks x two K-steps of
 //               M=128, N=96, K=16 into one of two 192-column accumulators;
 //   warps 2-17  two quantizer sets of eight warps; set s takes the units whose
 //               index within the CTA is s mod 2, warp (s, j, q) block j of the
 //               pair for the 32 tokens of TMEM lane quarter q.
-// The issuer waits once per unit for its copy and once for its accumulator, so
-// its chain of waits, MMAs and commits stays well inside the copy's time, and
-// each quantizer set has two units' time for one block.
-// A CTA walks a contiguous range of units ordered by block pair, so it needs the
-// terms of only a few pairs. They sit in two shared-memory buffers (pair i of
-// the CTA's range in buffer i%2); the producer refills a buffer only after the
-// issuer has signalled that the MMAs of the pair that used it have finished.
+// Warps 1-17 build the strip's P terms (and its blocks' clip ratios) while the
+// producer's first copies are in flight. The issuer waits once per unit for its
+// copy and once for its accumulator, so its chain of waits, MMAs and commits
+// stays inside the copy's time, and each quantizer set has two units' time for
+// one block.
 #pragma once
 
 #include "bat_common.cuh"
@@ -42,16 +43,19 @@ namespace bat {
 namespace pro {
 constexpr int kTok = 128;                        // tokens per unit (MMA M)
 constexpr int kBlk = 2;                          // 32-element blocks per unit
+constexpr int kStrip = 4;                        // block pairs per strip
 constexpr int kStages = 10;
 constexpr int kStageBytes = kTok * 128;          // 128 rows x 64 bf16: 16 KB
 constexpr int kPTermBytes = 32 * 32 * 2;         // one bf16 term of one block's P: 2 KB
 constexpr int kPBlockBytes = 3 * kPTermBytes;    // one block's three terms: 6 KB
-constexpr int kPBytes = kBlk * kPBlockBytes;     // one pair: 12 KB
+constexpr int kPPairBytes = kBlk * kPBlockBytes; // 12 KB
+constexpr int kPBytes = kStrip * kPPairBytes;    // one strip: 96 KB
 constexpr int kSets = 2;                         // quantizer sets (alternate units)
 constexpr int kSetWarps = 4 * kBlk;              // lane quarters x blocks
 constexpr int kThreads = 32 * (2 + kSets * kSetWarps);
-constexpr int kBarBytes = 256;
-constexpr int kSmemBytes = kStages * kStageBytes + 2 * kPBytes + kBarBytes + 1024;
+constexpr int kBuilders = kThreads - 32;         // every warp but the producer
+constexpr int kBarBytes = 2048;                  // barriers, TMEM address, clip ratios, A, B
+constexpr int kSmemBytes = kStages * kStageBytes + kPBytes + kBarBytes + 1024;
 constexpr int kSlotCols = 96;                    // one block's accumulator: 3 terms x 32 columns
 constexpr uint32_t kAccCols = kBlk * kSlotCols;  // one unit's accumulator: 192 columns
 constexpr uint32_t kTmemCols = 512;              // allocation (power of two) holding 2 x 192
@@ -71,7 +75,8 @@ struct PrologueParams {
   int nbp2;              // ceil(nb / 2): block pairs
   int nbp4;              // ceil(nb / 4): groups of the tiled scale layout
   int64_t mtiles;        // ceil(rows / 128)
-  int64_t units;         // nbp2 * mtiles, unit u = (pair u / mtiles, token tile u % mtiles)
+  int strips;            // ceil(nbp2 / kStrip)
+  int cps;               // CTAs per strip (grid = strips * cps)
 };
 
 // fp32(sigma(g)) evaluated in fp64; +inf gives exactly 1.
@@ -123,18 +128,18 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
 // three together are one N=96 operand). Operand element (n, k) is
 // P_b[k][n] = B_b[k/8][n/8] * A[k%8][n%8]; a block past nb gets 0.
 // `row` in [0, 128) picks n = row/4 and the eight k of core-matrix column row%4:
-// one 16-byte row of a core matrix per term.
-__device__ __forceinline__ void build_p_row(uint8_t* dst, const PrologueParams& p, int64_t b,
-                                            int row) {
+// one 16-byte row of a core matrix per term. `a` is A (8x8) and `bb` is B_b (4x4,
+// zeros for a block past nb), both staged in shared memory.
+__device__ __forceinline__ void build_p_row(uint8_t* dst, const float* a, const float* bb, int row) {
   const int n = row >> 2, kc = row & 3;
   uint32_t w[3][4];
-  const float bv = b < p.nb ? p.b[b * 16 + kc * 4 + (n >> 3)] : 0.0f;  // B_b[k/8][n/8], k/8 = kc
+  const float bv = bb[kc * 4 + (n >> 3)];  // B_b[k/8][n/8], k/8 = kc
 #pragma unroll
   for (int i = 0; i < 8; i += 2) {
     uint32_t hh[2], mm[2], ll[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const float prod = __fmul_rn(bv, p.a[(i + h) * 8 + (n & 7)]);  // A[k%8][n%8]
+      const float prod = __fmul_rn(bv, a[(i + h) * 8 + (n & 7)]);  // A[k%8][n%8]
       const uint32_t hi = bf16_bits(prod);
       const float r1 = prod - __uint_as_float(hi << 16);
       const uint32_t mid = bf16_bits(r1);
@@ -180,19 +185,19 @@ __device__ __forceinline__ uint32_t quantize_block(const float (&y)[32], float r
   const int sbyte = efield > 2 ? efield - 2 : 0;  // e + 127
   const float inv_scale = __uint_as_float(static_cast<uint32_t>(254 - sbyte) << 23);  // 2^-e
   const uint64_t s2 = pack2(inv_scale, inv_scale);
-  // codes: v = c * 2^-e (+0 turns an exact -0 into +0), E2M1 round-to-nearest-even
-  uint32_t byte[16];
+  // codes: v = c * 2^-e (+0 turns an exact -0 into +0), E2M1 round-to-nearest-even,
+  // eight codes per 32-bit word
 #pragma unroll
-  for (int h = 0; h < 16; ++h) {
-    const float c0 = fminf(fmaxf(y[2 * h], lo), hi);
-    const float c1 = fminf(fmaxf(y[2 * h + 1], lo), hi);
-    float v0, v1;
-    unpack2(ffma2(pack2(c0, c1), s2, 0ull), v0, v1);
-    byte[h] = e2m1x2(v0, v1);
+  for (int c = 0; c < 4; ++c) {
+    float v[8];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float c0 = fminf(fmaxf(y[8 * c + 2 * h], lo), hi);
+      const float c1 = fminf(fmaxf(y[8 * c + 2 * h + 1], lo), hi);
+      unpack2(ffma2(pack2(c0, c1), s2, 0ull), v[2 * h], v[2 * h + 1]);
+    }
+    packed[c] = e2m1x8(v);
   }
-#pragma unroll
-  for (int c = 0; c < 4; ++c)
-    packed[c] = (byte[4 * c] | (byte[4 * c + 1] << 8)) | ((byte[4 * c + 2] << 16) | (byte[4 * c + 3] << 24));
   return static_cast<uint32_t>(sbyte);
 }
 
@@ -206,40 +211,49 @@ __global__ void __launch_bounds__(pro::kThreads, 1)
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t base = (raw_u32 + 1023u) & ~1023u;  // 128-byte swizzle atoms: 1 KB aligned
   uint8_t* base_ptr = smem_raw + (base - raw_u32);
-  const uint32_t pbase = base + kStages * kStageBytes;  // [buffer][block][term][2 KB]
+  const uint32_t pbase = base + kStages * kStageBytes;  // [pair][block][term][2 KB]
   uint8_t* pbase_ptr = base_ptr + kStages * kStageBytes;
-  const uint32_t bars = pbase + 2 * kPBytes;
+  const uint32_t bars = pbase + kPBytes;
   auto full_bar = [&](int s) { return bars + 8u * s; };
   auto empty_bar = [&](int s) { return bars + 8u * (kStages + s); };
-  auto tfull = [&](int a) { return bars + 8u * (2 * kStages + a); };
-  auto tempty = [&](int a) { return bars + 8u * (2 * kStages + 2 + a); };
-  auto pfull = [&](int buf) { return bars + 8u * (2 * kStages + 4 + buf); };
-  auto pdone = [&](int buf) { return bars + 8u * (2 * kStages + 6 + buf); };
-  const uint32_t done_bar = bars + 8u * (2 * kStages + 8);
+  auto tfull = [&](uint32_t a) { return bars + 8u * (2 * kStages + a); };
+  auto tempty = [&](uint32_t a) { return bars + 8u * (2 * kStages + 2 + a); };
+  const uint32_t pfull = bars + 8u * (2 * kStages + 4);
+  const uint32_t done_bar = pfull + 8u;
   const uint32_t tmem_slot = done_bar + 8u;
   volatile uint32_t* tmem_slot_ptr =
       reinterpret_cast<volatile uint32_t*>(base_ptr + (tmem_slot - base));
+  // clip ratios of the strip's blocks: [2 * kStrip] lo, then [2 * kStrip] hi
+  float* ratios = reinterpret_cast<float*>(base_ptr + (bars - base) + 256);
+  // A and the strip's B_b, staged for the P build
+  float* sA = reinterpret_cast<float*>(base_ptr + (bars - base) + 512);
+  float* sB = sA + 64;  // [2 * kStrip][16]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // contiguous unit range of this CTA and the block pairs it spans
-  const int64_t u_begin = p.units * blockIdx.x / gridDim.x;
-  const int64_t u_end = p.units * (blockIdx.x + 1) / gridDim.x;
-  const int64_t pair0 = u_begin / p.mtiles;
-  const int64_t mt0 = u_begin - pair0 * p.mtiles;
+  // this CTA's strip and its contiguous range of the strip's units, unit v of the
+  // strip = (token tile v / npair, pair strip * kStrip + v % npair)
+  const int strip = static_cast<int>(blockIdx.x) / p.cps;
+  const int part = static_cast<int>(blockIdx.x) - strip * p.cps;
+  const int pair_base = strip * kStrip;
+  const int npair = min(kStrip, p.nbp2 - pair_base);
+  const int64_t sunits = p.mtiles * npair;
+  const int64_t v_begin = sunits * part / p.cps;
+  const int64_t v_end = sunits * (part + 1) / p.cps;
+  const int64_t mt0 = v_begin / npair;
+  const int pr0 = static_cast<int>(v_begin - mt0 * npair);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (uint32_t a = 0; a < 2; ++a) {
       mbar_init(tfull(a), 1);
       mbar_init(tempty(a), kSetWarps);
-      mbar_init(pfull(a), 32);  // the producer warp's lanes
-      mbar_init(pdone(a), 1);
     }
+    mbar_init(pfull, kBuilders);
     mbar_init(done_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&tmap_x);
@@ -255,182 +269,178 @@ __global__ void __launch_bounds__(pro::kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    int stage = 0;
-    uint32_t phase = 0;
-    uint32_t inflight = 0;  // bit s: stage s was loaded; bit 16+s: parity of that load
-    int64_t pair = pair0, mt = mt0;
-    uint32_t rel = 0;       // pair index within the CTA's range
-    bool ok = true;
-    for (int64_t u = u_begin; u < u_end && ok; ++u) {
-      if (u == u_begin || mt == 0) {
-        // a new pair: its terms go to buffer rel%2 once the pair that used that
-        // buffer (rel-2) has no MMA left in flight
-        if (rel >= 2 && !mbar_wait(pdone(rel & 1u), ((rel - 2) >> 1) & 1u, kErrWaitEmpty)) break;
-        build_p_row(pbase_ptr + (rel & 1u) * kPBytes, p, 2 * pair, lane);
-        build_p_row(pbase_ptr + (rel & 1u) * kPBytes, p, 2 * pair, lane + 32);
-        build_p_row(pbase_ptr + (rel & 1u) * kPBytes, p, 2 * pair, lane + 64);
-        build_p_row(pbase_ptr + (rel & 1u) * kPBytes, p, 2 * pair, lane + 96);
-        build_p_row(pbase_ptr + (rel & 1u) * kPBytes + kPBlockBytes, p, 2 * pair + 1, lane);
-        build_p_row(pbase_ptr + (rel & 1u) * kPBytes + kPBlockBytes, p, 2 * pair + 1, lane + 32);
-        build_p_row(pbase_ptr + (rel & 1u) * kPBytes + kPBlockBytes, p, 2 * pair + 1, lane + 64);
-        build_p_row(pbase_ptr + (rel & 1u) * kPBytes + kPBlockBytes, p, 2 * pair + 1, lane + 96);
-        fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor cores
-        mbar_arrive(pfull(rel & 1u));
-      }
-      if (lane == 0) {
-        if (!mbar_wait(empty_bar(stage), phase ^ 1u, kErrWaitEmpty)) {
-          ok = false;
-        } else {
-          mbar_expect_tx(full_bar(stage), kStageBytes);
-          tma_load_2d(base + stage * kStageBytes, &tmap_x, full_bar(stage),
-                      static_cast<int32_t>(pair * 64), static_cast<int32_t>(mt * kTok));
-          inflight = (inflight & ~(0x10001u << stage)) | (1u << stage) | (phase << (16 + stage));
-        }
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (++stage == kStages) { stage = 0; phase ^= 1u; }
-      if (++mt == p.mtiles) { mt = 0; ++pair; ++rel; }
-    }
-    // no copy may still be writing shared memory when the CTA exits
-    if (lane == 0)
-      for (int s = 0; s < kStages; ++s)
-        if ((inflight >> s) & 1u) mbar_wait(full_bar(s), (inflight >> (16 + s)) & 1u, kErrWaitFull);
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // The boxes of one token tile (the strip's pairs, adjacent 128-byte pieces of
+    // the same 128 rows) are issued back to back once enough stages are free, so
+    // that the memory system sees whole row segments rather than lone 128-byte
+    // pieces of rows 8 KB apart.
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(kTok, kSlotCols);
-      // Descriptors differ only in the start-address field (bits 0-13, address / 16).
-      const uint64_t adesc0 = smem_desc(base, 16, 1024, 2);
-      const uint64_t bdesc0 = smem_desc(pbase, 128, 512, 0);
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t rel = 0;
+      uint32_t inflight = 0;  // bit s: stage s was loaded; bit 16+s: parity of that load
       int64_t mt = mt0;
-      uint32_t n = 0;
-      for (int64_t u = u_begin; u < u_end; ++u, ++n) {
-        if (u == u_begin || mt == 0)
-          if (!mbar_wait(pfull(rel & 1u), (rel >> 1) & 1u, kErrWaitFull)) break;
-        const uint32_t a = n & 1u;
-        if (!mbar_wait(full_bar(stage), phase, kErrWaitFull)) break;
-        if (!mbar_wait(tempty(a), ((n >> 1) & 1u) ^ 1u, kErrWaitTmemEmpty)) break;
-        tc_fence_after();
-        const uint64_t ad = adesc0 + static_cast<uint32_t>(stage * (kStageBytes >> 4));
-        const uint64_t bd = bdesc0 + (rel & 1u) * static_cast<uint32_t>(kPBytes >> 4);
-        const uint32_t d = tmem_base + a * kAccCols;
-#pragma unroll
-        for (int j = 0; j < kBlk; ++j)
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks)
-            // A: block j is the j-th 64 bytes of the box's 128-byte rows, K-step 32 bytes;
-            // B: block j's three terms (96 rows), K-step 256 bytes
-            mma_bf16(d + j * kSlotCols, ad + ((j * 64 + ks * 32) >> 4),
-                     bd + ((j * kPBlockBytes + ks * 256) >> 4), idesc, static_cast<uint32_t>(ks));
-        tc_commit(tfull(a));
-        tc_commit(empty_bar(stage));
-        if (++stage == kStages) { stage = 0; phase ^= 1u; }
-        if (++mt == p.mtiles || u + 1 == u_end) {
-          tc_commit(pdone(rel & 1u));  // this pair's MMAs: its buffer may be refilled
-          mt = 0;
-          ++rel;
+      int pr = pr0;
+      bool ok = true;
+      for (int64_t v = v_begin; v < v_end && ok;) {
+        int64_t cnt = npair - pr;
+        if (cnt > v_end - v) cnt = v_end - v;
+        if (cnt > kStages) cnt = kStages;
+        // wait for the next cnt stages to be free
+        int s2 = stage;
+        uint32_t ph2 = phase;
+        for (int i = 0; i < cnt; ++i) {
+          if (!mbar_wait(empty_bar(s2), ph2 ^ 1u, kErrWaitEmpty)) { ok = false; break; }
+          if (++s2 == kStages) { s2 = 0; ph2 ^= 1u; }
+        }
+        for (int i = 0; i < cnt && ok; ++i) {
+          mbar_expect_tx(full_bar(stage), kStageBytes);
+          tma_load_2d(base + stage * kStageBytes, &tmap_x, full_bar(stage),
+                      (pair_base + pr) * 64, static_cast<int32_t>(mt * kTok));
+          inflight = (inflight & ~(0x10001u << stage)) | (1u << stage) | (phase << (16 + stage));
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+          if (++pr == npair) { pr = 0; ++mt; }
+          ++v;
         }
       }
-      // every MMA issued above has finished before TMEM is released
-      tc_commit(done_bar);
-      mbar_wait(done_bar, 0, kErrWaitTmemFull);
+      // no copy may still be writing shared memory when the CTA exits
+      for (int s = 0; s < kStages; ++s)
+        if ((inflight >> s) & 1u) mbar_wait(full_bar(s), (inflight >> (16 + s)) & 1u, kErrWaitFull);
     }
   } else {
-    // ------------------------------------------------------------ quantizer sets
-    const int w = warp - 2;
-    const int set = w / kSetWarps;       // units n with n % 2 == set
-    const int j = (w >> 2) & 1;          // block of the pair
-    const int q = warp & 3;              // TMEM lane quarter of this warp
-    const uint32_t taddr0 = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
-                            static_cast<uint32_t>(set) * kAccCols + j * kSlotCols;
-    // unit state: pair, token tile; per-pair: block column, clip ratios, output pointers
-    int64_t pair = pair0, mt = mt0;
-    if (set == 1 && u_begin + 1 < u_end) {
-      if (++mt == p.mtiles) { mt = 0; ++pair; }
+    // ------------------------------------------------ P terms and clip ratios
+    {
+      const int t = threadIdx.x - 32;
+      // stage A and the strip's B_b with one coalesced load each
+      if (t < 64) {
+        sA[t] = p.a[t];
+      } else if (t < 64 + 32 * npair) {
+        const int64_t e = 2 * static_cast<int64_t>(pair_base) * 16 + (t - 64);  // [block][16]
+        sB[t - 64] = e < static_cast<int64_t>(p.nb) * 16 ? p.b[e] : 0.0f;
+      } else if (!kPerRowClip && t >= 320 && t < 320 + 2 * npair) {
+        const int lb = t - 320;
+        const int64_t blk = 2 * static_cast<int64_t>(pair_base) + lb;
+        const bool ok = blk < p.nb;
+        ratios[lb] = (ok && p.g_lo) ? clip_ratio(p.g_lo[blk]) : 1.0f;
+        ratios[2 * kStrip + lb] = (ok && p.g_hi) ? clip_ratio(p.g_hi[blk]) : 1.0f;
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kBuilders) : "memory");  // warps 1-17
+      // pairs this CTA's units touch: all of the strip's, or a short run of them
+      const int64_t nv = v_end - v_begin;
+      for (int r = t; r < npair * 2 * 128; r += kBuilders) {
+        const int pr = r >> 8, jj = (r >> 7) & 1;
+        const bool used = nv >= npair || ((pr - pr0 + npair) % npair) < nv;
+        if (used)
+          build_p_row(pbase_ptr + pr * kPPairBytes + jj * kPBlockBytes, sA, sB + (2 * pr + jj) * 16, r & 127);
+      }
+      fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor cores
+      mbar_arrive(pfull);
     }
-    int64_t b = 0, m = 0;
-    bool bvalid = false, pad2 = false;
-    float r_lo = 1.0f, r_hi = 1.0f;
-    uint8_t* cptr = nullptr;   // 16 code bytes of (m, b)
-    uint8_t* sptr = nullptr;   // scale byte of (m, b)
-    float* yptr = nullptr;     // trace of (m, b)
-    auto enter_pair = [&]() {
-      b = 2 * pair + j;
-      bvalid = b < p.nb;
-      // the last pair also writes the padding scale bytes of blocks [2*nbp2, 4*nbp4)
-      pad2 = (b & 3) < 2 && b + 2 >= 2 * static_cast<int64_t>(p.nbp2) && b + 2 < 4 * static_cast<int64_t>(p.nbp4);
-      if (!kPerRowClip && bvalid) {
-        r_lo = p.g_lo ? clip_ratio(p.g_lo[b]) : 1.0f;
-        r_hi = p.g_hi ? clip_ratio(p.g_hi[b]) : 1.0f;
-      }
-    };
-    auto set_ptrs = [&]() {
-      m = mt * kTok + 32 * q + lane;
-      cptr = p.codes + m * (p.K / 2) + b * (kG / 2);
-      sptr = p.scales + scale_offset(m, b, p.nbp4);
-      if (kTrace) yptr = p.y_out + m * p.K + b * kG;
-    };
-    enter_pair();
-    set_ptrs();
-    uint32_t k = 0;  // this set's units handled so far
-    for (int64_t u = u_begin + set; u < u_end; u += kSets, ++k) {
-      if (!mbar_wait(tfull(set), k & 1u, kErrWaitTmemFull)) break;
-      tc_fence_after();
-      // the three partial products y_hi, y_mid, y_lo, summed in that order
-      uint32_t r[32], r2[32];
-      tmem_ld_32x32b_x32(taddr0, r);
-      tmem_ld_32x32b_x32(taddr0 + 32, r2);
-      tmem_wait_ld();
-      uint64_t y2[16];
+    if (warp == 1) {
+      // ---------------------------------------------------------- MMA issuer
+      if (lane == 0 && mbar_wait(pfull, 0, kErrWaitFull)) {
+        constexpr uint32_t idesc = idesc_bf16(kTok, kSlotCols);
+        // Descriptors differ only in the start-address field (bits 0-13, address / 16).
+        const uint64_t adesc0 = smem_desc(base, 16, 1024, 2);
+        const uint64_t bdesc0 = smem_desc(pbase, 128, 512, 0);
+        int stage = 0;
+        uint32_t phase = 0;
+        int pr = pr0;
+        uint32_t n = 0;
+        for (int64_t v = v_begin; v < v_end; ++v, ++n) {
+          const uint32_t a = n & 1u;
+          if (!mbar_wait(full_bar(stage), phase, kErrWaitFull)) break;
+          if (!mbar_wait(tempty(a), ((n >> 1) & 1u) ^ 1u, kErrWaitTmemEmpty)) break;
+          tc_fence_after();
+          const uint64_t ad = adesc0 + static_cast<uint32_t>(stage * (kStageBytes >> 4));
+          const uint64_t bd = bdesc0 + static_cast<uint32_t>(pr * (kPPairBytes >> 4));
+          const uint32_t d = tmem_base + a * kAccCols;
 #pragma unroll
-      for (int c = 0; c < 16; ++c)
-        y2[c] = fadd2(pack2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])),
-                      pack2(__uint_as_float(r2[2 * c]), __uint_as_float(r2[2 * c + 1])));
-      tmem_ld_32x32b_x32(taddr0 + 64, r);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tempty(set));  // accumulator read: the issuer may reuse it
-      float y[32];
+          for (int j = 0; j < kBlk; ++j)
 #pragma unroll
-      for (int c = 0; c < 16; ++c)
-        unpack2(fadd2(y2[c], pack2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1]))), y[2 * c],
-                y[2 * c + 1]);
-      const bool valid = bvalid && m < p.rows;
-      if (kPerRowClip && valid) {
-        const int64_t ri = m * p.nb + b;
-        r_lo = p.g_lo ? clip_ratio(p.g_lo[ri]) : 1.0f;
-        r_hi = p.g_hi ? clip_ratio(p.g_hi[ri]) : 1.0f;
-      }
-      uint32_t packed[4];
-      const uint32_t sbyte = quantize_block(y, r_lo, r_hi, packed);
-      if (valid) {
-        *reinterpret_cast<uint4*>(cptr) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-        if (kTrace) {
-          float4* dst = reinterpret_cast<float4*>(yptr);
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            dst[c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
+            for (int ks = 0; ks < 2; ++ks)
+              // A: block j is the j-th 64 bytes of the box's 128-byte rows, K-step 32 bytes;
+              // B: block j's three terms (96 rows), K-step 256 bytes
+              mma_bf16(d + j * kSlotCols, ad + ((j * 64 + ks * 32) >> 4),
+                       bd + ((j * kPBlockBytes + ks * 256) >> 4), idesc, static_cast<uint32_t>(ks));
+          tc_commit(tfull(a));
+          tc_commit(empty_bar(stage));
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+          if (++pr == npair) pr = 0;
         }
+        // every MMA issued above has finished before TMEM is released
+        tc_commit(done_bar);
+        mbar_wait(done_bar, 0, kErrWaitTmemFull);
       }
-      // rows past M and blocks past nb are padding of the tiled scale buffer: 0
-      *sptr = static_cast<uint8_t>(valid ? sbyte : 0u);
-      if (pad2) sptr[2] = 0;
-      // next unit of this set: two token tiles on (possibly into the next pairs)
-      const int64_t old_pair = pair;
-      mt += kSets;
-      while (mt >= p.mtiles) { mt -= p.mtiles; ++pair; }
-      if (pair != old_pair) {
-        enter_pair();
-        set_ptrs();
-      } else {
-        m += kSets * kTok;
-        cptr += kSets * kTok * (p.K / 2);
-        sptr += static_cast<int64_t>(kSets) * p.nbp4 * 512;
-        if (kTrace) yptr += kSets * kTok * p.K;
+    } else {
+      // ------------------------------------------------------ quantizer sets
+      const int w = warp - 2;
+      const int set = w / kSetWarps;       // units n with n % 2 == set
+      const int j = (w >> 2) & 1;          // block of the pair
+      const int q = warp & 3;              // TMEM lane quarter of this warp
+      const uint32_t taddr0 = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                              static_cast<uint32_t>(set) * kAccCols + j * kSlotCols;
+      // unit state: token tile and pair index within the strip
+      int64_t mt = mt0;
+      int pr = pr0;
+      if (set == 1 && ++pr == npair) { pr = 0; ++mt; }
+      uint32_t k = 0;  // this set's units handled so far
+      // the clip ratios were written by other warps: wait for all builders
+      const bool ready = mbar_wait(pfull, 0, kErrWaitFull);
+      for (int64_t v = v_begin + set; ready && v < v_end; v += kSets, ++k) {
+        if (!mbar_wait(tfull(set), k & 1u, kErrWaitTmemFull)) break;
+        tc_fence_after();
+        // the three partial products y_hi, y_mid, y_lo, summed in that order
+        uint32_t r[32], r2[32];
+        tmem_ld_32x32b_x32(taddr0, r);
+        tmem_ld_32x32b_x32(taddr0 + 32, r2);
+        tmem_wait_ld();
+        uint64_t y2[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          y2[c] = fadd2(pack2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])),
+                        pack2(__uint_as_float(r2[2 * c]), __uint_as_float(r2[2 * c + 1])));
+        tmem_ld_32x32b_x32(taddr0 + 64, r);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty(set));  // accumulator read: the issuer may reuse it
+        float y[32];
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          unpack2(fadd2(y2[c], pack2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1]))), y[2 * c],
+                  y[2 * c + 1]);
+        const int lb = 2 * pr + j;  // block within the strip
+        const int64_t b = 2 * static_cast<int64_t>(pair_base) + lb;
+        const int64_t m = mt * kTok + 32 * q + lane;  // token
+        const bool valid = b < p.nb && m < p.rows;
+        float r_lo, r_hi;
+        if (kPerRowClip) {
+          r_lo = (valid && p.g_lo) ? clip_ratio(p.g_lo[m * p.nb + b]) : 1.0f;
+          r_hi = (valid && p.g_hi) ? clip_ratio(p.g_hi[m * p.nb + b]) : 1.0f;
+        } else {
+          r_lo = ratios[lb];
+          r_hi = ratios[2 * kStrip + lb];
+        }
+        uint32_t packed[4];
+        const uint32_t sbyte = quantize_block(y, r_lo, r_hi, packed);
+        if (valid) {
+          *reinterpret_cast<uint4*>(p.codes + m * (p.K / 2) + b * (kG / 2)) =
+              make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          if (kTrace) {
+            float4* dst = reinterpret_cast<float4*>(p.y_out + m * p.K + b * kG);
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              dst[c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
+          }
+        }
+        // rows past M and blocks past nb are padding of the tiled scale buffer: 0;
+        // the last pair also covers the padding blocks [2*nbp2, 4*nbp4)
+        uint8_t* sp = p.scales + scale_offset(m, b, p.nbp4);
+        *sp = static_cast<uint8_t>(valid ? sbyte : 0u);
+        if ((b & 3) < 2 && b + 2 >= 2 * static_cast<int64_t>(p.nbp2) && b + 2 < 4 * static_cast<int64_t>(p.nbp4))
+          sp[2] = 0;
+        // next unit of this set
+        pr += kSets;
+        while (pr >= npair) { pr -= npair; ++mt; }
       }
     }
   }
