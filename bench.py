@@ -325,7 +325,10 @@ def main():
     torch.cuda.synchronize()
 
     K_ = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K_)]
+    # Pass 1 (the headline): one event pair per step around both kernels. Nothing sits
+    # between them on the stream, so the GEMM, launched with programmatic stream
+    # serialization, does its set-up while the quantizer finishes.
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_)]
     sampler = ClockSampler(local)
     if not args.no_clocks and rank == 0:
         sampler.start()
@@ -335,17 +338,28 @@ def main():
     for i in range(K_):
         flush_l2(i)  # evict L2 between steps (outside the timed events)
         ev[i][0].record(stream)
-        bat.bat_quantize_act(X, A, B, gl, gh, Xq=Xq, stream=stream)
+        step()
         ev[i][1].record(stream)
-        bat.bat_mxfp4_gemm(Xq, Wq, Y=Y, out_dtype=torch.bfloat16, stream=stream)
-        ev[i][2].record(stream)
     torch.cuda.synchronize()
     if pg:
         pg.barrier()
     clocks = sampler.stop() if (not args.no_clocks and rank == 0) else None
-    t_pro = [ev[i][0].elapsed_time(ev[i][1]) * 1e-3 for i in range(K_)]
-    t_gemm = [ev[i][1].elapsed_time(ev[i][2]) * 1e-3 for i in range(K_)]
-    t_step, sp, sg = max_over_ranks(pg, [sum(t_pro) + sum(t_gemm), sum(t_pro), sum(t_gemm)], dev)
+    t_steps = [ev[i][0].elapsed_time(ev[i][1]) * 1e-3 for i in range(K_)]
+    # Pass 2 (per-kernel durations for the roofline fields): the same steps with an
+    # event between the two kernels, which also keeps them from overlapping.
+    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K_)]
+    torch.cuda.synchronize()
+    for i in range(K_):
+        flush_l2(i)
+        ev2[i][0].record(stream)
+        bat.bat_quantize_act(X, A, B, gl, gh, Xq=Xq, stream=stream)
+        ev2[i][1].record(stream)
+        bat.bat_mxfp4_gemm(Xq, Wq, Y=Y, out_dtype=torch.bfloat16, stream=stream)
+        ev2[i][2].record(stream)
+    torch.cuda.synchronize()
+    t_pro = [ev2[i][0].elapsed_time(ev2[i][1]) * 1e-3 for i in range(K_)]
+    t_gemm = [ev2[i][1].elapsed_time(ev2[i][2]) * 1e-3 for i in range(K_)]
+    t_step, sp, sg = max_over_ranks(pg, [sum(t_steps), sum(t_pro), sum(t_gemm)], dev)
     assert bat.bat_device_error() == 0, "a kernel reported a stalled wait"
 
     flop = 2.0 * w.M * w.N * w.K
@@ -400,7 +414,7 @@ def main():
             "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "out": "bf16",
                        "l2": "flushed between steps (256 MiB write + read outside the timed events)",
                        "parallelism": f"replicas x{world} (independent token batches)"},
-            "gpu_launches": 2 * K_ * world,
+            "gpu_launches": 2 * K_ * world,  # the timed pass: quantizer + GEMM per step
             "roofline": {"bound": "tensor", "achieved": gemm_tf, "peak": fp4_peak,
                          "unit": "TFLOP/s", "frac": gemm_tf / fp4_peak,
                          "traffic": recorded_traffic("bat_mxf4_gemm_kernel", w.name),

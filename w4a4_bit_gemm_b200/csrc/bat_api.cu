@@ -280,8 +280,20 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
   const int64_t tiles = ((p.M + bat::gemm::kBM - 1) / bat::gemm::kBM) *
                         ((p.N + bat::gemm::kBN - 1) / bat::gemm::kBN);
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  bat::bat_mxf4_gemm_kernel<<<grid, bat::gemm::kThreads, bat::gemm::kSmemBytes, stream>>>(ta, tb, ty, p);
-  return cuda_status(cudaGetLastError());
+  // Programmatic stream serialization: the kernel's set-up may overlap the previous
+  // kernel on the stream; it waits for that kernel's completion (griddepcontrol.wait)
+  // before touching the operands or Y, so the stream order of results is unchanged.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(bat::gemm::kThreads);
+  cfg.dynamicSmemBytes = bat::gemm::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, bat::bat_mxf4_gemm_kernel, ta, tb, ty, p));
 }
 
 bat_status_t check_gemm_args(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, const void* Y,

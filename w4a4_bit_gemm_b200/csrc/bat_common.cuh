@@ -96,6 +96,18 @@ __device__ __forceinline__ void setmaxnreg_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
 }
 
+// Programmatic dependent launch. A kernel launched with programmatic stream
+// serialization may start while the kernel before it on the stream is still
+// running; grid_dependency_wait() returns once that kernel has completed and its
+// memory operations are visible, so everything before it must not touch global
+// memory other kernels write. allow_dependents() lets the next such kernel start.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");

@@ -19,6 +19,8 @@
 //               (M=128, N=256, K=64) accumulating in TMEM;
 //   warps 10,11 idle (they complete the third warpgroup).
 // Every wait is bounded (see mbar_wait) and reports through the error word.
+// Launched with programmatic stream serialization, so barrier set-up and the TMEM
+// allocation overlap the end of the kernel before it (normally the quantizer).
 #pragma once
 
 #include "bat_common.cuh"
@@ -193,6 +195,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot_ptr;
+  // Everything above is local setup; the operands (and Y) belong to the kernels before.
+  grid_dependency_wait();
 
   const int64_t m_tiles = (p.M + kBM - 1) / kBM;
   const int64_t n_tiles = (p.N + kBN - 1) / kBN;

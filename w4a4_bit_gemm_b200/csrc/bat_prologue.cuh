@@ -266,6 +266,9 @@ __global__ void __launch_bounds__(pro::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot_ptr;
+  // The next kernel on the stream (normally the GEMM) may start its own set-up now;
+  // it waits for this grid to finish before it reads the codes.
+  allow_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
