@@ -316,7 +316,7 @@ def main():
         # write, then read, a buffer twice the L2: the next kernel starts with a cold L2
         # holding only clean lines of unrelated data (no write-back lands on it)
         flush.fill_(i & 0xFF)
-        flush_view.sum(dtype=torch.int64)
+        flush_view.amax()
 
     flush_view = flush.view(torch.int32)
     for i in range(args.warmup):
