@@ -23,9 +23,12 @@
  *   - P^-1 comes from a Gauss-Jordan inverse with partial pivoting, in fp64.
  *
  * Readings of points the pages leave open (all shared with the CUDA path only
- * through their written statement, never through code):
+ *   through their written statement, never through code):
  *   - x's 32 elements are read as a row-major 4x8 matrix X_r[i][p] = x[8i+p];
- *     then x P_b = vec_row(B_b^T X_r A).
+ *     then x P_b = vec_row(B_b^T X_r A). In general (the variant sweep over the
+ *     shared factor's size, note Key Designs 2 and the review's size study) A is
+ *     s x s and B_b is t x t with s t = 32, X_r[i][p] = x[s i + p], and
+ *     P_b[(s i + p)][(s j + q)] = B_b[i][j] A[p][q]; s = 8 is the default.
  *   - lo = fp32(r_lo * min), hi = fp32(r_hi * max), c = min(max(y, lo), hi)
  *     (hi wins if lo > hi); r = fp32 of the fp64 logistic function.
  *   - scale exponent e = floor(log2(amax)) - 2, clamped to [-127, 127]; amax = 0
@@ -53,26 +56,34 @@ static double bf16_bits_to_double(uint16_t h) {
   return (double)f;
 }
 
-/* Explicit Kronecker product: P[(8i+p)][(8j+q)] = B[i][j] * A[p][q]. */
-void orc_kron(const double* B /*4x4*/, const double* A /*8x8*/, double* P /*32x32*/) {
-  for (int i = 0; i < 4; ++i)
-    for (int j = 0; j < 4; ++j)
-      for (int p = 0; p < 8; ++p)
-        for (int q = 0; q < 8; ++q)
-          P[(8 * i + p) * 32 + (8 * j + q)] = B[i * 4 + j] * A[p * 8 + q];
+/* Explicit Kronecker product with an s x s shared factor A and a t x t private
+ * factor B (s t = 32): P[(s i + p)][(s j + q)] = B[i][j] * A[p][q]. */
+void orc_kron_gen(const double* B, const double* A, int s, double* P /*32x32*/) {
+  const int t = ORC_G / s;
+  for (int i = 0; i < t; ++i)
+    for (int j = 0; j < t; ++j)
+      for (int p = 0; p < s; ++p)
+        for (int q = 0; q < s; ++q)
+          P[(s * i + p) * 32 + (s * j + q)] = B[i * t + j] * A[p * s + q];
 }
 
-/* y = x . P_b for every row and block, fp64 result (not rounded). */
-void orc_transform_f64(const uint16_t* X, int64_t M, int64_t K, const float* A, const float* B,
-                       double* Y) {
+/* The default sizes: A 8x8, B 4x4. */
+void orc_kron(const double* B /*4x4*/, const double* A /*8x8*/, double* P /*32x32*/) {
+  orc_kron_gen(B, A, 8, P);
+}
+
+/* y = x . P_b for every row and block, fp64 result (not rounded); A is s x s and
+ * B holds nb blocks of t x t. */
+void orc_transform_f64_gen(const uint16_t* X, int64_t M, int64_t K, const float* A, int s,
+                           const float* B, double* Y) {
   const int64_t nb = K / ORC_G;
-  double Ad[64];
-  for (int t = 0; t < 64; ++t) Ad[t] = A[t];
+  const int t2 = (ORC_G / s) * (ORC_G / s);
+  double Ad[1024], Bd[1024];
+  for (int u = 0; u < s * s; ++u) Ad[u] = A[u];
   double* P = (double*)malloc(sizeof(double) * 1024 * (size_t)nb);
   for (int64_t b = 0; b < nb; ++b) {
-    double Bd[16];
-    for (int t = 0; t < 16; ++t) Bd[t] = B[b * 16 + t];
-    orc_kron(Bd, Ad, P + 1024 * b);
+    for (int u = 0; u < t2; ++u) Bd[u] = B[b * t2 + u];
+    orc_kron_gen(Bd, Ad, s, P + 1024 * b);
   }
 #pragma omp parallel for schedule(static)
   for (int64_t m = 0; m < M; ++m) {
@@ -90,13 +101,23 @@ void orc_transform_f64(const uint16_t* X, int64_t M, int64_t K, const float* A, 
   free(P);
 }
 
+void orc_transform_f64(const uint16_t* X, int64_t M, int64_t K, const float* A, const float* B,
+                       double* Y) {
+  orc_transform_f64_gen(X, M, K, A, 8, B, Y);
+}
+
 /* The "transformed values": the fp64 product rounded once to fp32. */
-void orc_transform(const uint16_t* X, int64_t M, int64_t K, const float* A, const float* B,
-                   float* Y) {
+void orc_transform_gen(const uint16_t* X, int64_t M, int64_t K, const float* A, int s,
+                       const float* B, float* Y) {
   double* Yd = (double*)malloc(sizeof(double) * (size_t)(M * K));
-  orc_transform_f64(X, M, K, A, B, Yd);
+  orc_transform_f64_gen(X, M, K, A, s, B, Yd);
   for (int64_t t = 0; t < M * K; ++t) Y[t] = (float)Yd[t];
   free(Yd);
+}
+
+void orc_transform(const uint16_t* X, int64_t M, int64_t K, const float* A, const float* B,
+                   float* Y) {
+  orc_transform_gen(X, M, K, A, 8, B, Y);
 }
 
 /* Clip ratio sigma(gamma) = 1 / (1 + exp(-gamma)), in fp64, rounded once to fp32. */
@@ -271,26 +292,27 @@ int orc_inverse(int n, const double* Min, double* Mout) {
 
 /* Weight side: row n, block b of W becomes w_b . (B_b^-T (x) A^-T), i.e. the
  * rows of (P^-1 W^T)^T = W P^-T. fp64 result, not rounded. Returns 0, or 1 if
- * A or some B_b is singular. */
-int orc_weight_transform_f64(const uint16_t* W, int64_t N, int64_t K, const float* A,
-                             const float* B, double* Wt) {
+ * A or some B_b is singular. A is s x s, B holds nb blocks of t x t. */
+int orc_weight_transform_f64_gen(const uint16_t* W, int64_t N, int64_t K, const float* A, int s,
+                                 const float* B, double* Wt) {
   const int64_t nb = K / ORC_G;
-  double Ad[64], Ainv[64], AinvT[64];
-  for (int t = 0; t < 64; ++t) Ad[t] = A[t];
-  if (orc_inverse(8, Ad, Ainv)) return 1;
-  for (int p = 0; p < 8; ++p)
-    for (int q = 0; q < 8; ++q) AinvT[p * 8 + q] = Ainv[q * 8 + p];
+  const int t = ORC_G / s;
+  double Ad[1024], Ainv[1024], AinvT[1024];
+  for (int u = 0; u < s * s; ++u) Ad[u] = A[u];
+  if (orc_inverse(s, Ad, Ainv)) return 1;
+  for (int p = 0; p < s; ++p)
+    for (int q = 0; q < s; ++q) AinvT[p * s + q] = Ainv[q * s + p];
   double* P = (double*)malloc(sizeof(double) * 1024 * (size_t)nb);
   for (int64_t b = 0; b < nb; ++b) {
-    double Bd[16], Binv[16], BinvT[16];
-    for (int t = 0; t < 16; ++t) Bd[t] = B[b * 16 + t];
-    if (orc_inverse(4, Bd, Binv)) {
+    double Bd[1024], Binv[1024], BinvT[1024];
+    for (int u = 0; u < t * t; ++u) Bd[u] = B[b * t * t + u];
+    if (orc_inverse(t, Bd, Binv)) {
       free(P);
       return 1;
     }
-    for (int i = 0; i < 4; ++i)
-      for (int j = 0; j < 4; ++j) BinvT[i * 4 + j] = Binv[j * 4 + i];
-    orc_kron(BinvT, AinvT, P + 1024 * b);
+    for (int i = 0; i < t; ++i)
+      for (int j = 0; j < t; ++j) BinvT[i * t + j] = Binv[j * t + i];
+    orc_kron_gen(BinvT, AinvT, s, P + 1024 * b);
   }
 #pragma omp parallel for schedule(static)
   for (int64_t n = 0; n < N; ++n)
@@ -306,6 +328,11 @@ int orc_weight_transform_f64(const uint16_t* W, int64_t N, int64_t K, const floa
     }
   free(P);
   return 0;
+}
+
+int orc_weight_transform_f64(const uint16_t* W, int64_t N, int64_t K, const float* A,
+                             const float* B, double* Wt) {
+  return orc_weight_transform_f64_gen(W, N, K, A, 8, B, Wt);
 }
 
 /* Threads the OpenMP loops above use (1 without OpenMP). */

@@ -44,6 +44,11 @@ def lib():
         L.orc_weight_transform_f64.argtypes = [P, I64, I64, P, P, P]
         L.orc_weight_transform_f64.restype = ctypes.c_int
         L.orc_kron.argtypes = [P, P, P]
+        L.orc_kron_gen.argtypes = [P, P, ctypes.c_int, P]
+        L.orc_transform_f64_gen.argtypes = [P, I64, I64, P, ctypes.c_int, P, P]
+        L.orc_transform_gen.argtypes = [P, I64, I64, P, ctypes.c_int, P, P]
+        L.orc_weight_transform_f64_gen.argtypes = [P, I64, I64, P, ctypes.c_int, P, P]
+        L.orc_weight_transform_f64_gen.restype = ctypes.c_int
         L.orc_num_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -57,12 +62,28 @@ def _c(a, dtype):
     return np.ascontiguousarray(a, dtype=dtype)
 
 
+SHARED_SIZES = (1, 2, 4, 8, 16, 32)
+
+
+def factor_sizes(A: np.ndarray, B: np.ndarray, K: Optional[int] = None) -> int:
+    """Shared size s of an (s x s) A with (K/32, 32/s, 32/s) private factors B."""
+    s = int(np.shape(A)[0])
+    if s not in SHARED_SIZES or np.shape(A) != (s, s):
+        raise ValueError(f"shared factor must be s x s with s in {SHARED_SIZES}")
+    t = G // s
+    nb = np.shape(B)[0] if K is None else K // G
+    if np.shape(B) != (nb, t, t):
+        raise ValueError(f"private factors must be ({nb}, {t}, {t})")
+    return s
+
+
 def kron_block(B: np.ndarray, A: np.ndarray) -> np.ndarray:
-    """The explicit 32x32 block P_b = B_b (x) A, fp64."""
+    """The explicit 32x32 block P_b = B_b (x) A, fp64 (A is s x s, B_b (32/s) x (32/s))."""
     B = _c(B, np.float64)
     A = _c(A, np.float64)
+    s = factor_sizes(A, B[None])
     P = np.empty((32, 32), np.float64)
-    lib().orc_kron(_p(B), _p(A), _p(P))
+    lib().orc_kron_gen(_p(B), _p(A), s, _p(P))
     return P
 
 
@@ -70,9 +91,11 @@ def transform_f64(X: np.ndarray, A: np.ndarray, B: np.ndarray) -> np.ndarray:
     """x . P_b for every row and 32-element block; fp64, unrounded."""
     X = _c(X, np.uint16)
     M, K = X.shape
-    assert K % G == 0 and B.shape == (K // G, 4, 4)
+    assert K % G == 0
+    s = factor_sizes(A, B, K)
     Y = np.empty((M, K), np.float64)
-    lib().orc_transform_f64(_p(X), M, K, _p(_c(A, np.float32)), _p(_c(B, np.float32)), _p(Y))
+    lib().orc_transform_f64_gen(_p(X), M, K, _p(_c(A, np.float32)), s,
+                                _p(_c(B, np.float32)), _p(Y))
     return Y
 
 
@@ -80,8 +103,11 @@ def transform(X: np.ndarray, A: np.ndarray, B: np.ndarray) -> np.ndarray:
     """The transformed values: fp64 product rounded once to fp32."""
     X = _c(X, np.uint16)
     M, K = X.shape
+    assert K % G == 0
+    s = factor_sizes(A, B, K)
     Y = np.empty((M, K), np.float32)
-    lib().orc_transform(_p(X), M, K, _p(_c(A, np.float32)), _p(_c(B, np.float32)), _p(Y))
+    lib().orc_transform_gen(_p(X), M, K, _p(_c(A, np.float32)), s,
+                            _p(_c(B, np.float32)), _p(Y))
     return Y
 
 
@@ -145,9 +171,10 @@ def inverse(Mtx: np.ndarray) -> np.ndarray:
 def weight_transform_f64(W: np.ndarray, A: np.ndarray, B: np.ndarray) -> np.ndarray:
     W = _c(W, np.uint16)
     N, K = W.shape
+    s = factor_sizes(A, B, K)
     out = np.empty((N, K), np.float64)
-    if lib().orc_weight_transform_f64(_p(W), N, K, _p(_c(A, np.float32)),
-                                      _p(_c(B, np.float32)), _p(out)):
+    if lib().orc_weight_transform_f64_gen(_p(W), N, K, _p(_c(A, np.float32)), s,
+                                          _p(_c(B, np.float32)), _p(out)):
         raise np.linalg.LinAlgError("singular factor")
     return out
 

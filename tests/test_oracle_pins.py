@@ -152,9 +152,9 @@ def test_block_locality():
 
 def test_inverse_roundtrip_and_library():
     rng = np.random.default_rng(3)
-    for n in (4, 8):
+    for n in (1, 2, 4, 8, 16, 32):
         for _ in range(20):
-            M = np.eye(n) + 0.3 * rng.standard_normal((n, n))
+            M = np.eye(n) + 0.3 * min(1.0, np.sqrt(8.0 / n)) * rng.standard_normal((n, n))
             inv = oracle.inverse(M)
             assert np.max(np.abs(inv @ M - np.eye(n))) < 1e-12
             assert np.allclose(inv, np.linalg.inv(M), rtol=1e-12, atol=1e-12)
@@ -353,3 +353,105 @@ def test_formats_roundtrip():
     nbp4 = 3
     assert I[0, 0] == 0 and I[1, 0] == 16 and I[32, 0] == 4 and I[0, 1] == 1
     assert I[0, 4] == 512 and I[128, 0] == nbp4 * 512 and I[31, 3] == 31 * 16 + 3
+
+
+# --- factor sizes other than 8 x 8 shared / 4 x 4 private --------------------------
+# The review's size study and the note's Key Designs 2 vary the shared factor's
+# size s (A is s x s, each B_b is (32/s) x (32/s)); s = 32 leaves one scalar per
+# block (a shared 32 x 32 transform, scaled), s = 1 a fully private 32 x 32 block.
+
+SIZES = (1, 2, 4, 8, 16, 32)
+
+
+@pytest.mark.parametrize("s", SIZES)
+def test_kron_block_all_sizes(s):
+    A, B, _, _ = wl.random_factors(2, seed=20 + s, shared=s)
+    t = 32 // s
+    A64 = A.astype(np.float64)
+    for b in range(2):
+        P = oracle.kron_block(B[b], A)
+        assert np.array_equal(P, np.kron(B[b].astype(np.float64), A64))
+        # block (i, j) of P is B_b[i][j] times A
+        i, j = t - 1, 0
+        assert np.array_equal(P[s * i:s * i + s, s * j:s * j + s], B[b][i, j] * A64)
+
+
+@pytest.mark.parametrize("s", SIZES)
+def test_transform_factored_all_sizes(s):
+    """x P_b equals the block-diagonal matmul and vec_row(B_b^T X_r A), X_r = x as t x s."""
+    nb, rows = 4, 24
+    A, B, _, _ = wl.random_factors(nb, seed=30 + s, shared=s)
+    t = 32 // s
+    X = wl.random_bf16((rows, 32 * nb), seed=31 + s, scale=3.0)
+    Xd = _bf16_to_f64(X)
+    Y = oracle.transform_f64(X, A, B)
+    P = scipy.linalg.block_diag(*[np.kron(B[b].astype(np.float64), A.astype(np.float64))
+                                  for b in range(nb)])
+    ref = Xd @ P
+    assert np.max(np.abs(Y - ref)) <= 1e-13 * np.max(np.abs(ref))
+    for b in range(nb):
+        Xr = Xd[:, 32 * b:32 * b + 32].reshape(rows, t, s)
+        fac = (B[b].astype(np.float64).T[None] @ Xr @ A.astype(np.float64)[None]).reshape(rows, 32)
+        assert np.max(np.abs(Y[:, 32 * b:32 * b + 32] - fac)) <= 1e-13 * np.max(np.abs(fac))
+    assert np.array_equal(oracle.transform(X, A, B), Y.astype(np.float32))
+
+
+@pytest.mark.parametrize("s", SIZES)
+def test_inverse_fusion_all_sizes(s):
+    nb = 4
+    A, B, _, _ = wl.random_factors(nb, seed=40 + s, shared=s)
+    X = wl.random_bf16((16, 32 * nb), seed=41 + s)
+    W = wl.random_bf16((8, 32 * nb), seed=42 + s)
+    got = oracle.transform_f64(X, A, B) @ oracle.weight_transform_f64(W, A, B).T
+    ref = _bf16_to_f64(X) @ _bf16_to_f64(W).T
+    assert np.linalg.norm(got - ref) <= 1e-10 * np.linalg.norm(ref)
+
+
+def test_extreme_sizes_closed_forms():
+    """s = 32: P_b = beta_b A; s = 1: P_b = alpha B_b."""
+    nb = 3
+    X = wl.random_bf16((8, 32 * nb), seed=50)
+    Xd = _bf16_to_f64(X).reshape(8, nb, 32)
+    A, B, _, _ = wl.random_factors(nb, seed=51, shared=32)
+    assert B.shape == (nb, 1, 1)
+    Y = oracle.transform_f64(X, A, B).reshape(8, nb, 32)
+    for b in range(nb):
+        ref = float(B[b, 0, 0]) * (Xd[:, b] @ A.astype(np.float64))
+        assert np.allclose(Y[:, b], ref, rtol=1e-13, atol=1e-13)
+    A, B, _, _ = wl.random_factors(nb, seed=52, shared=1)
+    assert A.shape == (1, 1)
+    Y = oracle.transform_f64(X, A, B).reshape(8, nb, 32)
+    for b in range(nb):
+        ref = float(A[0, 0]) * (Xd[:, b] @ B[b].astype(np.float64))
+        assert np.allclose(Y[:, b], ref, rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("s", SIZES)
+def test_block_hadamard_every_size(s):
+    """Normalised Sylvester Hadamards H_t/sqrt(t) (x) H_s/sqrt(s) = H_32/sqrt(32) for
+    every split, so each size gives BRQ's 32-point block rotation; the weight side
+    equals the activation side because that block is orthonormal and symmetric."""
+    t = 32 // s
+    A = (scipy.linalg.hadamard(s) / np.sqrt(s)).astype(np.float32)
+    nb = 4
+    B = np.repeat((scipy.linalg.hadamard(t) / np.sqrt(t))[None].astype(np.float32), nb, axis=0)
+    H32 = scipy.linalg.hadamard(32) / np.sqrt(32.0)
+    assert np.allclose(oracle.kron_block(B[0], A), H32, atol=1e-7)
+    X = wl.random_bf16((8, 32 * nb), seed=60 + s)
+    Y = oracle.transform_f64(X, A, B)
+    Xd = _bf16_to_f64(X)
+    assert np.allclose(Y.reshape(8, nb, 32), Xd.reshape(8, nb, 32) @ H32, atol=1e-5)
+    assert np.allclose(oracle.weight_transform_f64(X, A, B), Y, rtol=1e-6, atol=1e-6)
+
+
+def test_factor_shape_errors():
+    A, B, _, _ = wl.random_factors(2, seed=70, shared=4)
+    X = wl.random_bf16((2, 64), seed=71)
+    with pytest.raises(ValueError):
+        oracle.transform_f64(X, A, B[:, :2, :2])
+    with pytest.raises(ValueError):
+        oracle.transform_f64(X, np.eye(3, dtype=np.float32), B)
+    with pytest.raises(np.linalg.LinAlgError):
+        Bs = B.copy()
+        Bs[1] = 0.0
+        oracle.weight_transform_f64(X, A, Bs)

@@ -124,11 +124,21 @@ def make_inputs(name: str, seed: int = 0, M: Optional[int] = None, N: Optional[i
     return Inputs(f32_to_bf16_bits(x), f32_to_bf16_bits(w), A, B, g_lo, g_hi, chans)
 
 
-def random_factors(nb: int, seed: int) -> tuple[np.ndarray, np.ndarray, np.ndarray, np.ndarray]:
-    """A, B, gamma_lo, gamma_hi with the standard recipe, for ad-hoc shapes."""
+def random_factors(nb: int, seed: int, shared: int = 8
+                   ) -> tuple[np.ndarray, np.ndarray, np.ndarray, np.ndarray]:
+    """A, B, gamma_lo, gamma_hi with the standard recipe, for ad-hoc shapes.
+
+    ``shared`` is the size s of the shared factor A (s x s); the private
+    factors are (32/s) x (32/s). An n x n factor is I + c N(0,1) with
+    c = 0.1 min(1, sqrt(8/n)), so the 16 and 32 sizes stay as well conditioned
+    as the default 8 and 4 ones; with s = 8 the draws are the default ones.
+    """
     rng = np.random.Generator(np.random.PCG64(seed))
-    A = (np.eye(8) + 0.1 * rng.standard_normal((8, 8))).astype(np.float32)
-    B = (np.eye(4)[None] + 0.1 * rng.standard_normal((nb, 4, 4))).astype(np.float32)
+    t = 32 // shared
+    ca = 0.1 * min(1.0, np.sqrt(8.0 / shared))
+    cb = 0.1 * min(1.0, np.sqrt(8.0 / t))
+    A = (np.eye(shared) + ca * rng.standard_normal((shared, shared))).astype(np.float32)
+    B = (np.eye(t)[None] + cb * rng.standard_normal((nb, t, t))).astype(np.float32)
     g_lo = rng.uniform(1.0, 4.0, size=nb).astype(np.float32)
     g_hi = rng.uniform(1.0, 4.0, size=nb).astype(np.float32)
     return A, B, g_lo, g_hi
