@@ -255,6 +255,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--shared", type=int, default=8, choices=[1, 2, 4, 8, 16, 32],
+                    help="size s of the shared transform factor (A s x s, each B_b 32/s x 32/s)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -291,14 +293,32 @@ def main():
         return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev)
 
     X = bf16(X_host)
-    A, B = f32(inp.A), f32(inp.B)
     gl, gh = f32(inp.g_lo), f32(inp.g_hi)
+    stream = torch.cuda.current_stream(dev)
+    if args.shared == 8:
+        A, B = f32(inp.A), f32(inp.B)
+
+        def quantize(Xin, out):
+            bat.bat_quantize_act(Xin, A, B, gl, gh, Xq=out, stream=stream)
+
+        def prepare(Win):
+            return bat.bat_prepare_weight(Win, A, B)
+    else:
+        # another split of the 32 channels: factors of the standard recipe at that size
+        inp.A, inp.B, _, _ = wl.random_factors(w.K // 32, seed=1, shared=args.shared)
+        A, B = f32(inp.A), f32(inp.B)
+
+        def quantize(Xin, out):
+            bat.bat_quantize_act_gpk(Xin, A, B, gl, gh, Xq=out, stream=stream)
+
+        def prepare(Win):
+            return bat.bat_prepare_weight_gpk(Win, A, B)
     Wdev = bf16(inp.W)
-    bat.bat_prepare_weight(Wdev, A, B)  # first call: module load, attributes
+    prepare(Wdev)  # first call: module load, attributes
     torch.cuda.synchronize()
     wp0, wp1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     wp0.record()
-    Wq = bat.bat_prepare_weight(Wdev, A, B)  # offline weight side, timed for information only
+    Wq = prepare(Wdev)  # offline weight side, timed for information only
     wp1.record()
     torch.cuda.synchronize()
     prep_ms = wp0.elapsed_time(wp1)
@@ -306,10 +326,9 @@ def main():
     Xq = bat.MXFP4.empty(w.M, w.K, dev)
     Y = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
 
     def step():
-        bat.bat_quantize_act(X, A, B, gl, gh, Xq=Xq, stream=stream)
+        quantize(X, Xq)
         bat.bat_mxfp4_gemm(Xq, Wq, Y=Y, out_dtype=torch.bfloat16, stream=stream)
 
     def flush_l2(i):
@@ -352,7 +371,7 @@ def main():
     for i in range(K_):
         flush_l2(i)
         ev2[i][0].record(stream)
-        bat.bat_quantize_act(X, A, B, gl, gh, Xq=Xq, stream=stream)
+        quantize(X, Xq)
         ev2[i][1].record(stream)
         bat.bat_mxfp4_gemm(Xq, Wq, Y=Y, out_dtype=torch.bfloat16, stream=stream)
         ev2[i][2].record(stream)
@@ -380,8 +399,12 @@ def main():
 
         def e2e_step():
             Xdev.copy_(Xh, non_blocking=True)
-            bat.bat_linear(Xdev, Wq, A, B, gl, gh, Y=Y, out_dtype=torch.bfloat16, workspace=ws,
-                           stream=stream)
+            if args.shared == 8:
+                bat.bat_linear(Xdev, Wq, A, B, gl, gh, Y=Y, out_dtype=torch.bfloat16,
+                               workspace=ws, stream=stream)
+            else:
+                quantize(Xdev, Xq)
+                bat.bat_mxfp4_gemm(Xq, Wq, Y=Y, out_dtype=torch.bfloat16, stream=stream)
             Yh.copy_(Y, non_blocking=True)
 
         for _ in range(3):
@@ -412,6 +435,8 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "mxfp4", "data": "synthetic",
             "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "out": "bf16",
+                       "transform": f"GPK A {args.shared}x{args.shared} shared, "
+                                    f"B_b {32 // args.shared}x{32 // args.shared} private",
                        "l2": "flushed between steps (256 MiB write + read outside the timed events)",
                        "parallelism": f"replicas x{world} (independent token batches)"},
             "gpu_launches": 2 * K_ * world,  # the timed pass: quantizer + GEMM per step

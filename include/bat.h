@@ -19,9 +19,9 @@
  *
  * Conventions for every entry point:
  *   - Tensor pointers are DEVICE pointers owned by the caller. The online entry
- *     points never allocate device memory; the offline bat_prepare_weight
- *     allocates (and frees, stream-ordered) one temporary of 256 + 64*K/32 bytes
- *     for the inverted factors. No state is kept between calls except a sticky
+ *     points never allocate device memory; the offline bat_prepare_weight(_gpk)
+ *     allocates (and frees, stream-ordered) one temporary of about
+ *     4*s*s + 4*K*32/s bytes for the inverted factors. No state is kept between calls except a sticky
  *     device error word (see bat_device_error).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
  *     asynchronous on it unless stated otherwise.
@@ -149,6 +149,46 @@ BAT_API bat_status_t bat_e2m1_encode(const float* v, int64_t n, uint8_t* codes, 
 BAT_API bat_status_t bat_prepare_weight(const void* W, int64_t N, int64_t K, const float* A,
                                 const float* B, const float* gw_lo, const float* gw_hi,
                                 const bat_mxfp4_t* Wq, float* wt_out, void* stream);
+
+/*
+ * The same two transforms with the 32 channels of a block split another way
+ * (the shared/private size sweep of the BATQuant note, Key Designs 2 "GPK
+ * decomposition", and the size study in the nubint.ai review): A is s x s and
+ * shared by every block, each B_b is t x t with t = 32 / s, and
+ *   P_b = B_b (x) A,  P_b[s i + p][s j + q] = B_b[i][j] * A[p][q],
+ * so x P_b = vec_row(B_b^T X_r A) with X_r the t x s row-major view of the
+ * block. s = 8 is bat_quantize_act / bat_prepare_weight; s = 32 is one shared
+ * 32 x 32 transform scaled per block; s = 1 is a fully private 32 x 32 block.
+ *
+ *   shared : s, one of 1, 2, 4, 8, 16, 32 (anything else: BAT_ERR_UNSUPPORTED).
+ *   A      : device fp32 [s][s] row-major, 16-byte aligned.
+ *   B      : device fp32 [K/32][t][t] row-major, 16-byte aligned.
+ *   y_out  : optional device fp32 [M][K] trace of the transformed values
+ *            (NULL to skip), as in bat_quantize_act_trace.
+ * All other arguments, requirements and errors are those of bat_quantize_act
+ * and bat_prepare_weight (the weight side inverts A and every B_b in fp64 on
+ * the host and synchronizes `stream`).
+ */
+BAT_API bat_status_t bat_quantize_act_gpk(const void* X, int64_t M, int64_t K, const float* A,
+                                          int shared, const float* B, const float* g_lo,
+                                          const float* g_hi, const bat_mxfp4_t* Xq, float* y_out,
+                                          void* stream);
+BAT_API bat_status_t bat_prepare_weight_gpk(const void* W, int64_t N, int64_t K, const float* A,
+                                            int shared, const float* B, const float* gw_lo,
+                                            const float* gw_hi, const bat_mxfp4_t* Wq,
+                                            float* wt_out, void* stream);
+
+/*
+ * Factors of the block Hadamard rotation (the BRQ article, "Block Rotation"):
+ * every 32-channel block is rotated by H_32 / sqrt(32), the normalised
+ * Sylvester Hadamard matrix, which is H_t/sqrt(t) (x) H_s/sqrt(s) for any split
+ * s t = 32. Writes A = H_s / sqrt(s) ([s][s]) and B_b = H_t / sqrt(t) for
+ * b < nb ([nb][t][t]) to HOST buffers (H_n[i][j] = (-1)^popcount(i & j)). Feed
+ * them (copied to the device) to the _gpk calls with the same s. Pure host code:
+ * no CUDA call. Errors: BAT_ERR_UNSUPPORTED for another s, BAT_ERR_INVALID_ARG
+ * for null buffers or nb < 1.
+ */
+BAT_API bat_status_t bat_block_hadamard_factors(int shared, int64_t nb, float* A, float* B);
 
 /*
  * Block-scaled MXFP4 GEMM on the 5th-generation tensor cores (tcgen05,

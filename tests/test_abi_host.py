@@ -84,3 +84,34 @@ def test_host_validation_returns_before_cuda(L):
     # element conversion / ratios: bad sizes
     assert L.bat_e2m1_encode(p, 0, p, None) == 1
     assert L.bat_clip_ratios(p, 0, p, None) == 1
+
+
+def test_gpk_host_validation(L):
+    S = bat.MXFP4Struct
+    good = S(0x7F0000100000, 0x7F0000200000, 4, 64)
+    p = _fake_ptr()
+    # unsupported shared sizes are rejected before anything else
+    for s in (0, 3, 5, 64, -8):
+        assert L.bat_quantize_act_gpk(p, 4, 64, p, s, p, None, None, ctypes.byref(good), None,
+                                      None) == 6
+        assert L.bat_prepare_weight_gpk(p, 4, 64, p, s, p, None, None, ctypes.byref(good), None,
+                                        None) == 6
+    assert L.bat_quantize_act_gpk(None, 4, 64, p, 4, p, None, None, ctypes.byref(good), None,
+                                  None) == 1
+    assert L.bat_quantize_act_gpk(p, 4, 64, p, 4, p, None, None, ctypes.byref(good), _fake_ptr(4),
+                                  None) == 3
+
+
+def test_block_hadamard_factors_host():
+    """Host-only helper: H_s/sqrt(s) and H_t/sqrt(t) in Sylvester order (scipy's)."""
+    import numpy as np
+    import scipy.linalg
+    for s in (1, 2, 4, 8, 16, 32):
+        A, B = bat.bat_block_hadamard_factors(s, 3)
+        t = 32 // s
+        assert np.array_equal(A.numpy(), (scipy.linalg.hadamard(s) / np.sqrt(s)).astype(np.float32))
+        for b in range(3):
+            assert np.array_equal(B[b].numpy(),
+                                  (scipy.linalg.hadamard(t) / np.sqrt(t)).astype(np.float32))
+    with pytest.raises(bat.BatError):
+        bat.bat_block_hadamard_factors(3, 2)

@@ -183,6 +183,119 @@ def test_prepare_weight_singular(bat):
     assert e.value.status == 4
 
 
+
+# ---------------------------------------------------------------- other factor splits
+SHARED_SIZES = (1, 2, 4, 8, 16, 32)
+
+
+def _check_act_gpk(bat, X, A, B, g_lo, g_hi):
+    rows, K = X.shape
+    nb = K // 32
+    Xd, Ad, Bd = _dev_bf16(X), _dev_f32(A), _dev_f32(B)
+    gl = None if g_lo is None else _dev_f32(g_lo)
+    gh = None if g_hi is None else _dev_f32(g_hi)
+    y = torch.empty(rows, K, dtype=torch.float32, device="cuda")
+    Xq = bat.bat_quantize_act_gpk(Xd, Ad, Bd, gl, gh, y_out=y)
+    Xq2 = bat.bat_quantize_act_gpk(Xd, Ad, Bd, gl, gh)
+    torch.cuda.synchronize()
+    assert torch.equal(Xq.codes, Xq2.codes) and torch.equal(Xq.scales, Xq2.scales)
+    y_gpu = y.cpu().numpy()
+    _check_transform(y_gpu, oracle.transform(X, A, B))
+    r_lo = bat.bat_clip_ratios(gl, nb).cpu().numpy()
+    r_hi = bat.bat_clip_ratios(gh, nb).cpu().numpy()
+    oc, os_, bad = oracle.quantize(y_gpu, r_lo, r_hi)
+    assert bad == 0
+    codes, scales, tiled = _host(Xq, rows, K)
+    assert np.array_equal(codes, oc)
+    assert np.array_equal(scales, os_)
+    assert np.all(tiled[formats.padding_mask(rows, nb)] == 0)
+    return Xq, y_gpu
+
+
+@pytest.mark.parametrize("s", SHARED_SIZES)
+@pytest.mark.parametrize("M,K", [(130, 1056), (3, 4128), (257, 256)])
+def test_quantize_act_gpk_sizes(bat, s, M, K):
+    X = wl.random_bf16((M, K), seed=M + K + s, scale=3.0)
+    A, B, g_lo, g_hi = wl.random_factors(K // 32, seed=K + s, shared=s)
+    _check_act_gpk(bat, X, A, B, g_lo, g_hi)
+
+
+def test_quantize_act_gpk_default_split_matches(bat):
+    """s = 8 through the generic entry point is bat_quantize_act, bit for bit."""
+    inp = wl.make_inputs("tiny", with_weight=False)
+    Xd, Ad, Bd = _dev_bf16(inp.X), _dev_f32(inp.A), _dev_f32(inp.B)
+    gl, gh = _dev_f32(inp.g_lo), _dev_f32(inp.g_hi)
+    q1 = bat.bat_quantize_act(Xd, Ad, Bd, gl, gh)
+    q2 = bat.bat_quantize_act_gpk(Xd, Ad, Bd, gl, gh)
+    torch.cuda.synchronize()
+    assert torch.equal(q1.codes, q2.codes) and torch.equal(q1.scales, q2.scales)
+
+
+@pytest.mark.parametrize("s", SHARED_SIZES)
+def test_prepare_weight_gpk_sizes(bat, s):
+    N, K = 136, 1056
+    W = wl.random_bf16((N, K), seed=N + K + s, scale=0.02)
+    A, B, _, _ = wl.random_factors(K // 32, seed=K + 1 + s, shared=s)
+    rng = np.random.default_rng(s)
+    gw_lo = rng.uniform(1, 4, size=(N, K // 32)).astype(np.float32)
+    gw_hi = rng.uniform(1, 4, size=(N, K // 32)).astype(np.float32)
+    wt = torch.empty(N, K, dtype=torch.float32, device="cuda")
+    Wq = bat.bat_prepare_weight_gpk(_dev_bf16(W), _dev_f32(A), _dev_f32(B), _dev_f32(gw_lo),
+                                    _dev_f32(gw_hi), wt_out=wt)
+    torch.cuda.synchronize()
+    wt_gpu = wt.cpu().numpy()
+    _check_transform(wt_gpu, oracle.weight_transform_f64(W, A, B).astype(np.float32))
+    r_lo = oracle.clip_ratios(gw_lo.reshape(-1)).reshape(N, -1)
+    r_hi = oracle.clip_ratios(gw_hi.reshape(-1)).reshape(N, -1)
+    oc, os_, _ = oracle.quantize(wt_gpu, r_lo, r_hi, per_row=True)
+    codes, scales, tiled = _host(Wq, N, K)
+    assert np.array_equal(codes, oc)
+    assert np.array_equal(scales, os_)
+
+
+def test_gpk_errors(bat):
+    X = torch.zeros(4, 64, dtype=torch.bfloat16, device="cuda")
+    A = torch.eye(3, device="cuda")
+    B = torch.eye(4, device="cuda").repeat(2, 1, 1).contiguous()
+    Xq = bat.MXFP4.empty(4, 64)
+    st = bat.lib().bat_quantize_act_gpk(bat._ptr(X), 4, 64, bat._ptr(A), 3, bat._ptr(B), None, None,
+                                        bat.ctypes.byref(Xq.struct()), None, bat._stream(None))
+    assert st == 6  # BAT_ERR_UNSUPPORTED
+    A, B, _, _ = wl.random_factors(2, seed=3, shared=2)
+    B[1] = 0.0
+    with pytest.raises(bat.BatError) as e:
+        bat.bat_prepare_weight_gpk(_dev_bf16(wl.random_bf16((8, 64), seed=4)), _dev_f32(A), _dev_f32(B))
+    assert e.value.status == 4
+    assert bat.bat_device_error() == 0
+
+
+def test_block_hadamard_mode(bat):
+    """Every split of the normalised Sylvester Hadamard gives the same 32-point block
+    rotation (the BRQ article's block rotation), in fp32 to the bit: the factor
+    products are powers of two times fp32(1/sqrt 2) or exact. Checked against the
+    oracle, and the whole linear layer against the oracle's fp64 product."""
+    M, N, K = 200, 264, 1056
+    X = wl.random_bf16((M, K), seed=5, scale=3.0)
+    W = wl.random_bf16((N, K), seed=6, scale=0.02)
+    nb = K // 32
+    outs = []
+    for s in SHARED_SIZES:
+        A, B = bat.bat_block_hadamard_factors(s, nb)
+        Xq, y = _check_act_gpk(bat, X, A.numpy(), B.numpy(), None, None)
+        outs.append((Xq, y))
+    for Xq, y in outs[1:]:
+        assert torch.equal(Xq.codes, outs[0][0].codes) and torch.equal(Xq.scales, outs[0][0].scales)
+        assert np.array_equal(y, outs[0][1])
+    A, B = bat.bat_block_hadamard_factors(4, nb)
+    Wq = bat.bat_prepare_weight_gpk(_dev_bf16(W), A.cuda(), B.cuda())
+    Y = bat.bat_mxfp4_gemm(outs[2][0], Wq, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ref = oracle.linear(X, W, A.numpy(), B.numpy(), None, None)
+    rel = np.linalg.norm(Y.cpu().numpy() - ref) / np.linalg.norm(ref)
+    assert rel <= 1e-2, rel  # codes may differ where the two transforms round to a tie
+    # and exactly, on the GPU's own codes
+    _gemm_check(bat, outs[2][0], Wq, M, N, K)
+
 # ---------------------------------------------------------------- GEMM
 def _gemm_check(bat, Xq, Wq, M, N, K, rows=None, cols=None):
     xc, xs, _ = _host(Xq, M, K)

@@ -64,6 +64,9 @@ def lib() -> ctypes.CDLL:
         "bat_clip_ratios": (S, [P, I64, P, P]),
         "bat_e2m1_encode": (S, [P, I64, P, P]),
         "bat_prepare_weight": (S, [P, I64, I64, P, P, P, P, SP, P, P]),
+        "bat_quantize_act_gpk": (S, [P, I64, I64, P, S, P, P, P, SP, P, P]),
+        "bat_prepare_weight_gpk": (S, [P, I64, I64, P, S, P, P, P, SP, P, P]),
+        "bat_block_hadamard_factors": (S, [S, I64, P, P]),
         "bat_mxfp4_gemm": (S, [SP, SP, P, S, P]),
         "bat_linear_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
         "bat_linear": (S, [P, I64, SP, P, P, P, P, P, S, P, ctypes.c_size_t, P]),
@@ -227,6 +230,66 @@ def bat_prepare_weight(W, A, B, gw_lo=None, gw_hi=None, Wq: Optional[MXFP4] = No
                                     ctypes.byref(st), _ptr(wt_out), _stream(stream)),
            "bat_prepare_weight")
     return Wq
+
+
+def _gpk_factors(A, B, K):
+    s = A.shape[0] if isinstance(A, torch.Tensor) and A.dim() == 2 else 0
+    t = 32 // s if s else 0
+    _need(A, torch.float32, "A", (s, s))
+    _need(B, torch.float32, "B", (K // 32, t, t))
+    return s
+
+
+def bat_quantize_act_gpk(X, A, B, g_lo=None, g_hi=None, Xq: Optional[MXFP4] = None,
+                         y_out: Optional[torch.Tensor] = None, stream=None) -> MXFP4:
+    """Activation side with an s x s shared factor A and (32/s) x (32/s) private B_b."""
+    M, K = X.shape
+    _need(X, torch.bfloat16, "X")
+    s = _gpk_factors(A, B, K)
+    if (g_lo is None) != (g_hi is None):
+        raise ValueError("g_lo and g_hi must both be given or both be None")
+    if g_lo is not None:
+        _need(g_lo, torch.float32, "g_lo", (K // 32,))
+        _need(g_hi, torch.float32, "g_hi", (K // 32,))
+    if y_out is not None:
+        _need(y_out, torch.float32, "y_out", (M, K))
+    Xq = MXFP4.empty(M, K, X.device) if Xq is None else Xq
+    st = Xq.struct()
+    _check(lib().bat_quantize_act_gpk(_ptr(X), M, K, _ptr(A), s, _ptr(B), _ptr(g_lo), _ptr(g_hi),
+                                      ctypes.byref(st), _ptr(y_out), _stream(stream)),
+           "bat_quantize_act_gpk")
+    return Xq
+
+
+def bat_prepare_weight_gpk(W, A, B, gw_lo=None, gw_hi=None, Wq: Optional[MXFP4] = None,
+                           wt_out: Optional[torch.Tensor] = None, stream=None) -> MXFP4:
+    """Weight side for the factor split of ``bat_quantize_act_gpk``."""
+    N, K = W.shape
+    _need(W, torch.bfloat16, "W")
+    s = _gpk_factors(A, B, K)
+    if (gw_lo is None) != (gw_hi is None):
+        raise ValueError("gw_lo and gw_hi must both be given or both be None")
+    if gw_lo is not None:
+        _need(gw_lo, torch.float32, "gw_lo", (N, K // 32))
+        _need(gw_hi, torch.float32, "gw_hi", (N, K // 32))
+    if wt_out is not None:
+        _need(wt_out, torch.float32, "wt_out", (N, K))
+    Wq = MXFP4.empty(N, K, W.device) if Wq is None else Wq
+    st = Wq.struct()
+    _check(lib().bat_prepare_weight_gpk(_ptr(W), N, K, _ptr(A), s, _ptr(B), _ptr(gw_lo),
+                                        _ptr(gw_hi), ctypes.byref(st), _ptr(wt_out),
+                                        _stream(stream)), "bat_prepare_weight_gpk")
+    return Wq
+
+
+def bat_block_hadamard_factors(shared: int, nb: int):
+    """Host (CPU) fp32 factors A = H_s/sqrt(s), B_b = H_t/sqrt(t) of the block Hadamard rotation."""
+    t = 32 // shared if shared in (1, 2, 4, 8, 16, 32) else 1
+    A = torch.empty(shared, shared, dtype=torch.float32) if shared > 0 else torch.empty(1)
+    B = torch.empty(max(nb, 1), t, t, dtype=torch.float32)
+    _check(lib().bat_block_hadamard_factors(shared, nb, _ptr(A), _ptr(B)),
+           "bat_block_hadamard_factors")
+    return A, B
 
 
 def _out_code(out_dtype: torch.dtype) -> int:

@@ -198,7 +198,8 @@ bat_status_t check_act_args(const void* X, int64_t M, int64_t K, const float* A,
 
 bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float* A,
                              const float* B, const float* g_lo, const float* g_hi, bool per_row,
-                             const bat_mxfp4_t* out, float* y_out, cudaStream_t stream) {
+                             const bat_mxfp4_t* out, float* y_out, cudaStream_t stream,
+                             int ls = 3) {
   int dev = 0, sms = 0;
   bat_status_t st = current_device(&dev, &sms);
   if (st != BAT_OK) return st;
@@ -216,6 +217,7 @@ bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float
   p.rows = rows;
   p.K = K;
   p.nb = static_cast<int>(K / 32);
+  p.ls = ls;
   p.nbp2 = (p.nb + 1) / 2;
   p.nbp4 = (p.nb + 3) / 4;
   p.mtiles = (rows + bat::pro::kTok - 1) / bat::pro::kTok;
@@ -375,9 +377,30 @@ bat_status_t bat_clip_ratios(const float* g, int64_t n, float* r, void* stream) 
 
 bat_status_t bat_e2m1_encode(const float* v, int64_t n, uint8_t* codes, void* stream);
 
-bat_status_t bat_prepare_weight(const void* W, int64_t N, int64_t K, const float* A,
-                                const float* B, const float* gw_lo, const float* gw_hi,
-                                const bat_mxfp4_t* Wq, float* wt_out, void* stream) {
+// log2 of a supported shared-factor size (1, 2, 4, ..., 32), or -1.
+static int shared_log2(int shared) {
+  for (int l = 0; l <= 5; ++l)
+    if (shared == (1 << l)) return l;
+  return -1;
+}
+
+bat_status_t bat_quantize_act_gpk(const void* X, int64_t M, int64_t K, const float* A, int shared,
+                                  const float* B, const float* g_lo, const float* g_hi,
+                                  const bat_mxfp4_t* Xq, float* y_out, void* stream) {
+  const int ls = shared_log2(shared);
+  if (ls < 0) return BAT_ERR_UNSUPPORTED;
+  bat_status_t st = check_act_args(X, M, K, A, B, g_lo, g_hi, Xq);
+  if (st != BAT_OK) return st;
+  if (y_out && !aligned16(y_out)) return BAT_ERR_ALIGN;
+  return launch_prologue(X, M, K, A, B, g_lo, g_hi, false, Xq, y_out,
+                         static_cast<cudaStream_t>(stream), ls);
+}
+
+bat_status_t bat_prepare_weight_gpk(const void* W, int64_t N, int64_t K, const float* A, int shared,
+                                    const float* B, const float* gw_lo, const float* gw_hi,
+                                    const bat_mxfp4_t* Wq, float* wt_out, void* stream) {
+  const int ls = shared_log2(shared);
+  if (ls < 0) return BAT_ERR_UNSUPPORTED;
   if (!W || !A || !B || !Wq) return BAT_ERR_INVALID_ARG;
   if ((gw_lo == nullptr) != (gw_hi == nullptr)) return BAT_ERR_INVALID_ARG;
   if (N < 1 || K < 32) return BAT_ERR_INVALID_ARG;
@@ -390,29 +413,36 @@ bat_status_t bat_prepare_weight(const void* W, int64_t N, int64_t K, const float
   st = current_device(&dev, &sms);
   if (st != BAT_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int sa = shared, tb = 32 / shared;
   const int64_t nb = K / 32;
-  std::vector<float> ha(64), hb(static_cast<size_t>(nb) * 16);
-  if (cudaMemcpyAsync(ha.data(), A, 64 * sizeof(float), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+  std::vector<float> ha(static_cast<size_t>(sa) * sa), hb(static_cast<size_t>(nb) * tb * tb);
+  if (cudaMemcpyAsync(ha.data(), A, ha.size() * sizeof(float), cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
       cudaMemcpyAsync(hb.data(), B, hb.size() * sizeof(float), cudaMemcpyDeviceToHost, s) !=
           cudaSuccess ||
       cudaStreamSynchronize(s) != cudaSuccess)
     return BAT_ERR_CUDA;
   // Inverse-transposed factors: w_b (B_b^-T (x) A^-T) = vec_row(B_b^-1 W_r A^-T), which the
-  // prologue computes as vec_row(F_b^T W_r G) with G = A^-T and F_b = B_b^-T.
-  std::vector<float> fac(64 + static_cast<size_t>(nb) * 16);
+  // prologue computes as vec_row(F_b^T W_r G) with G = A^-T and F_b = B_b^-T. G is padded to
+  // a multiple of four floats so that the F_b start 16-byte aligned.
+  const size_t a_len = (static_cast<size_t>(sa) * sa + 3) & ~size_t{3};
+  std::vector<float> fac(a_len + hb.size(), 0.0f);
   {
-    double a[64], inv[64];
-    for (int i = 0; i < 64; ++i) a[i] = ha[i];
-    if (!invert(8, a, inv)) return BAT_ERR_SINGULAR;
-    for (int p = 0; p < 8; ++p)
-      for (int q = 0; q < 8; ++q) fac[p * 8 + q] = static_cast<float>(inv[q * 8 + p]);
+    std::vector<double> a(ha.begin(), ha.end()), inv(ha.size());
+    if (!invert(sa, a.data(), inv.data())) return BAT_ERR_SINGULAR;
+    for (int p = 0; p < sa; ++p)
+      for (int q = 0; q < sa; ++q) fac[p * sa + q] = static_cast<float>(inv[q * sa + p]);
   }
-  for (int64_t b = 0; b < nb; ++b) {
-    double m[16], inv[16];
-    for (int i = 0; i < 16; ++i) m[i] = hb[b * 16 + i];
-    if (!invert(4, m, inv)) return BAT_ERR_SINGULAR;
-    for (int i = 0; i < 4; ++i)
-      for (int j = 0; j < 4; ++j) fac[64 + b * 16 + i * 4 + j] = static_cast<float>(inv[j * 4 + i]);
+  {
+    std::vector<double> m(static_cast<size_t>(tb) * tb), inv(m.size());
+    for (int64_t b = 0; b < nb; ++b) {
+      const float* src = hb.data() + b * tb * tb;
+      for (int i = 0; i < tb * tb; ++i) m[i] = src[i];
+      if (!invert(tb, m.data(), inv.data())) return BAT_ERR_SINGULAR;
+      float* dst = fac.data() + a_len + b * tb * tb;
+      for (int i = 0; i < tb; ++i)
+        for (int j = 0; j < tb; ++j) dst[i * tb + j] = static_cast<float>(inv[j * tb + i]);
+    }
   }
   // Offline only: one temporary device buffer for the inverse factors (stream-ordered).
   void* dfac = nullptr;
@@ -421,12 +451,34 @@ bat_status_t bat_prepare_weight(const void* W, int64_t N, int64_t K, const float
                                    cudaMemcpyHostToDevice, s));
   if (st == BAT_OK) {
     const float* da = static_cast<const float*>(dfac);
-    st = launch_prologue(W, N, K, da, da + 64, gw_lo, gw_hi, true, Wq, wt_out, s);
+    st = launch_prologue(W, N, K, da, da + a_len, gw_lo, gw_hi, true, Wq, wt_out, s, ls);
   }
   cudaFreeAsync(dfac, s);
   // `fac` is read by the async copy: wait before it goes out of scope.
   if (cudaStreamSynchronize(s) != cudaSuccess) return BAT_ERR_CUDA;
   return st;
+}
+
+bat_status_t bat_prepare_weight(const void* W, int64_t N, int64_t K, const float* A,
+                                const float* B, const float* gw_lo, const float* gw_hi,
+                                const bat_mxfp4_t* Wq, float* wt_out, void* stream) {
+  return bat_prepare_weight_gpk(W, N, K, A, 8, B, gw_lo, gw_hi, Wq, wt_out, stream);
+}
+
+bat_status_t bat_block_hadamard_factors(int shared, int64_t nb, float* A, float* B) {
+  const int ls = shared_log2(shared);
+  if (ls < 0) return BAT_ERR_UNSUPPORTED;
+  if (!A || !B || nb < 1) return BAT_ERR_INVALID_ARG;
+  // Sylvester order: H_n[i][j] = (-1)^popcount(i & j), normalised by 1/sqrt(n).
+  auto fill = [](int n, float* h) {
+    const float c = static_cast<float>(1.0 / std::sqrt(static_cast<double>(n)));
+    for (int i = 0; i < n; ++i)
+      for (int j = 0; j < n; ++j) h[i * n + j] = (__builtin_popcount(i & j) & 1) ? -c : c;
+  };
+  const int tb = 32 / shared;
+  fill(shared, A);
+  for (int64_t b = 0; b < nb; ++b) fill(tb, B + b * tb * tb);
+  return BAT_OK;
 }
 
 bat_status_t bat_mxfp4_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,

@@ -49,21 +49,29 @@ constexpr int kStageBytes = kTok * 128;          // 128 rows x 64 bf16: 16 KB
 constexpr int kPTermBytes = 32 * 32 * 2;         // one bf16 term of one block's P: 2 KB
 constexpr int kPBlockBytes = 3 * kPTermBytes;    // one block's three terms: 6 KB
 constexpr int kPPairBytes = kBlk * kPBlockBytes; // 12 KB
-constexpr int kPBytes = kStrip * kPPairBytes;    // one strip: 96 KB
+constexpr int kPBytes = kStrip * kPPairBytes;    // one strip: 48 KB
 constexpr int kSets = 2;                         // quantizer sets (alternate units)
 constexpr int kSetWarps = 4 * kBlk;              // lane quarters x blocks
 constexpr int kThreads = 32 * (2 + kSets * kSetWarps);
 constexpr int kBuilders = kThreads - 32;         // every warp but the producer
-constexpr int kBarBytes = 2048;                  // barriers, TMEM address, clip ratios, A, B
-constexpr int kSmemBytes = kStages * kStageBytes + kPBytes + kBarBytes + 1024;
+constexpr int kBarBytes = 2048;                  // barriers, TMEM address, clip ratios
+// A and the strip's B_b staged for the P build: s*s + 2*kStrip*(32/s)^2 floats, at most
+// 2052 (s = 2); the fully private split (s = 1, 8193 floats) reads them from global memory
+constexpr int kFacFloats = 2112;
+constexpr bool fac_fits(int ls) {
+  return ls > 5 || (((1 << (2 * ls)) + 3) / 4 * 4 + 2 * kStrip * (1 << (10 - 2 * ls)) <= kFacFloats &&
+                    fac_fits(ls + 1));
+}
+static_assert(fac_fits(1), "the staged factors of every split s >= 2 fit the staging area");
+constexpr int kSmemBytes = kStages * kStageBytes + kPBytes + kBarBytes + 4 * kFacFloats + 1024;
 constexpr int kSlotCols = 96;                    // one block's accumulator: 3 terms x 32 columns
 constexpr uint32_t kAccCols = kBlk * kSlotCols;  // one unit's accumulator: 192 columns
 constexpr uint32_t kTmemCols = 512;              // allocation (power of two) holding 2 x 192
 }  // namespace pro
 
 struct PrologueParams {
-  const float* a;        // fp32 [8][8]
-  const float* b;        // fp32 [nb][4][4]
+  const float* a;        // fp32 [s][s], shared factor (s = 1 << ls)
+  const float* b;        // fp32 [nb][32/s][32/s], private factors
   const float* g_lo;     // clip logits: [nb] (shared by rows) or [rows][nb]; may be null
   const float* g_hi;
   uint8_t* codes;        // [rows][K/2]
@@ -77,6 +85,7 @@ struct PrologueParams {
   int64_t mtiles;        // ceil(rows / 128)
   int strips;            // ceil(nbp2 / kStrip)
   int cps;               // CTAs per strip (grid = strips * cps)
+  int ls;                // log2 of the shared factor's size: 0..5 (3 is the 8 x 8 / 4 x 4 split)
 };
 
 // fp32(sigma(g)) evaluated in fp64; +inf gives exactly 1.
@@ -125,21 +134,27 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
 // The three bf16 terms of P_b for block b, in the MMA's B-operand layout (N x K,
 // K-major, no swizzle: 8x8 core matrices of 128 bytes, K-adjacent ones 128 bytes
 // apart, N-adjacent ones 512 bytes apart; the terms follow one another, so the
-// three together are one N=96 operand). Operand element (n, k) is
-// P_b[k][n] = B_b[k/8][n/8] * A[k%8][n%8]; a block past nb gets 0.
-// `row` in [0, 128) picks n = row/4 and the eight k of core-matrix column row%4:
-// one 16-byte row of a core matrix per term. `a` is A (8x8) and `bb` is B_b (4x4,
-// zeros for a block past nb), both staged in shared memory.
-__device__ __forceinline__ void build_p_row(uint8_t* dst, const float* a, const float* bb, int row) {
+// three together are one N=96 operand). With A of size s x s (s = 1 << ls) and
+// B_b of size t x t (t = 32 / s), operand element (n, k) is
+// P_b[k][n] = B_b[k/s][n/s] * A[k%s][n%s], rounded once to fp32 and split
+// exactly into three bf16 terms. `row` in [0, 128) picks n = row/4 and the eight
+// k of core-matrix column row%4: one 16-byte row of a core matrix per term.
+// `a` and `bb` point at A and B_b, staged in shared memory or in global memory;
+// `bb` is null for a block past nb, which gets 0.
+__device__ __forceinline__ void build_p_row(uint8_t* dst, const float* a, const float* bb, int ls,
+                                            int row) {
   const int n = row >> 2, kc = row & 3;
+  const int sm = (1 << ls) - 1, t = 32 >> ls;
+  const int an = n & sm, bn = n >> ls;
   uint32_t w[3][4];
-  const float bv = bb[kc * 4 + (n >> 3)];  // B_b[k/8][n/8], k/8 = kc
 #pragma unroll
   for (int i = 0; i < 8; i += 2) {
     uint32_t hh[2], mm[2], ll[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const float prod = __fmul_rn(bv, a[(i + h) * 8 + (n & 7)]);  // A[k%8][n%8]
+      const int k = kc * 8 + i + h;
+      const float bv = bb ? bb[(k >> ls) * t + bn] : 0.0f;
+      const float prod = __fmul_rn(bv, a[((k & sm) << ls) + an]);
       const uint32_t hi = bf16_bits(prod);
       const float r1 = prod - __uint_as_float(hi << 16);
       const uint32_t mid = bf16_bits(r1);
@@ -225,9 +240,11 @@ __global__ void __launch_bounds__(pro::kThreads, 1)
       reinterpret_cast<volatile uint32_t*>(base_ptr + (tmem_slot - base));
   // clip ratios of the strip's blocks: [2 * kStrip] lo, then [2 * kStrip] hi
   float* ratios = reinterpret_cast<float*>(base_ptr + (bars - base) + 256);
-  // A and the strip's B_b, staged for the P build
-  float* sA = reinterpret_cast<float*>(base_ptr + (bars - base) + 512);
-  float* sB = sA + 64;  // [2 * kStrip][16]
+  // A and the strip's B_b, staged for the P build (s > 1): A [s][s], then [2 * kStrip][t][t]
+  const bool staged = p.ls > 0;
+  const int fa = 1 << (2 * p.ls), fb = 1 << (10 - 2 * p.ls);  // s*s and t*t
+  float* sA = reinterpret_cast<float*>(base_ptr + (bars - base) + kBarBytes);
+  float* sB = sA + ((fa + 3) & ~3);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -312,13 +329,14 @@ __global__ void __launch_bounds__(pro::kThreads, 1)
     // ------------------------------------------------ P terms and clip ratios
     {
       const int t = threadIdx.x - 32;
-      // stage A and the strip's B_b with one coalesced load each
-      if (t < 64) {
-        sA[t] = p.a[t];
-      } else if (t < 64 + 32 * npair) {
-        const int64_t e = 2 * static_cast<int64_t>(pair_base) * 16 + (t - 64);  // [block][16]
-        sB[t - 64] = e < static_cast<int64_t>(p.nb) * 16 ? p.b[e] : 0.0f;
-      } else if (!kPerRowClip && t >= 320 && t < 320 + 2 * npair) {
+      // stage A and the strip's B_b with coalesced loads (zeros for blocks past nb)
+      if (staged) {
+        for (int i = t; i < fa; i += kBuilders) sA[i] = p.a[i];
+        const int64_t e0 = 2 * static_cast<int64_t>(pair_base) * fb;
+        const int64_t e_end = static_cast<int64_t>(p.nb) * fb;
+        for (int i = t; i < 2 * npair * fb; i += kBuilders) sB[i] = e0 + i < e_end ? p.b[e0 + i] : 0.0f;
+      }
+      if (!kPerRowClip && t >= 320 && t < 320 + 2 * npair) {
         const int lb = t - 320;
         const int64_t blk = 2 * static_cast<int64_t>(pair_base) + lb;
         const bool ok = blk < p.nb;
@@ -331,8 +349,17 @@ __global__ void __launch_bounds__(pro::kThreads, 1)
       for (int r = t; r < npair * 2 * 128; r += kBuilders) {
         const int pr = r >> 8, jj = (r >> 7) & 1;
         const bool used = nv >= npair || ((pr - pr0 + npair) % npair) < nv;
-        if (used)
-          build_p_row(pbase_ptr + pr * kPPairBytes + jj * kPBlockBytes, sA, sB + (2 * pr + jj) * 16, r & 127);
+        if (!used) continue;
+        uint8_t* dst = pbase_ptr + pr * kPPairBytes + jj * kPBlockBytes;
+        if (p.ls == 3) {  // the default split, with its shifts folded into constants
+          build_p_row(dst, sA, sB + (2 * pr + jj) * 16, 3, r & 127);
+        } else if (staged) {
+          build_p_row(dst, sA, sB + (2 * pr + jj) * fb, p.ls, r & 127);
+        } else {
+          const int blk = 2 * (pair_base + pr) + jj;
+          build_p_row(dst, p.a, blk < p.nb ? p.b + static_cast<int64_t>(blk) * fb : nullptr, p.ls,
+                      r & 127);
+        }
       }
       fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor cores
       mbar_arrive(pfull);
