@@ -36,6 +36,11 @@
  *   - a clipped value that is exactly zero encodes as +0 (code 0x0); any other
  *     value keeps its sign bit, so a negative value that rounds to zero is 0x8.
  *   - ties on the grid go to the even code (mantissa bit 0); |v| > 6 gives 6.
+ *   - MXFP8 activations (the W4A8 settings; "MXFP8 uses E4M3", note, Loss &
+ *     Training): OCP E4M3 elements (bias 7, no infinities, largest finite 448),
+ *     same UE8M0 scale per 32 with e = floor(log2(amax)) - 8 (8 is E4M3's
+ *     largest exponent), nearest code with ties to the even code, |v| > 448
+ *     gives 448, and the same zero and sign rules as MXFP4.
  */
 #include <math.h>
 #ifdef _OPENMP
@@ -158,10 +163,48 @@ double orc_e2m1_value(uint8_t code) {
   return (code & 8) ? -m : m;
 }
 
-/* Quantize one 32-element block of transformed values. Returns 0, or 1 if the
- * block holds a non-finite value (outside the contract; scale byte 0xFF). */
-int orc_quantize_block(const float* y, float r_lo, float r_hi, uint8_t* codes, uint8_t* scale,
-                       float* clipped /* nullable, 32 */) {
+/* E4M3 value of a non-negative code c (0..126): exponent field c >> 3 with bias
+ * 7, three mantissa bits; field 0 is subnormal (m/8 * 2^-6). */
+double orc_e4m3_value(uint8_t code) {
+  const int c = code & 0x7F;
+  if (c == 0x7F) return NAN;
+  const int ef = c >> 3, m = c & 7;
+  const double mag = ef == 0 ? ldexp(m / 8.0, -6) : ldexp(1.0 + m / 8.0, ef - 7);
+  return (code & 0x80) ? -mag : mag;
+}
+
+/* E4M3 encoder: nearest of the 127 finite magnitudes by exhaustive search, ties
+ * to the even code, saturating at 448. Returns 0xFF (a NaN code) for NaN input. */
+uint8_t orc_e4m3_encode(float v) {
+  if (isnan(v)) return 0xFF;
+  const double a = fabs((double)v);
+  int best = 0;
+  double best_d = fabs(a - orc_e4m3_value(0));
+  for (int c = 1; c < 127; ++c) {
+    const double d = fabs(a - orc_e4m3_value((uint8_t)c));
+    if (d < best_d || (d == best_d && (c % 2 == 0) && (best % 2 != 0))) {
+      best = c;
+      best_d = d;
+    }
+  }
+  if (a > 448.0) best = 126;
+  return (uint8_t)(best | (signbit(v) ? 0x80 : 0));
+}
+
+void orc_e4m3_encode_array(const float* v, int64_t n, uint8_t* codes) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < n; ++t) codes[t] = orc_e4m3_encode(v[t]);
+}
+
+/* Element formats of the quantizer: the largest exponent of the element type
+ * sets the scale, e = floor(log2 amax) - emax. */
+enum { ORC_E2M1 = 0, ORC_E4M3 = 1 };
+
+/* Quantize one 32-element block of transformed values into `fmt` elements.
+ * Returns 0, or 1 if the block holds a non-finite value (outside the contract;
+ * scale byte 0xFF). */
+int orc_quantize_block_fmt(const float* y, float r_lo, float r_hi, int fmt, uint8_t* codes,
+                           uint8_t* scale, float* clipped /* nullable, 32 */) {
   float mn = y[0], mx = y[0];
   for (int k = 0; k < 32; ++k) {
     if (!isfinite(y[k])) {
@@ -190,17 +233,22 @@ int orc_quantize_block(const float* y, float r_lo, float r_hi, uint8_t* codes, u
   } else {
     int ex;
     frexpf(amax, &ex); /* amax = m * 2^ex, m in [0.5, 1): floor(log2 amax) = ex - 1 */
-    e = (ex - 1) - 2;
+    e = (ex - 1) - (fmt == ORC_E4M3 ? 8 : 2);
     if (e < -127) e = -127;
     if (e > 127) e = 127;
   }
   *scale = (uint8_t)(e + 127);
   for (int k = 0; k < 32; ++k) {
     float v = ldexpf(c[k], -e);
-    codes[k] = orc_e2m1_encode(v);
+    codes[k] = fmt == ORC_E4M3 ? orc_e4m3_encode(v) : orc_e2m1_encode(v);
     if (clipped) clipped[k] = c[k];
   }
   return 0;
+}
+
+int orc_quantize_block(const float* y, float r_lo, float r_hi, uint8_t* codes, uint8_t* scale,
+                       float* clipped /* nullable, 32 */) {
+  return orc_quantize_block_fmt(y, r_lo, r_hi, ORC_E2M1, codes, scale, clipped);
 }
 
 /* Quantize a [rows][K] matrix of transformed values, one ratio pair per block
@@ -208,8 +256,9 @@ int orc_quantize_block(const float* y, float r_lo, float r_hi, uint8_t* codes, u
  * (per_row != 0: r_lo[rows][nb]). Codes come out one per byte [rows][K]
  * (unpacked); scales plain row-major [rows][nb]. Returns the number of
  * non-finite blocks. */
-int64_t orc_quantize_matrix(const float* Y, int64_t rows, int64_t K, const float* r_lo,
-                            const float* r_hi, int per_row, uint8_t* codes, uint8_t* scales) {
+int64_t orc_quantize_matrix_fmt(const float* Y, int64_t rows, int64_t K, const float* r_lo,
+                                const float* r_hi, int per_row, int fmt, uint8_t* codes,
+                                uint8_t* scales) {
   const int64_t nb = K / ORC_G;
   int64_t bad = 0;
 #pragma omp parallel for schedule(static) reduction(+ : bad)
@@ -218,24 +267,35 @@ int64_t orc_quantize_matrix(const float* Y, int64_t rows, int64_t K, const float
       const int64_t ri = per_row ? m * nb + b : b;
       const float rl = r_lo ? r_lo[ri] : 1.0f;
       const float rh = r_hi ? r_hi[ri] : 1.0f;
-      bad += orc_quantize_block(Y + m * K + b * 32, rl, rh, codes + m * K + b * 32,
-                                scales + m * nb + b, NULL);
+      bad += orc_quantize_block_fmt(Y + m * K + b * 32, rl, rh, fmt, codes + m * K + b * 32,
+                                    scales + m * nb + b, NULL);
     }
   }
   return bad;
 }
 
-/* Dequantize: value = grid(code) * 2^(scale - 127). */
-void orc_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t K,
-                    double* out) {
+int64_t orc_quantize_matrix(const float* Y, int64_t rows, int64_t K, const float* r_lo,
+                            const float* r_hi, int per_row, uint8_t* codes, uint8_t* scales) {
+  return orc_quantize_matrix_fmt(Y, rows, K, r_lo, r_hi, per_row, ORC_E2M1, codes, scales);
+}
+
+/* Dequantize: value = element(code) * 2^(scale - 127), elements E2M1 or E4M3. */
+void orc_dequantize_fmt(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t K,
+                        int fmt, double* out) {
   const int64_t nb = K / ORC_G;
 #pragma omp parallel for schedule(static)
   for (int64_t m = 0; m < rows; ++m)
     for (int64_t k = 0; k < K; ++k) {
       const uint8_t s = scales[m * nb + k / 32];
       const double sc = (s == 0xFF) ? NAN : ldexp(1.0, (int)s - 127);
-      out[m * K + k] = orc_e2m1_value(codes[m * K + k]) * sc;
+      const uint8_t c = codes[m * K + k];
+      out[m * K + k] = (fmt == ORC_E4M3 ? orc_e4m3_value(c) : orc_e2m1_value(c)) * sc;
     }
+}
+
+void orc_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t K,
+                    double* out) {
+  orc_dequantize_fmt(codes, scales, rows, K, ORC_E2M1, out);
 }
 
 /* Y[i][j] = sum_k Xd[rows[i]][k] * Wd[cols[j]][k] in fp64, serial sum per output

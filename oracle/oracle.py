@@ -16,6 +16,8 @@ from . import build as _build
 
 G = 32
 GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+# element formats of the quantizer (the C side's ORC_E2M1 / ORC_E4M3)
+FORMATS = {"e2m1": 0, "e4m3": 1}
 
 _lib = None
 
@@ -50,6 +52,12 @@ def lib():
         L.orc_weight_transform_f64_gen.argtypes = [P, I64, I64, P, ctypes.c_int, P, P]
         L.orc_weight_transform_f64_gen.restype = ctypes.c_int
         L.orc_num_threads.restype = ctypes.c_int
+        L.orc_e4m3_encode_array.argtypes = [P, I64, P]
+        L.orc_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_value.restype = ctypes.c_double
+        L.orc_quantize_matrix_fmt.argtypes = [P, I64, I64, P, P, ctypes.c_int, ctypes.c_int, P, P]
+        L.orc_quantize_matrix_fmt.restype = I64
+        L.orc_dequantize_fmt.argtypes = [P, P, I64, I64, ctypes.c_int, P]
         _lib = L
     return _lib
 
@@ -134,28 +142,41 @@ def e2m1_value(codes: np.ndarray) -> np.ndarray:
     return np.where(codes & 8, -mag, mag)
 
 
+def e4m3_encode(v: np.ndarray) -> np.ndarray:
+    v = _c(v, np.float32)
+    out = np.empty(v.shape, np.uint8)
+    lib().orc_e4m3_encode_array(_p(v), v.size, _p(out))
+    return out
+
+
+def e4m3_value(codes: np.ndarray) -> np.ndarray:
+    table = np.array([lib().orc_e4m3_value(c) for c in range(256)])
+    return table[np.asarray(codes, np.uint8)]
+
+
 def quantize(Y: np.ndarray, r_lo: Optional[np.ndarray], r_hi: Optional[np.ndarray],
-             per_row: bool = False):
-    """Clip + MXFP4-quantize fp32 transformed values. Returns (codes, scales, n_bad)."""
+             per_row: bool = False, fmt: str = "e2m1"):
+    """Clip + MX-quantize fp32 transformed values (E2M1 = MXFP4, E4M3 = MXFP8).
+    Returns (codes, scales, n_bad); codes one per byte."""
     Y = _c(Y, np.float32)
     rows, K = Y.shape
     codes = np.empty((rows, K), np.uint8)
     scales = np.empty((rows, K // G), np.uint8)
     rl = None if r_lo is None else _c(r_lo, np.float32)
     rh = None if r_hi is None else _c(r_hi, np.float32)
-    bad = lib().orc_quantize_matrix(_p(Y), rows, K, _p(rl), _p(rh), int(per_row),
-                                    _p(codes), _p(scales))
+    bad = lib().orc_quantize_matrix_fmt(_p(Y), rows, K, _p(rl), _p(rh), int(per_row),
+                                        FORMATS[fmt], _p(codes), _p(scales))
     return codes, scales, int(bad)
 
 
 def quantize_act(X: np.ndarray, A: np.ndarray, B: np.ndarray, g_lo: Optional[np.ndarray],
-                 g_hi: Optional[np.ndarray]):
-    """The whole online activation path: transform, clip, MXFP4 quantize."""
+                 g_hi: Optional[np.ndarray], fmt: str = "e2m1"):
+    """The whole online activation path: transform, clip, MX quantize."""
     nb = X.shape[1] // G
     Y = transform(X, A, B)
     r_lo = clip_ratios(g_lo, nb)
     r_hi = clip_ratios(g_hi, nb)
-    codes, scales, _ = quantize(Y, r_lo, r_hi)
+    codes, scales, _ = quantize(Y, r_lo, r_hi, fmt=fmt)
     return Y, codes, scales
 
 
@@ -190,12 +211,12 @@ def prepare_weight(W: np.ndarray, A: np.ndarray, B: np.ndarray,
     return Wt, codes, scales
 
 
-def dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+def dequantize(codes: np.ndarray, scales: np.ndarray, fmt: str = "e2m1") -> np.ndarray:
     codes = _c(codes, np.uint8)
     scales = _c(scales, np.uint8)
     rows, K = codes.shape
     out = np.empty((rows, K), np.float64)
-    lib().orc_dequantize(_p(codes), _p(scales), rows, K, _p(out))
+    lib().orc_dequantize_fmt(_p(codes), _p(scales), rows, K, FORMATS[fmt], _p(out))
     return out
 
 
@@ -212,11 +233,12 @@ def gemm_sampled(Xd: np.ndarray, Wd: np.ndarray, rows: Optional[Sequence[int]] =
     return Y
 
 
-def linear(X, W, A, B, g_lo, g_hi, rows=None, cols=None):
-    """Y = Q(XP) Q(P^-1 W^T) in fp64, optionally on a sample of outputs."""
-    _, xc, xs = quantize_act(X, A, B, g_lo, g_hi)
+def linear(X, W, A, B, g_lo, g_hi, rows=None, cols=None, act_fmt: str = "e2m1"):
+    """Y = Q(XP) Q(P^-1 W^T) in fp64, optionally on a sample of outputs; activations
+    in MXFP4 (W4A4) or MXFP8 E4M3 (W4A8), weights in MXFP4."""
+    _, xc, xs = quantize_act(X, A, B, g_lo, g_hi, fmt=act_fmt)
     _, wc, ws = prepare_weight(W, A, B)
-    return gemm_sampled(dequantize(xc, xs), dequantize(wc, ws), rows, cols)
+    return gemm_sampled(dequantize(xc, xs, act_fmt), dequantize(wc, ws), rows, cols)
 
 
 def gpk_param_counts(K: int, shared: int = 8, private: int = 4) -> dict:

@@ -455,3 +455,103 @@ def test_factor_shape_errors():
         Bs = B.copy()
         Bs[1] = 0.0
         oracle.weight_transform_f64(X, A, Bs)
+
+
+# --- MXFP8 (E4M3) activations: the W4A8 settings ------------------------------------
+# The note (Loss & Training) names W4A8 with "MXFP8 uses E4M3"; the element format
+# is OCP FP8 E4M3 (bias 7, no infinities, 448 the largest finite value).
+
+def test_e4m3_decode_table_matches_torch():
+    import torch
+    dec = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    mine = oracle.e4m3_value(np.arange(256))
+    fin = np.isfinite(dec)
+    assert np.array_equal(np.isfinite(mine), fin)
+    assert np.array_equal(mine[fin], dec[fin].astype(np.float64))
+    assert mine[0x7E] == 448.0 and mine[0x01] == 2.0 ** -9 and mine[0x08] == 2.0 ** -6
+
+
+def _e4m3_edges() -> np.ndarray:
+    """Every midpoint between adjacent finite E4M3 magnitudes, one fp32 ulp either
+    side of it, and the magnitudes themselves."""
+    mags = oracle.e4m3_value(np.arange(127)).astype(np.float32)
+    mids = ((mags[:-1].astype(np.float64) + mags[1:]) / 2).astype(np.float32)
+    pts = np.concatenate([mags, mids, np.nextafter(mids, np.float32(np.inf)),
+                          np.nextafter(mids, np.float32(0))])
+    return np.concatenate([pts, -pts]).astype(np.float32)
+
+
+def test_e4m3_encode_matches_torch():
+    """RNE conversion against torch's float8_e4m3fn cast (a library routine) for
+    |v| <= 448 plus the tie at 464; torch turns larger values into NaN, the oracle
+    saturates them to 448 (checked separately)."""
+    import torch
+    rng = np.random.default_rng(7)
+    top = int(np.float32(448.0).view(np.uint32))
+    bits = rng.integers(0, top + 1, size=1 << 20, dtype=np.uint32)
+    bits[: 1 << 19] |= np.uint32(0x80000000)
+    v = np.concatenate([bits.view(np.float32), _e4m3_edges(), np.float32([464.0, -464.0, 0.0, -0.0])])
+    got = oracle.e4m3_encode(v)
+    want = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, (v[bad[:5]], got[bad[:5]], want[bad[:5]])
+    big = np.float32([464.5, 480.0, 512.0, 1e6, 3.4e38, -500.0])
+    assert np.array_equal(oracle.e4m3_encode(big), np.uint8([0x7E] * 5 + [0xFE]))
+
+
+def _e4m3_by_binade(v: np.ndarray) -> np.ndarray:
+    """E4M3 as a 3-mantissa-bit float, written independently: below 2^-6 the step is
+    2^-9, in [2^k, 2^(k+1)) it is 2^(k-3); np.rint ties to even; saturate at 448."""
+    a = np.abs(v.astype(np.float64))
+    with np.errstate(divide="ignore"):
+        k = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    step = np.where(a < 2.0 ** -6, 2.0 ** -9, np.exp2(k - 3))
+    q = np.minimum(np.rint(a / step) * step, 448.0)
+    table = oracle.e4m3_value(np.arange(127))
+    code = np.searchsorted(table, q).astype(np.uint8)
+    assert np.all(table[code] == q)
+    return code | (np.signbit(v).astype(np.uint8) << 7)
+
+
+def test_e4m3_encode_by_binade():
+    rng = np.random.default_rng(8)
+    v = np.concatenate([(rng.standard_normal(1 << 18) * np.exp2(rng.uniform(-12, 10, 1 << 18))),
+                        rng.uniform(-600, 600, 1 << 16)]).astype(np.float32)
+    v = np.concatenate([v, _e4m3_edges()])
+    assert np.array_equal(oracle.e4m3_encode(v), _e4m3_by_binade(v))
+
+
+def test_mxfp8_scale_rule_and_rtn():
+    """Identity factors and no clip: MXFP8 RTN of X by an independent numpy quantizer;
+    the block maximum lands in [256, 512) times the scale (e = floor(log2 amax) - 8)."""
+    inp = wl.make_inputs("tiny")
+    nb = inp.B.shape[0]
+    A = np.eye(8, dtype=np.float32)
+    B = np.repeat(np.eye(4, dtype=np.float32)[None], nb, axis=0)
+    Y, codes, scales = oracle.quantize_act(inp.X, A, B, None, None, fmt="e4m3")
+    x = wl.bf16_bits_to_f32(inp.X)
+    rows, K = x.shape
+    blocks = x.reshape(rows, nb, 32).astype(np.float64)
+    amax = np.abs(blocks).max(axis=2)
+    e = np.clip(np.floor(np.log2(amax)) - 8, -127, 127)
+    assert np.array_equal(scales.astype(np.int64) - 127, e.astype(np.int64))
+    v = (blocks / np.exp2(e)[..., None]).astype(np.float32).reshape(rows, K)
+    v = np.where(v == 0, np.float32(0.0), v)
+    assert np.array_equal(codes, _e4m3_by_binade(v))
+    ratio = amax / np.exp2(e)
+    assert np.all((ratio >= 256) & (ratio < 512))
+    deq = oracle.dequantize(codes, scales, "e4m3")
+    rel = np.abs(deq - x) / np.repeat(amax, 32, axis=1)
+    # a half step of the top binade is at most amax / 16; a block maximum in [448, 512) x 2^e
+    # saturates to 448 x 2^e, at most amax / 8 away
+    assert rel.max() <= 2.0 ** -3
+
+
+def test_mxfp8_linear_error_below_mxfp4():
+    """W4A8 sits between W4A4 and the unquantized product (the settings' ordering)."""
+    inp = wl.make_inputs("tiny")
+    ref = _bf16_to_f64(inp.X) @ _bf16_to_f64(inp.W).T
+    e4 = np.linalg.norm(oracle.linear(inp.X, inp.W, inp.A, inp.B, inp.g_lo, inp.g_hi) - ref)
+    e8 = np.linalg.norm(oracle.linear(inp.X, inp.W, inp.A, inp.B, inp.g_lo, inp.g_hi,
+                                      act_fmt="e4m3") - ref)
+    assert e8 < e4
