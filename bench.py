@@ -29,8 +29,11 @@ import numpy as np  # noqa: E402
 import workloads as wl  # noqa: E402
 
 METRIC = "W4A4 BAT linear TFLOP/s (% FP4 peak); act-quant prologue GB/s (% HBM)"
+METRIC_W4A8 = "W4A8 BAT linear TFLOP/s (% FP8 peak); act-quant prologue GB/s (% HBM)"
 PROLOGUE_BYTES_PER_ELT = 2.0 + 0.5 + 1.0 / 32.0  # bf16 in, 4-bit code out, 1/32 scale byte
+PROLOGUE8_BYTES_PER_ELT = 2.0 + 1.0 + 1.0 / 32.0  # bf16 in, E4M3 code out, 1/32 scale byte
 FP4_OVER_BF16 = 9.0 / 2.25  # nominal dense FP4 / BF16 tensor throughput on B200
+FP8_OVER_BF16 = 4.5 / 2.25  # nominal dense FP8 (and FP8 x FP4) / BF16
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 
@@ -158,7 +161,7 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- CPU oracle leg
-def oracle_sample(inp, w, budget_s: float, seed: int = 0):
+def oracle_sample(inp, w, budget_s: float, seed: int = 0, act_fmt: str = "e2m1"):
     """Time the oracle (as it stands) on a bounded sample of the layer.
 
     The sample is `rows` token rows against `cols` weight rows: the oracle's
@@ -174,8 +177,8 @@ def oracle_sample(inp, w, budget_s: float, seed: int = 0):
     def run(rows, cols):
         t0 = time.perf_counter()
         X = inp.X[rows]
-        _, xc, xs = oracle.quantize_act(X, inp.A, inp.B, inp.g_lo, inp.g_hi)
-        Xd = oracle.dequantize(xc, xs)
+        _, xc, xs = oracle.quantize_act(X, inp.A, inp.B, inp.g_lo, inp.g_hi, fmt=act_fmt)
+        Xd = oracle.dequantize(xc, xs, act_fmt)
         oracle.gemm_sampled(Xd, Wd, None, cols)
         return time.perf_counter() - t0
 
@@ -257,6 +260,8 @@ def main():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--shared", type=int, default=8, choices=[1, 2, 4, 8, 16, 32],
                     help="size s of the shared transform factor (A s x s, each B_b 32/s x 32/s)")
+    ap.add_argument("--act", default="mxfp4", choices=["mxfp4", "mxfp8"],
+                    help="activation format: MXFP4 (W4A4) or MXFP8 E4M3 (W4A8)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -295,7 +300,19 @@ def main():
     X = bf16(X_host)
     gl, gh = f32(inp.g_lo), f32(inp.g_hi)
     stream = torch.cuda.current_stream(dev)
-    if args.shared == 8:
+    a8 = args.act == "mxfp8"
+    if a8:
+        # W4A8: MXFP8 activations through the E4M3 quantizer, MXFP4 weights
+        if args.shared != 8:
+            inp.A, inp.B, _, _ = wl.random_factors(w.K // 32, seed=1, shared=args.shared)
+        A, B = f32(inp.A), f32(inp.B)
+
+        def quantize(Xin, out):
+            bat.bat_quantize_act_mxfp8(Xin, A, B, gl, gh, Xq=out, stream=stream)
+
+        def prepare(Win):
+            return bat.bat_prepare_weight_gpk(Win, A, B)
+    elif args.shared == 8:
         A, B = f32(inp.A), f32(inp.B)
 
         def quantize(Xin, out):
@@ -323,13 +340,14 @@ def main():
     torch.cuda.synchronize()
     prep_ms = wp0.elapsed_time(wp1)
     del Wdev
-    Xq = bat.MXFP4.empty(w.M, w.K, dev)
+    Xq = (bat.MXFP8 if a8 else bat.MXFP4).empty(w.M, w.K, dev)
     Y = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    gemm_fn = bat.bat_w4a8_gemm if a8 else bat.bat_mxfp4_gemm
 
     def step():
         quantize(X, Xq)
-        bat.bat_mxfp4_gemm(Xq, Wq, Y=Y, out_dtype=torch.bfloat16, stream=stream)
+        gemm_fn(Xq, Wq, Y=Y, out_dtype=torch.bfloat16, stream=stream)
 
     def flush_l2(i):
         # write, then read, a buffer twice the L2: the next kernel starts with a cold L2
@@ -373,7 +391,7 @@ def main():
         ev2[i][0].record(stream)
         quantize(X, Xq)
         ev2[i][1].record(stream)
-        bat.bat_mxfp4_gemm(Xq, Wq, Y=Y, out_dtype=torch.bfloat16, stream=stream)
+        gemm_fn(Xq, Wq, Y=Y, out_dtype=torch.bfloat16, stream=stream)
         ev2[i][2].record(stream)
     torch.cuda.synchronize()
     t_pro = [ev2[i][0].elapsed_time(ev2[i][1]) * 1e-3 for i in range(K_)]
@@ -384,9 +402,10 @@ def main():
     flop = 2.0 * w.M * w.N * w.K
     value = job_throughput(flop, K_, world, t_step) / 1e12
     peaks, peak_src = load_peaks()
-    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    ratio = FP8_OVER_BF16 if a8 else FP4_OVER_BF16
+    fp4_peak = peaks["bf16_tflops"] * ratio
     gemm_tf = flop / (sg / K_) / 1e12
-    pro_bytes = PROLOGUE_BYTES_PER_ELT * w.M * w.K
+    pro_bytes = (PROLOGUE8_BYTES_PER_ELT if a8 else PROLOGUE_BYTES_PER_ELT) * w.M * w.K
     pro_gbs = pro_bytes / (sp / K_) / 1e9
 
     # end to end through the public API: pinned host X -> device, linear, Y -> pinned host
@@ -399,12 +418,12 @@ def main():
 
         def e2e_step():
             Xdev.copy_(Xh, non_blocking=True)
-            if args.shared == 8:
+            if args.shared == 8 and not a8:
                 bat.bat_linear(Xdev, Wq, A, B, gl, gh, Y=Y, out_dtype=torch.bfloat16,
                                workspace=ws, stream=stream)
             else:
                 quantize(Xdev, Xq)
-                bat.bat_mxfp4_gemm(Xq, Wq, Y=Y, out_dtype=torch.bfloat16, stream=stream)
+                gemm_fn(Xq, Wq, Y=Y, out_dtype=torch.bfloat16, stream=stream)
             Yh.copy_(Y, non_blocking=True)
 
         for _ in range(3):
@@ -424,16 +443,19 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        fl, dt, desc, thr = oracle_sample(inp, w, args.cpu_budget_s)
+        fl, dt, desc, thr = oracle_sample(inp, w, args.cpu_budget_s,
+                                          act_fmt="e4m3" if a8 else "e2m1")
         cpu = {"value": fl / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                "sample": desc, "seconds": round(dt, 2)}
 
+    gemm_kernel = "bat_mxf4_gemm_kernel<true> (W4A8)" if a8 else "bat_mxf4_gemm_kernel"
+    pro_kernel = "bat_prologue_kernel<..., MXFP8>" if a8 else "bat_prologue_kernel"
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-            "steps": K_, "warmup": args.warmup, "ms_per_step": 1e3 * t_step / K_,
+            "metric": METRIC_W4A8 if a8 else METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": K_, "warmup": args.warmup, "ms_per_step": 1e3 * t_step / K_,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "mxfp4", "data": "synthetic",
+            "dtype": "mxfp8 x mxfp4" if a8 else "mxfp4", "data": "synthetic",
             "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "out": "bf16",
                        "transform": f"GPK A {args.shared}x{args.shared} shared, "
                                     f"B_b {32 // args.shared}x{32 // args.shared} private",
@@ -442,14 +464,15 @@ def main():
             "gpu_launches": 2 * K_ * world,  # the timed pass: quantizer + GEMM per step
             "roofline": {"bound": "tensor", "achieved": gemm_tf, "peak": fp4_peak,
                          "unit": "TFLOP/s", "frac": gemm_tf / fp4_peak,
-                         "traffic": recorded_traffic("bat_mxf4_gemm_kernel", w.name),
-                         "kernel": "bat_mxf4_gemm_kernel",
-                         "peak_source": f"{peak_src} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/BF16)"},
+                         "traffic": recorded_traffic(gemm_kernel, w.name),
+                         "kernel": gemm_kernel,
+                         "peak_source": f"{peak_src} bf16 burst x {ratio:g} (nominal "
+                                        f"{'FP8' if a8 else 'FP4'}/BF16)"},
             "prologue": {"bound": "hbm", "achieved": pro_gbs, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": pro_gbs / peaks["hbm_gbs"],
                          "us_per_launch": 1e6 * sp / K_,
-                         "traffic": recorded_traffic("bat_prologue_kernel", w.name),
-                         "kernel": "bat_prologue_kernel", "peak_source": peak_src},
+                         "traffic": recorded_traffic(pro_kernel, w.name),
+                         "kernel": pro_kernel, "peak_source": peak_src},
             "gemm_us_per_launch": 1e6 * sg / K_,
             "prepare_weight_ms": prep_ms,
             "clocks": clocks,

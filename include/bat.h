@@ -78,6 +78,14 @@ typedef struct {
   int64_t k;
 } bat_mxfp4_t;
 
+/*
+ * An MXFP8 matrix (the W4A8 activations): the same struct, with
+ *   codes : [rows][k] bytes, row-major, one OCP E4M3 code per element (sign in
+ *           bit 7; largest finite 448, no infinities);
+ *   scales: the tiled UE8M0 layout of bat_mxfp4_t (bat_mxfp4_scales_bytes).
+ */
+typedef bat_mxfp4_t bat_mxfp8_t;
+
 /* Sizes of the two buffers of an MXFP4 matrix (0 if k % 32 != 0 or a size < 1). */
 BAT_API size_t bat_mxfp4_codes_bytes(int64_t rows, int64_t k);
 BAT_API size_t bat_mxfp4_scales_bytes(int64_t rows, int64_t k);
@@ -189,6 +197,40 @@ BAT_API bat_status_t bat_prepare_weight_gpk(const void* W, int64_t N, int64_t K,
  * for null buffers or nb < 1.
  */
 BAT_API bat_status_t bat_block_hadamard_factors(int shared, int64_t nb, float* A, float* B);
+
+/*
+ * W4A8 activation side: the transform and clip of bat_quantize_act_gpk, then MXFP8
+ * quantization (the W4A8 settings of the BATQuant note, Loss & Training: "MXFP8
+ * uses E4M3"). Per 32-element block, e = floor(log2 amax) - 8 (8 is E4M3's largest
+ * exponent), clamped to [-127, 127]; elements v * 2^-e rounded to the nearest E4M3
+ * (ties to even), saturating at +-448; an exact zero is +0.
+ *   Xq : output, Xq->rows == M, Xq->k == K, codes of bat_mxfp8_codes_bytes(M, K).
+ * Other arguments, requirements and errors as bat_quantize_act_gpk (shared = 8 with
+ * 8 x 8 / [K/32][4][4] factors is the default split).
+ */
+BAT_API size_t bat_mxfp8_codes_bytes(int64_t rows, int64_t k);
+BAT_API bat_status_t bat_quantize_act_mxfp8(const void* X, int64_t M, int64_t K, const float* A,
+                                            int shared, const float* B, const float* g_lo,
+                                            const float* g_hi, const bat_mxfp8_t* Xq,
+                                            float* y_out, void* stream);
+
+/*
+ * E4M3 element conversion exactly as the MXFP8 prologue performs it (values
+ * converted in groups of four, round to nearest even, saturating at +-448).
+ * v: device fp32 [n]; codes: device uint8 [n].
+ */
+BAT_API bat_status_t bat_e4m3_encode(const float* v, int64_t n, uint8_t* codes, void* stream);
+
+/*
+ * W4A8 GEMM: Y = Xq . Wq^T with MXFP8 (E4M3) activations and MXFP4 weights from
+ * bat_prepare_weight(_gpk), on tcgen05 kind::mxf8f6f4 (fp32 accumulation).
+ *   Y[m][n] = sum_b 2^(eX[m][b] + eW[n][b]) * sum_{j<32} x[m][32b+j] * w[n][32b+j]
+ * Requirements beyond bat_mxfp4_gemm's: K % 128 == 0 and Wq->codes 32-byte
+ * aligned (the weights' codes are unpacked to one byte per element by the TMA
+ * load); otherwise BAT_ERR_SHAPE / BAT_ERR_ALIGN.
+ */
+BAT_API bat_status_t bat_w4a8_gemm(const bat_mxfp8_t* Xq, const bat_mxfp4_t* Wq, void* Y,
+                                   bat_out_dtype_t out_dtype, void* stream);
 
 /*
  * Block-scaled MXFP4 GEMM on the 5th-generation tensor cores (tcgen05,

@@ -386,3 +386,146 @@ def test_argument_errors_launch_nothing(bat):
     st = bat.lib().bat_quantize_act(None, 4, 64, None, None, None, None, None, None)
     assert st == 1
     assert bat.bat_device_error() == 0
+
+
+# ---------------------------------------------------------------- W4A8 (MXFP8 activations)
+def _host8(q, rows, K):
+    codes = q.codes.cpu().numpy().reshape(rows, K)
+    tiled = q.scales.cpu().numpy()
+    return codes, formats.untile_scales(tiled, rows, K // 32), tiled
+
+
+def test_e4m3_conversion(bat):
+    rng = np.random.default_rng(4)
+    top = int(np.float32(1024.0).view(np.uint32))
+    bits = rng.integers(0, top, size=1 << 22, dtype=np.uint32)
+    bits[::2] |= np.uint32(0x80000000)
+    mags = oracle.e4m3_value(np.arange(127)).astype(np.float32)
+    mids = ((mags[:-1].astype(np.float64) + mags[1:]) / 2).astype(np.float32)
+    edges = np.concatenate([mags, mids, np.nextafter(mids, np.float32(np.inf)),
+                            np.nextafter(mids, np.float32(0)), np.float32([464, 465, 1e30, 0.0, -0.0])])
+    v = np.concatenate([bits.view(np.float32), edges, -edges])
+    got = bat.bat_e4m3_encode(_dev_f32(v)).cpu().numpy()
+    assert np.array_equal(got, oracle.e4m3_encode(v))
+
+
+def _check_act8(bat, X, A, B, g_lo, g_hi):
+    rows, K = X.shape
+    nb = K // 32
+    Xd, Ad, Bd = _dev_bf16(X), _dev_f32(A), _dev_f32(B)
+    gl = None if g_lo is None else _dev_f32(g_lo)
+    gh = None if g_hi is None else _dev_f32(g_hi)
+    y = torch.empty(rows, K, dtype=torch.float32, device="cuda")
+    Xq = bat.bat_quantize_act_mxfp8(Xd, Ad, Bd, gl, gh, y_out=y)
+    Xq2 = bat.bat_quantize_act_mxfp8(Xd, Ad, Bd, gl, gh)
+    torch.cuda.synchronize()
+    assert torch.equal(Xq.codes, Xq2.codes) and torch.equal(Xq.scales, Xq2.scales)
+    y_gpu = y.cpu().numpy()
+    _check_transform(y_gpu, oracle.transform(X, A, B))
+    r_lo = bat.bat_clip_ratios(gl, nb).cpu().numpy()
+    r_hi = bat.bat_clip_ratios(gh, nb).cpu().numpy()
+    oc, os_, bad = oracle.quantize(y_gpu, r_lo, r_hi, fmt="e4m3")
+    assert bad == 0
+    codes, scales, tiled = _host8(Xq, rows, K)
+    mism = np.argwhere(codes != oc)
+    assert mism.size == 0, (mism[:5], codes[tuple(mism[0])], oc[tuple(mism[0])])
+    assert np.array_equal(scales, os_)
+    assert np.all(tiled[formats.padding_mask(rows, nb)] == 0)
+    return Xq
+
+
+@pytest.mark.parametrize("M,K", [(1, 32), (17, 96), (130, 1056), (3, 4128), (257, 256)])
+def test_quantize_act_mxfp8_ragged(bat, M, K):
+    X = wl.random_bf16((M, K), seed=M + 11 * K, scale=3.0)
+    A, B, g_lo, g_hi = wl.random_factors(K // 32, seed=K + 5)
+    _check_act8(bat, X, A, B, g_lo, g_hi)
+
+
+@pytest.mark.parametrize("s", [2, 4, 16])
+def test_quantize_act_mxfp8_splits(bat, s):
+    X = wl.random_bf16((130, 1056), seed=s, scale=3.0)
+    A, B, g_lo, g_hi = wl.random_factors(1056 // 32, seed=s + 3, shared=s)
+    _check_act8(bat, X, A, B, g_lo, g_hi)
+
+
+@pytest.mark.parametrize("name", ["tiny", "mlp_gate_up", "mlp_down"])
+def test_quantize_act_mxfp8_workloads(bat, name):
+    inp = wl.make_inputs(name, with_weight=False)
+    _check_act8(bat, inp.X, inp.A, inp.B, inp.g_lo, inp.g_hi)
+
+
+def _w4a8_check(bat, Xq, Wq, M, N, K, rows=None, cols=None):
+    xc, xs, _ = _host8(Xq, M, K)
+    wc, ws, _ = _host(Wq, N, K)
+    Xd = oracle.dequantize(xc, xs, "e4m3")
+    Wd = oracle.dequantize(wc, ws)
+    Y32 = bat.bat_w4a8_gemm(Xq, Wq, out_dtype=torch.float32)
+    Y16 = bat.bat_w4a8_gemm(Xq, Wq, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    ref = oracle.gemm_sampled(Xd, Wd, rows, cols)
+    r = np.arange(M) if rows is None else np.asarray(rows)
+    c = np.arange(N) if cols is None else np.asarray(cols)
+    y32 = Y32.cpu().numpy()[np.ix_(r, c)].astype(np.float64)
+    y16 = Y16.float().cpu().numpy()[np.ix_(r, c)].astype(np.float64)
+    assert np.all(np.isfinite(y32))
+    rel = np.linalg.norm(y32 - ref) / max(np.linalg.norm(ref), 1e-300)
+    assert rel <= GEMM_TOL, rel
+    mag = oracle.gemm_sampled(np.abs(Xd), np.abs(Wd), rows, cols)
+    assert np.all(np.abs(y32 - ref) <= 1e-5 * mag + 1e-30), np.max(np.abs(y32 - ref) / (mag + 1e-30))
+    ref16 = torch.from_numpy(ref).to(torch.bfloat16).float().numpy().astype(np.float64)
+    rel16 = np.linalg.norm(y16 - ref16) / max(np.linalg.norm(ref16), 1e-300)
+    assert rel16 <= GEMM_TOL, rel16
+    return rel
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (1, 8, 128), (17, 200, 256), (130, 300, 512),
+                                   (256, 512, 1024), (200, 264, 4096), (300, 1000, 2048)])
+def test_w4a8_gemm_shapes(bat, M, N, K):
+    X = wl.random_bf16((M, K), seed=M + 7 * K, scale=2.0)
+    W = wl.random_bf16((N, K), seed=N + 9 * K, scale=0.02)
+    A, B, g_lo, g_hi = wl.random_factors(K // 32, seed=K + 2)
+    Ad, Bd = _dev_f32(A), _dev_f32(B)
+    Xq = bat.bat_quantize_act_mxfp8(_dev_bf16(X), Ad, Bd, _dev_f32(g_lo), _dev_f32(g_hi))
+    Wq = bat.bat_prepare_weight(_dev_bf16(W), Ad, Bd)
+    _w4a8_check(bat, Xq, Wq, M, N, K)
+    assert bat.bat_device_error() == 0
+
+
+@pytest.mark.parametrize("name", ["mlp_gate_up", "prefill_o", "decode_qkv"])
+def test_w4a8_linear_workloads(bat, name):
+    """W4A8 at the full workload sizes: sampled outputs against the oracle, and the
+    error of the layer against the unquantized product below W4A4's."""
+    inp = wl.make_inputs(name)
+    w = wl.WORKLOADS[name]
+    Ad, Bd = _dev_f32(inp.A), _dev_f32(inp.B)
+    gl, gh = _dev_f32(inp.g_lo), _dev_f32(inp.g_hi)
+    Xd = _dev_bf16(inp.X)
+    Wq = bat.bat_prepare_weight(_dev_bf16(inp.W), Ad, Bd)
+    Xq8 = bat.bat_quantize_act_mxfp8(Xd, Ad, Bd, gl, gh)
+    rows = None if w.M <= 64 else _sample(w.M, 24, 3)
+    cols = None if w.N <= 512 else _sample(w.N, 200, 4)
+    _w4a8_check(bat, Xq8, Wq, w.M, w.N, w.K, rows, cols)
+    Xq4 = bat.bat_quantize_act(Xd, Ad, Bd, gl, gh)
+    Y4 = bat.bat_mxfp4_gemm(Xq4, Wq, out_dtype=torch.float32)
+    Y8 = bat.bat_w4a8_gemm(Xq8, Wq, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    r = np.arange(w.M) if rows is None else rows
+    c = np.arange(w.N) if cols is None else cols
+    exact = oracle.gemm_sampled(wl.bf16_bits_to_f32(inp.X).astype(np.float64),
+                                wl.bf16_bits_to_f32(inp.W).astype(np.float64), r, c)
+    e4 = np.linalg.norm(Y4.cpu().numpy()[np.ix_(r, c)] - exact)
+    e8 = np.linalg.norm(Y8.cpu().numpy()[np.ix_(r, c)] - exact)
+    assert e8 < e4, (e8, e4)
+    assert bat.bat_device_error() == 0
+
+
+def test_w4a8_errors(bat):
+    X = torch.zeros(4, 96, dtype=torch.bfloat16, device="cuda")
+    A = torch.eye(8, device="cuda")
+    B = torch.eye(4, device="cuda").repeat(3, 1, 1).contiguous()
+    Xq = bat.bat_quantize_act_mxfp8(X, A, B)
+    Wq = bat.MXFP4.empty(8, 96)
+    with pytest.raises(bat.BatError) as e:
+        bat.bat_w4a8_gemm(Xq, Wq)  # K % 128 != 0
+    assert e.value.status == 2
+    assert bat.bat_device_error() == 0

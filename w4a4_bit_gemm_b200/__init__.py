@@ -67,6 +67,10 @@ def lib() -> ctypes.CDLL:
         "bat_quantize_act_gpk": (S, [P, I64, I64, P, S, P, P, P, SP, P, P]),
         "bat_prepare_weight_gpk": (S, [P, I64, I64, P, S, P, P, P, SP, P, P]),
         "bat_block_hadamard_factors": (S, [S, I64, P, P]),
+        "bat_mxfp8_codes_bytes": (ctypes.c_size_t, [I64, I64]),
+        "bat_quantize_act_mxfp8": (S, [P, I64, I64, P, S, P, P, P, SP, P, P]),
+        "bat_e4m3_encode": (S, [P, I64, P, P]),
+        "bat_w4a8_gemm": (S, [SP, SP, P, S, P]),
         "bat_mxfp4_gemm": (S, [SP, SP, P, S, P]),
         "bat_linear_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
         "bat_linear": (S, [P, I64, SP, P, P, P, P, P, S, P, ctypes.c_size_t, P]),
@@ -143,7 +147,33 @@ class MXFP4:
         return MXFP4Struct(self.codes.data_ptr(), self.scales.data_ptr(), self.rows, self.k)
 
 
+@dataclass
+class MXFP8:
+    """An MXFP8 matrix: E4M3 codes [rows][k] (one byte each) and tiled UE8M0 scales."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    rows: int
+    k: int
+
+    @staticmethod
+    def empty(rows: int, k: int, device="cuda") -> "MXFP8":
+        cb = bat_mxfp8_codes_bytes(rows, k)
+        sb = bat_mxfp4_scales_bytes(rows, k)
+        if cb == 0 or sb == 0:
+            raise ValueError(f"invalid MXFP8 shape rows={rows} k={k}")
+        return MXFP8(torch.empty(cb, dtype=torch.uint8, device=device),
+                     torch.empty(sb, dtype=torch.uint8, device=device), rows, k)
+
+    def struct(self) -> MXFP4Struct:
+        return MXFP4Struct(self.codes.data_ptr(), self.scales.data_ptr(), self.rows, self.k)
+
+
 # ---------------------------------------------------------------- C-ABI wrappers
+def bat_mxfp8_codes_bytes(rows: int, k: int) -> int:
+    return lib().bat_mxfp8_codes_bytes(rows, k)
+
+
+
 def bat_mxfp4_codes_bytes(rows: int, k: int) -> int:
     return lib().bat_mxfp4_codes_bytes(rows, k)
 
@@ -308,6 +338,45 @@ def bat_mxfp4_gemm(Xq: MXFP4, Wq: MXFP4, Y: Optional[torch.Tensor] = None,
     a, b = Xq.struct(), Wq.struct()
     _check(lib().bat_mxfp4_gemm(ctypes.byref(a), ctypes.byref(b), _ptr(Y), code, _stream(stream)),
            "bat_mxfp4_gemm")
+    return Y
+
+
+def bat_quantize_act_mxfp8(X, A, B, g_lo=None, g_hi=None, Xq: Optional[MXFP8] = None,
+                           y_out: Optional[torch.Tensor] = None, stream=None) -> MXFP8:
+    """W4A8 activation side: transform (any split of A, B), clip, MXFP8 (E4M3) quantize."""
+    M, K = X.shape
+    _need(X, torch.bfloat16, "X")
+    s = _gpk_factors(A, B, K)
+    if (g_lo is None) != (g_hi is None):
+        raise ValueError("g_lo and g_hi must both be given or both be None")
+    if g_lo is not None:
+        _need(g_lo, torch.float32, "g_lo", (K // 32,))
+        _need(g_hi, torch.float32, "g_hi", (K // 32,))
+    if y_out is not None:
+        _need(y_out, torch.float32, "y_out", (M, K))
+    Xq = MXFP8.empty(M, K, X.device) if Xq is None else Xq
+    st = Xq.struct()
+    _check(lib().bat_quantize_act_mxfp8(_ptr(X), M, K, _ptr(A), s, _ptr(B), _ptr(g_lo),
+                                        _ptr(g_hi), ctypes.byref(st), _ptr(y_out),
+                                        _stream(stream)), "bat_quantize_act_mxfp8")
+    return Xq
+
+
+def bat_e4m3_encode(v: torch.Tensor, codes=None, stream=None) -> torch.Tensor:
+    _need(v, torch.float32, "v")
+    codes = torch.empty(v.numel(), dtype=torch.uint8, device=v.device) if codes is None else codes
+    _check(lib().bat_e4m3_encode(_ptr(v), v.numel(), _ptr(codes), _stream(stream)), "bat_e4m3_encode")
+    return codes
+
+
+def bat_w4a8_gemm(Xq: MXFP8, Wq: MXFP4, Y: Optional[torch.Tensor] = None,
+                  out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
+    code = _out_code(out_dtype)
+    Y = torch.empty(Xq.rows, Wq.rows, dtype=out_dtype, device=Xq.codes.device) if Y is None else Y
+    _need(Y, out_dtype, "Y", (Xq.rows, Wq.rows))
+    a, b = Xq.struct(), Wq.struct()
+    _check(lib().bat_w4a8_gemm(ctypes.byref(a), ctypes.byref(b), _ptr(Y), code, _stream(stream)),
+           "bat_w4a8_gemm")
     return Y
 
 

@@ -29,7 +29,7 @@ int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 struct DeviceInfo {
   std::atomic<int> state{0};  // 0 unknown, 1 sm_100, 2 unsupported
   std::atomic<int> sms{0};
-  std::atomic<int> gemm_attr{0};
+  std::atomic<int> gemm_attr{0};    // bit 0: W4A4 GEMM, bit 1: W4A8 GEMM attribute set
   std::atomic<int> pro_attr{0};     // bit t: the prologue variant t has its smem attribute set
 };
 DeviceInfo g_dev[64];
@@ -96,6 +96,40 @@ bool make_code_map(CUtensorMap* map, const void* codes, int64_t rows, int64_t k,
   cuuint32_t estr[2] = {1u, 1u};
   CUresult r = f(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides,
                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// E4M3 codes of an MXFP8 matrix, [rows][k] bytes, box of 128 bytes x box_rows, 128-byte
+// swizzle.
+bool make_code8_map(CUtensorMap* map, const void* codes, int64_t rows, int64_t k, uint32_t box_rows) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(k)};
+  cuuint32_t box[2] = {128u, box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = f(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides,
+                 box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Packed E2M1 codes of an MXFP4 matrix as 4-bit elements [rows][k], loaded with the
+// unpacking data type: every 16 elements (8 bytes in memory) land in 16 bytes of shared
+// memory, the operand layout of kind::mxf8f6f4 for E2M1. Box of 128 elements (128 bytes
+// in shared memory) x box_rows, 128-byte swizzle. Needs k % 128 == 0 and 32-byte
+// aligned codes.
+bool make_code4_unpack_map(CUtensorMap* map, const void* codes, int64_t rows, int64_t k,
+                           uint32_t box_rows) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(k / 2)};
+  cuuint32_t box[2] = {128u, box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = f(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(codes), dims,
+                 strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -199,7 +233,7 @@ bat_status_t check_act_args(const void* X, int64_t M, int64_t K, const float* A,
 bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float* A,
                              const float* B, const float* g_lo, const float* g_hi, bool per_row,
                              const bat_mxfp4_t* out, float* y_out, cudaStream_t stream,
-                             int ls = 3) {
+                             int ls = 3, bool fp8 = false) {
   int dev = 0, sms = 0;
   bat_status_t st = current_device(&dev, &sms);
   if (st != BAT_OK) return st;
@@ -231,12 +265,14 @@ bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float
     p.cps = cps < 1 ? 1 : cps;
   }
   void (*kern)(CUtensorMap, bat::PrologueParams);
-  if (per_row)
+  if (fp8)  // activations only: clip logits per block
+    kern = y_out ? bat::bat_prologue_kernel<true, false, true> : bat::bat_prologue_kernel<false, false, true>;
+  else if (per_row)
     kern = y_out ? bat::bat_prologue_kernel<true, true> : bat::bat_prologue_kernel<false, true>;
   else
     kern = y_out ? bat::bat_prologue_kernel<true, false> : bat::bat_prologue_kernel<false, false>;
   DeviceInfo& d = g_dev[dev];
-  const int variant_bit = 1 << ((per_row ? 2 : 0) + (y_out ? 1 : 0));
+  const int variant_bit = 1 << ((fp8 ? 4 : (per_row ? 2 : 0)) + (y_out ? 1 : 0));
   if (!(d.pro_attr.load() & variant_bit)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              bat::pro::kSmemBytes) != cudaSuccess)
@@ -249,14 +285,20 @@ bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float
   return cuda_status(cudaGetLastError());
 }
 
+// a8: Xq holds MXFP8 (E4M3) activations and the W4A8 kernel runs; K % 128 == 0 then.
 bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
-                         bat_out_dtype_t out_dtype, cudaStream_t stream) {
+                         bat_out_dtype_t out_dtype, cudaStream_t stream, bool a8 = false) {
   int dev = 0, sms = 0;
   bat_status_t st = current_device(&dev, &sms);
   if (st != BAT_OK) return st;
   CUtensorMap ta, tb, ty;
-  if (!make_code_map(&ta, Xq->codes, Xq->rows, Xq->k, bat::gemm::kBM)) return BAT_ERR_CUDA;
-  if (!make_code_map(&tb, Wq->codes, Wq->rows, Wq->k, bat::gemm::kBN)) return BAT_ERR_CUDA;
+  if (a8) {
+    if (!make_code8_map(&ta, Xq->codes, Xq->rows, Xq->k, bat::gemm::kBM)) return BAT_ERR_CUDA;
+    if (!make_code4_unpack_map(&tb, Wq->codes, Wq->rows, Wq->k, bat::gemm::kBN)) return BAT_ERR_CUDA;
+  } else {
+    if (!make_code_map(&ta, Xq->codes, Xq->rows, Xq->k, bat::gemm::kBM)) return BAT_ERR_CUDA;
+    if (!make_code_map(&tb, Wq->codes, Wq->rows, Wq->k, bat::gemm::kBN)) return BAT_ERR_CUDA;
+  }
   std::memset(&ty, 0, sizeof(ty));
   bat::GemmParams p;
   p.sfa = static_cast<const uint8_t*>(Xq->scales);
@@ -271,13 +313,16 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
   // bf16 output with 16-byte rows goes through shared-memory staging and TMA stores
   p.tma_store = (!p.out_f32 && p.vec_ok) ? 1 : 0;
   if (p.tma_store && !make_out_map(&ty, Y, p.M, p.N)) return BAT_ERR_CUDA;
+  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, bat::GemmParams) =
+      a8 ? bat::bat_mxf4_gemm_kernel<true> : bat::bat_mxf4_gemm_kernel<false>;
+  const int smem = a8 ? bat::gemm::Cfg<true>::kSmemBytes : bat::gemm::Cfg<false>::kSmemBytes;
   DeviceInfo& d = g_dev[dev];
-  if (!d.gemm_attr.load()) {
-    const cudaError_t ae = cudaFuncSetAttribute(bat::bat_mxf4_gemm_kernel,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                bat::gemm::kSmemBytes);
+  const int variant_bit = a8 ? 2 : 1;
+  if (!(d.gemm_attr.load() & variant_bit)) {
+    const cudaError_t ae =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (ae != cudaSuccess) return cuda_status(ae);
-    d.gemm_attr.store(1);
+    d.gemm_attr.fetch_or(variant_bit);
   }
   const int64_t tiles = ((p.M + bat::gemm::kBM - 1) / bat::gemm::kBM) *
                         ((p.N + bat::gemm::kBN - 1) / bat::gemm::kBN);
@@ -288,22 +333,27 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(bat::gemm::kThreads);
-  cfg.dynamicSmemBytes = bat::gemm::kSmemBytes;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, bat::bat_mxf4_gemm_kernel, ta, tb, ty, p));
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, p));
 }
 
 bat_status_t check_gemm_args(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, const void* Y,
-                             bat_out_dtype_t out_dtype) {
+                             bat_out_dtype_t out_dtype, bool a8 = false) {
   if (!Xq || !Wq || !Y) return BAT_ERR_INVALID_ARG;
   if (out_dtype != BAT_OUT_BF16 && out_dtype != BAT_OUT_F32) return BAT_ERR_INVALID_ARG;
   if (Xq->rows < 1 || Wq->rows < 1 || Xq->k < 32) return BAT_ERR_INVALID_ARG;
   if (Xq->k != Wq->k || Xq->k % 32 != 0 || Xq->k > kMaxK) return BAT_ERR_SHAPE;
+  if (a8) {
+    // the unpacking load of the weights: k % 128 == 0, 32-byte aligned codes
+    if (Xq->k % 128 != 0) return BAT_ERR_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(Wq->codes) & 31u) != 0) return BAT_ERR_ALIGN;
+  }
   bat_status_t st = check_mxfp4(Xq, Xq->rows, Xq->k);
   if (st != BAT_OK) return st;
   st = check_mxfp4(Wq, Wq->rows, Wq->k);
@@ -488,6 +538,31 @@ bat_status_t bat_mxfp4_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* 
   return launch_gemm(Xq, Wq, Y, out_dtype, static_cast<cudaStream_t>(stream));
 }
 
+size_t bat_mxfp8_codes_bytes(int64_t rows, int64_t k) {
+  if (rows < 1 || k < 32 || k % 32 != 0) return 0;
+  return static_cast<size_t>(rows) * static_cast<size_t>(k);
+}
+
+bat_status_t bat_quantize_act_mxfp8(const void* X, int64_t M, int64_t K, const float* A,
+                                    int shared, const float* B, const float* g_lo,
+                                    const float* g_hi, const bat_mxfp8_t* Xq, float* y_out,
+                                    void* stream) {
+  const int ls = shared_log2(shared);
+  if (ls < 0) return BAT_ERR_UNSUPPORTED;
+  bat_status_t st = check_act_args(X, M, K, A, B, g_lo, g_hi, Xq);
+  if (st != BAT_OK) return st;
+  if (y_out && !aligned16(y_out)) return BAT_ERR_ALIGN;
+  return launch_prologue(X, M, K, A, B, g_lo, g_hi, false, Xq, y_out,
+                         static_cast<cudaStream_t>(stream), ls, true);
+}
+
+bat_status_t bat_w4a8_gemm(const bat_mxfp8_t* Xq, const bat_mxfp4_t* Wq, void* Y,
+                           bat_out_dtype_t out_dtype, void* stream) {
+  bat_status_t st = check_gemm_args(Xq, Wq, Y, out_dtype, true);
+  if (st != BAT_OK) return st;
+  return launch_gemm(Xq, Wq, Y, out_dtype, static_cast<cudaStream_t>(stream), true);
+}
+
 size_t bat_linear_workspace_bytes(int64_t M, int64_t K) {
   const size_t c = bat_mxfp4_codes_bytes(M, K);
   const size_t s = bat_mxfp4_scales_bytes(M, K);
@@ -551,7 +626,33 @@ __global__ void bat_e2m1_encode_kernel(const float* v, int64_t n, uint8_t* codes
     if (2 * t + 1 < n) codes[2 * t + 1] = static_cast<uint8_t>(byte >> 4);
   }
 }
+__global__ void bat_e4m3_encode_kernel(const float* v, int64_t n, uint8_t* codes) {
+  // Groups (4t .. 4t+3) go through the conversion the MXFP8 prologue uses (4t in the
+  // low byte); each code is returned in its own byte (sign in bit 7).
+  const int64_t quads = (n + 3) / 4;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < quads;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float f[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[i] = (4 * t + i < n) ? v[4 * t + i] : 0.0f;
+    const uint32_t w = e4m3x4(f[0], f[1], f[2], f[3]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (4 * t + i < n) codes[4 * t + i] = static_cast<uint8_t>(w >> (8 * i));
+  }
+}
 }  // namespace bat
+
+extern "C" bat_status_t bat_e4m3_encode(const float* v, int64_t n, uint8_t* codes, void* stream) {
+  if (!v || !codes || n < 1) return BAT_ERR_INVALID_ARG;
+  int dev = 0, sms = 0;
+  bat_status_t st = current_device(&dev, &sms);
+  if (st != BAT_OK) return st;
+  const int64_t blocks = ((n + 3) / 4 + 255) / 256;
+  bat::bat_e4m3_encode_kernel<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), 256, 0,
+                                static_cast<cudaStream_t>(stream)>>>(v, n, codes);
+  return cuda_status(cudaGetLastError());
+}
 
 extern "C" bat_status_t bat_e2m1_encode(const float* v, int64_t n, uint8_t* codes, void* stream) {
   if (!v || !codes || n < 1) return BAT_ERR_INVALID_ARG;

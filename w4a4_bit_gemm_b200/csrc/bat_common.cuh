@@ -80,6 +80,19 @@ __device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
   return r;
 }
 
+// Four fp32 values -> one word of OCP E4M3 codes, v[i] in byte i (round to nearest
+// even, saturating at +-448).
+__device__ __forceinline__ uint32_t e4m3x4(float v0, float v1, float v2, float v3) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 h0, h1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 h0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 h1, %4, %3;\n\t"
+      "mov.b32 %0, {h0, h1};\n\t}"
+      : "=r"(r)
+      : "f"(v0), "f"(v1), "f"(v2), "f"(v3));
+  return r;
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -218,6 +231,18 @@ __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
+// D (+)= A . B^T with one UE8M0 scale per 32 elements along K (K = 32 per
+// instruction); A and B element types come from the instruction descriptor.
+__device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::
+          "r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
 // Copy 32 rows x 16 bytes from shared memory into TMEM, replicated into all four
 // 32-lane sub-partitions (the scale-factor layout the block-scaled MMA reads).
 __device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
@@ -281,6 +306,19 @@ __host__ __device__ constexpr uint32_t idesc_mxf4(int m, int n, uint32_t a_sf_id
   return (b_sf_id & 3u) << 4 |            // B scale-factor id
          1u << 7 |                        // A format: E2M1
          1u << 10 |                       // B format: E2M1
+         static_cast<uint32_t>(n >> 3) << 17 |  // N / 8
+         1u << 23 |                       // scale format UE8M0
+         static_cast<uint32_t>(m >> 4) << 24 |  // M / 16
+         (a_sf_id & 3u) << 29;            // A scale-factor id
+}
+
+// Instruction descriptor of kind::mxf8f6f4 with A in E4M3 and B in E2M1 (format codes
+// 0 and 5 of that kind), fp32 accumulation, UE8M0 scales, both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_mxf8f6f4_e4m3_e2m1(int m, int n, uint32_t a_sf_id,
+                                                                uint32_t b_sf_id) {
+  return (b_sf_id & 3u) << 4 |            // B scale-factor id
+         0u << 7 |                        // A format: E4M3
+         5u << 10 |                       // B format: E2M1
          static_cast<uint32_t>(n >> 3) << 17 |  // N / 8
          1u << 23 |                       // scale format UE8M0
          static_cast<uint32_t>(m >> 4) << 24 |  // M / 16

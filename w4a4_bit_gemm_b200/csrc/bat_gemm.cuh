@@ -17,6 +17,9 @@
 //               kStages shared-memory stages guarded by mbarriers;
 //   warp 9      TMEM owner and MMA issuer: tcgen05.mma kind::mxf4.block_scale
 //               (M=128, N=256, K=64) accumulating in TMEM;
+//               with MXFP8 activations (W4A8, kA8), kind::mxf8f6f4.block_scale
+//               (E4M3 x E2M1, K=32), the weights' packed E2M1 codes unpacked by
+//               the TMA load into the 16-bytes-per-16-elements layout that MMA reads;
 //   warps 10,11 idle (they complete the third warpgroup).
 // Every wait is bounded (see mbar_wait) and reports through the error word.
 // Launched with programmatic stream serialization, so barrier set-up and the TMEM
@@ -30,15 +33,10 @@ namespace bat {
 namespace gemm {
 constexpr int kBM = 128;                     // rows of X per tile (MMA M)
 constexpr int kBN = 256;                     // rows of W per tile (MMA N)
-constexpr int kBK = 256;                     // K elements per stage (128 bytes of codes per row)
 constexpr int kStages = 4;
-constexpr int kABytes = kBM * kBK / 2;       // 16 KB
-constexpr int kBBytes = kBN * kBK / 2;       // 32 KB
+constexpr int kABytes = kBM * 128;           // 16 KB: 128 bytes of codes per row and stage
+constexpr int kBBytes = kBN * 128;           // 32 KB
 constexpr int kChunk = 512;                  // one 128-row x 4-scale block of the scale layout
-constexpr int kChunksPerStage = kBK / 128;   // 2
-constexpr int kSfaBytes = (kBM / 128) * kChunksPerStage * kChunk;  // 1 KB
-constexpr int kSfbBytes = (kBN / 128) * kChunksPerStage * kChunk;  // 2 KB
-constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
 constexpr int kThreads = 384;
 constexpr uint32_t kRegsEpi = 248;   // after setmaxnreg: 128 x 248 + 256 x 56 <= 384 x 168
 constexpr uint32_t kRegsOther = 56;
@@ -47,9 +45,20 @@ constexpr uint32_t kRegsOther = 56;
 // streams it through this box one 64-column slice at a time.
 constexpr int kEpiBoxBytes = kBM * 128;
 constexpr int kEpiBytes = kEpiBoxBytes;  // 16 KB
-constexpr int kSmemBytes = kStages * kStageBytes + kEpiBytes + 1024 /*align*/ + 256 /*barriers*/;
+// Per activation format: K elements per stage (128 bytes of codes per row: 256 packed
+// E2M1, or 128 E4M3 with the weights' E2M1 unpacked to a byte each in shared memory),
+// the stage's scale chunks, and the stage size (a multiple of 1 KB for the swizzle).
+template <bool kA8>
+struct Cfg {
+  static constexpr int kBK = kA8 ? 128 : 256;
+  static constexpr int kChunksPerStage = kBK / 128;                      // 1 or 2
+  static constexpr int kSfaBytes = (kBM / 128) * kChunksPerStage * kChunk;
+  static constexpr int kSfbBytes = (kBN / 128) * kChunksPerStage * kChunk;
+  static constexpr int kStageBytes = (kABytes + kBBytes + kSfaBytes + kSfbBytes + 1023) / 1024 * 1024;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kEpiBytes + 1024 /*align*/ + 256 /*barriers*/;
+};
 // TMEM columns: accumulator [0, 256); stage s's scales at 256 + 24 s: A words
-// [0, 8) (two 128-K chunks x 4), B words [8, 24) (two chunks x two 128-row groups x 4).
+// [0, 8) (up to two 128-K chunks x 4), B words [8, 24) (chunks x two 128-row groups x 4).
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCol0 = 256;
 constexpr uint32_t kSfStageCols = 24;
@@ -149,11 +158,19 @@ __device__ __forceinline__ void store_chunk(const GemmParams& p, int64_t row, in
   }
 }
 
+// kA8 = false: Xq MXFP4 (tmap_a over packed codes [M][K/2] bytes).
+// kA8 = true:  Xq MXFP8 E4M3 (tmap_a over codes [M][K] bytes) and tmap_b over Wq's packed
+//              E2M1 codes with the 16-elements-per-16-bytes shared-memory expansion.
+template <bool kA8>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
     bat_mxf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                          const __grid_constant__ CUtensorMap tmap_b,
                          const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
   using namespace gemm;
+  constexpr int kBK = Cfg<kA8>::kBK;
+  constexpr int kChunksPerStage = Cfg<kA8>::kChunksPerStage;
+  constexpr int kSfaBytes = Cfg<kA8>::kSfaBytes;
+  constexpr int kStageBytes = Cfg<kA8>::kStageBytes;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t base = (raw_u32 + 1023u) & ~1023u;
@@ -221,11 +238,16 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, kErrWaitEmpty)) { ok = false; break; }
           const int c0 = ks * kChunksPerStage;
           const int nch = min(kChunksPerStage, p.nbp4 - c0);
-          const uint32_t bytes = kABytes + kBBytes + static_cast<uint32_t>(nch) * kChunk * (1 + ngb);
+          // the unpacking load of W (kA8) moves 64 bytes per row: its 8-byte gaps in shared
+          // memory are not written and count no transaction bytes
+          constexpr uint32_t kBTx = kA8 ? kBBytes / 2 : kBBytes;
+          const uint32_t bytes = kABytes + kBTx + static_cast<uint32_t>(nch) * kChunk * (1 + ngb);
           const uint32_t sa = base + stage * kStageBytes;
           mbar_expect_tx(full_bar(stage), bytes);
-          tma_load_2d(sa, &tmap_a, full_bar(stage), ks * (kBK / 2), static_cast<int32_t>(mt * kBM));
-          tma_load_2d(sa + kABytes, &tmap_b, full_bar(stage), ks * (kBK / 2),
+          // x of both maps is 128 per stage: bytes of packed E2M1, E4M3 elements, or
+          // (unpacking load) E2M1 elements
+          tma_load_2d(sa, &tmap_a, full_bar(stage), ks * 128, static_cast<int32_t>(mt * kBM));
+          tma_load_2d(sa + kABytes, &tmap_b, full_bar(stage), ks * 128,
                       static_cast<int32_t>(nt * kBN));
           bulk_load(sa + kABytes + kBBytes, p.sfa + (mt * p.nbp4 + c0) * kChunk, nch * kChunk,
                     full_bar(stage));
@@ -261,7 +283,15 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
           const uint32_t t_sfb = t_sfa + 8;
           const int64_t krem = p.K - static_cast<int64_t>(ks) * kBK;
           const uint32_t acc0 = (ks != 0) ? 1u : 0u;
-          if (krem >= kBK) {
+          if constexpr (kA8) {
+            // four K=32 MMAs, 32 bytes of each operand apiece; scale byte c of each word
+            // (K % 128 == 0, so every stage is full)
+#pragma unroll
+            for (uint32_t c = 0; c < 4; ++c)
+              mma_mxf8f6f4(tmem_base, adesc0 + so + 2 * c, bdesc0 + so + 2 * c,
+                           idesc_mxf8f6f4_e4m3_e2m1(kBM, kBN, c, c), t_sfa | (c << 30),
+                           t_sfb | (c << 30), (acc0 | c) != 0 ? 1u : 0u);
+          } else if (krem >= kBK) {
             // four K=64 MMAs; 32 bytes of codes each; scale byte pair 0-1 then 2-3 of each chunk
             mma_mxf4(tmem_base, adesc0 + so, bdesc0 + so, id_lo, t_sfa, t_sfb, acc0);
             mma_mxf4(tmem_base, adesc0 + so + 2, bdesc0 + so + 2, id_hi, t_sfa | (2u << 30),
@@ -300,14 +330,14 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       for (int ks = 0; ks < k_stages; ++ks) {
         if (!mbar_wait(full_bar(stage), phase, kErrWaitFull)) { ok = false; break; }
         const uint32_t ssf = base + stage * kStageBytes + kABytes + kBBytes + lane * 16;
-        uint32_t fa[8], fb[16];
+        uint32_t fa[8] = {}, fb[16] = {};
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < kChunksPerStage; ++c) {
           const uint4 v = lds_v4_u32(ssf + c * kChunk);
           fa[4 * c] = v.x; fa[4 * c + 1] = v.y; fa[4 * c + 2] = v.z; fa[4 * c + 3] = v.w;
         }
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
+        for (int c = 0; c < kChunksPerStage; ++c)
 #pragma unroll
           for (int g = 0; g < 2; ++g) {
             const uint4 v = lds_v4_u32(ssf + kSfaBytes + g * (kChunksPerStage * kChunk) + c * kChunk);
@@ -316,7 +346,14 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
           }
         const uint32_t tcol = tmem_base + tlane + kSfCol0 + kSfStageCols * stage;
         tmem_st_32x32b_x8(tcol, fa);
-        tmem_st_32x32b_x16(tcol + 8, fb);
+        if constexpr (kA8) {
+          uint32_t fb8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) fb8[i] = fb[i];
+          tmem_st_32x32b_x8(tcol + 8, fb8);
+        } else {
+          tmem_st_32x32b_x16(tcol + 8, fb);
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();

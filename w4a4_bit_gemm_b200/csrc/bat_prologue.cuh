@@ -74,7 +74,7 @@ struct PrologueParams {
   const float* b;        // fp32 [nb][32/s][32/s], private factors
   const float* g_lo;     // clip logits: [nb] (shared by rows) or [rows][nb]; may be null
   const float* g_hi;
-  uint8_t* codes;        // [rows][K/2]
+  uint8_t* codes;        // [rows][K/2] packed E2M1, or [rows][K] E4M3 (kFp8)
   uint8_t* scales;       // tiled, rows padded to 128, blocks padded to 4
   float* y_out;          // optional fp32 [rows][K] trace of the transformed values
   int64_t rows;
@@ -174,9 +174,11 @@ __device__ __forceinline__ void build_p_row(uint8_t* dst, const float* a, const 
 }
 
 // Quantize one 32-element block held by this thread: clip to [r_lo*min, r_hi*max],
-// UE8M0 scale, E2M1 codes (16 bytes into `packed`). Returns the scale byte e + 127.
+// UE8M0 scale, then E2M1 codes (MXFP4: 16 bytes into `packed`) or, with kFp8, OCP
+// E4M3 codes (MXFP8: 32 bytes). Returns the scale byte e + 127.
+template <bool kFp8>
 __device__ __forceinline__ uint32_t quantize_block(const float (&y)[32], float r_lo, float r_hi,
-                                                   uint32_t (&packed)[4]) {
+                                                   uint32_t (&packed)[kFp8 ? 8 : 4]) {
   float tmn[11], tmx[11];
 #pragma unroll
   for (int k = 0; k < 10; ++k) {
@@ -195,30 +197,48 @@ __device__ __forceinline__ uint32_t quantize_block(const float (&y)[32], float r
   const float hi = __fmul_rn(r_hi, mx);
   // The clamp is monotone, so the clipped block's extremes are the clipped min/max.
   const float amax = fmaxf(fabsf(fminf(fmaxf(mn, lo), hi)), fabsf(fminf(fmaxf(mx, lo), hi)));
-  // UE8M0 scale: e = floor(log2 amax) - 2, clamped to >= -127 (amax = 0 -> -127)
+  // UE8M0 scale: e = floor(log2 amax) - emax, with emax 2 (E2M1) or 8 (E4M3), clamped
+  // to >= -127 (amax = 0 -> -127)
+  constexpr int kEmax = kFp8 ? 8 : 2;
   const int efield = static_cast<int>(__float_as_uint(amax) >> 23);
-  const int sbyte = efield > 2 ? efield - 2 : 0;  // e + 127
+  const int sbyte = efield > kEmax ? efield - kEmax : 0;  // e + 127
   const float inv_scale = __uint_as_float(static_cast<uint32_t>(254 - sbyte) << 23);  // 2^-e
   const uint64_t s2 = pack2(inv_scale, inv_scale);
-  // codes: v = c * 2^-e (+0 turns an exact -0 into +0), E2M1 round-to-nearest-even,
-  // eight codes per 32-bit word
+  // codes: v = c * 2^-e (+0 turns an exact -0 into +0), round to nearest even; E4M3:
+  // four codes per 32-bit word
+  if constexpr (kFp8) {
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    float v[8];
+    for (int c = 0; c < 8; ++c) {
+      float v[4];
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const float c0 = fminf(fmaxf(y[8 * c + 2 * h], lo), hi);
-      const float c1 = fminf(fmaxf(y[8 * c + 2 * h + 1], lo), hi);
-      unpack2(ffma2(pack2(c0, c1), s2, 0ull), v[2 * h], v[2 * h + 1]);
+      for (int h = 0; h < 2; ++h) {
+        const float c0 = fminf(fmaxf(y[4 * c + 2 * h], lo), hi);
+        const float c1 = fminf(fmaxf(y[4 * c + 2 * h + 1], lo), hi);
+        unpack2(ffma2(pack2(c0, c1), s2, 0ull), v[2 * h], v[2 * h + 1]);
+      }
+      packed[c] = e4m3x4(v[0], v[1], v[2], v[3]);
     }
-    packed[c] = e2m1x8(v);
+  } else {
+    // E2M1: eight codes per 32-bit word
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float v[8];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float c0 = fminf(fmaxf(y[8 * c + 2 * h], lo), hi);
+        const float c1 = fminf(fmaxf(y[8 * c + 2 * h + 1], lo), hi);
+        unpack2(ffma2(pack2(c0, c1), s2, 0ull), v[2 * h], v[2 * h + 1]);
+      }
+      packed[c] = e2m1x8(v);
+    }
   }
   return static_cast<uint32_t>(sbyte);
 }
 
 // tmap_x: bf16 X [rows][K], box 64 columns x 128 rows, 128-byte swizzle, zero fill.
 // kPerRowClip: clip logits indexed [row][block] (weight side) instead of [block].
-template <bool kTrace, bool kPerRowClip>
+// kFp8: MXFP8 (E4M3) codes, one byte per element, instead of packed MXFP4.
+template <bool kTrace, bool kPerRowClip, bool kFp8 = false>
 __global__ void __launch_bounds__(pro::kThreads, 1)
     bat_prologue_kernel(const __grid_constant__ CUtensorMap tmap_x, const PrologueParams p) {
   using namespace pro;
@@ -450,11 +470,17 @@ __global__ void __launch_bounds__(pro::kThreads, 1)
           r_lo = ratios[lb];
           r_hi = ratios[2 * kStrip + lb];
         }
-        uint32_t packed[4];
-        const uint32_t sbyte = quantize_block(y, r_lo, r_hi, packed);
+        uint32_t packed[kFp8 ? 8 : 4];
+        const uint32_t sbyte = quantize_block<kFp8>(y, r_lo, r_hi, packed);
         if (valid) {
-          *reinterpret_cast<uint4*>(p.codes + m * (p.K / 2) + b * (kG / 2)) =
-              make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          if constexpr (kFp8) {
+            uint4* dst = reinterpret_cast<uint4*>(p.codes + m * p.K + b * kG);
+            dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+          } else {
+            *reinterpret_cast<uint4*>(p.codes + m * (p.K / 2) + b * (kG / 2)) =
+                make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          }
           if (kTrace) {
             float4* dst = reinterpret_cast<float4*>(p.y_out + m * p.K + b * kG);
 #pragma unroll
