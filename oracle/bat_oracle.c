@@ -77,10 +77,10 @@ void orc_kron(const double* B /*4x4*/, const double* A /*8x8*/, double* P /*32x3
   orc_kron_gen(B, A, 8, P);
 }
 
-/* y = x . P_b for every row and block, fp64 result (not rounded); A is s x s and
- * B holds nb blocks of t x t. */
-void orc_transform_f64_gen(const uint16_t* X, int64_t M, int64_t K, const float* A, int s,
-                           const float* B, double* Y) {
+/* y = x . P_b for every row and block of an fp64 matrix, fp64 result (not
+ * rounded); A is s x s and B holds nb blocks of t x t. */
+void orc_transform_vals_f64(const double* X, int64_t M, int64_t K, const float* A, int s,
+                            const float* B, double* Y) {
   const int64_t nb = K / ORC_G;
   const int t2 = (ORC_G / s) * (ORC_G / s);
   double Ad[1024], Bd[1024];
@@ -94,16 +94,24 @@ void orc_transform_f64_gen(const uint16_t* X, int64_t M, int64_t K, const float*
   for (int64_t m = 0; m < M; ++m) {
     for (int64_t b = 0; b < nb; ++b) {
       const double* Pb = P + 1024 * b;
-      double x[32];
-      for (int k = 0; k < 32; ++k) x[k] = bf16_bits_to_double(X[m * K + b * 32 + k]);
+      const double* x = X + m * K + b * 32;
       for (int j = 0; j < 32; ++j) {
-        double s = 0.0;
-        for (int k = 0; k < 32; ++k) s += x[k] * Pb[k * 32 + j];
-        Y[m * K + b * 32 + j] = s;
+        double acc = 0.0;
+        for (int k = 0; k < 32; ++k) acc += x[k] * Pb[k * 32 + j];
+        Y[m * K + b * 32 + j] = acc;
       }
     }
   }
   free(P);
+}
+
+/* The same for bf16 input (the activations). */
+void orc_transform_f64_gen(const uint16_t* X, int64_t M, int64_t K, const float* A, int s,
+                           const float* B, double* Y) {
+  double* Xd = (double*)malloc(sizeof(double) * (size_t)(M * K));
+  for (int64_t t = 0; t < M * K; ++t) Xd[t] = bf16_bits_to_double(X[t]);
+  orc_transform_vals_f64(Xd, M, K, A, s, B, Y);
+  free(Xd);
 }
 
 void orc_transform_f64(const uint16_t* X, int64_t M, int64_t K, const float* A, const float* B,

@@ -51,6 +51,7 @@ def lib():
         L.orc_transform_gen.argtypes = [P, I64, I64, P, ctypes.c_int, P, P]
         L.orc_weight_transform_f64_gen.argtypes = [P, I64, I64, P, ctypes.c_int, P, P]
         L.orc_weight_transform_f64_gen.restype = ctypes.c_int
+        L.orc_transform_vals_f64.argtypes = [P, I64, I64, P, ctypes.c_int, P, P]
         L.orc_num_threads.restype = ctypes.c_int
         L.orc_e4m3_encode_array.argtypes = [P, I64, P]
         L.orc_e4m3_value.argtypes = [ctypes.c_uint8]
@@ -255,3 +256,51 @@ def gpk_param_counts(K: int, shared: int = 8, private: int = 4) -> dict:
 def num_threads() -> int:
     """Host threads the oracle's parallel loops use."""
     return int(lib().orc_num_threads())
+
+
+def transform_vals_f64(Xd: np.ndarray, A: np.ndarray, B: np.ndarray) -> np.ndarray:
+    """x . (B_b (x) A) for an fp64 matrix (any split); fp64, unrounded."""
+    Xd = _c(Xd, np.float64)
+    M, K = Xd.shape
+    s = factor_sizes(A, B, K)
+    Y = np.empty((M, K), np.float64)
+    lib().orc_transform_vals_f64(_p(Xd), M, K, _p(_c(A, np.float32)), s, _p(_c(B, np.float32)),
+                                 _p(Y))
+    return Y
+
+
+# ---------------------------------------------------------------- KV-cache path
+# The note (Key Designs 4, "Equivalent Transformer integration") puts one transform
+# set on the per-head key path and one on the value path, and the settings KV8 / KV4
+# quantize the cache to MXFP8 (E4M3) / MXFP4. Reading: every head's D-vector
+# (D = head_dim, a multiple of 32) is transformed by the same factors (A shared,
+# B[D/32] one per 32-channel block of the head), clipped with per-block logits
+# [D/32] shared by heads and tokens, quantized, and stored at the token's cache
+# slot; slot -1 means "do not store".
+
+def kv_quantize(kv: np.ndarray, A, B, g_lo, g_hi, fmt: str, slots, cache_codes, cache_scales):
+    """kv: bf16 bits [T][H][D]; cache_codes [S][H][D] (one code per byte),
+    cache_scales [S][H][D/32]; both updated in place at rows slots[t] >= 0.
+    Returns the fp32 transformed values [T][H][D]."""
+    T, H, D = kv.shape
+    Y, codes, scales = quantize_act(kv.reshape(T * H, D), A, B, g_lo, g_hi, fmt=fmt)
+    codes = codes.reshape(T, H, D)
+    scales = scales.reshape(T, H, D // G)
+    for t in range(T):
+        if slots[t] >= 0:
+            cache_codes[slots[t]] = codes[t]
+            cache_scales[slots[t]] = scales[t]
+    return Y.reshape(T, H, D)
+
+
+def kv_dequantize(cache_codes, cache_scales, slots, fmt: str, A_out=None, B_out=None):
+    """Values of the cache rows slots[t] ([T][H][D], fp64), optionally multiplied per
+    32-block by B_out (x) A_out (the inverse factors give back the untransformed K/V)."""
+    S, H, D = cache_codes.shape
+    T = len(slots)
+    c = np.asarray(cache_codes)[np.asarray(slots)].reshape(T * H, D)
+    sc = np.asarray(cache_scales)[np.asarray(slots)].reshape(T * H, D // G)
+    v = dequantize(c, sc, fmt)
+    if A_out is not None:
+        v = transform_vals_f64(v, A_out, B_out)
+    return v.reshape(T, H, D)

@@ -555,3 +555,96 @@ def test_mxfp8_linear_error_below_mxfp4():
     e8 = np.linalg.norm(oracle.linear(inp.X, inp.W, inp.A, inp.B, inp.g_lo, inp.g_hi,
                                       act_fmt="e4m3") - ref)
     assert e8 < e4
+
+
+# --- KV-cache path (KV8 / KV4) ------------------------------------------------------
+
+@pytest.mark.parametrize("s", SIZES)
+def test_inverse_factors_invert_the_block(s):
+    """B_b^-1 (x) A^-1 is the inverse of B_b (x) A: transforming back recovers x
+    (checked against numpy's inverse of the explicit block-diagonal P)."""
+    nb = 4
+    A, B, _, _ = wl.random_factors(nb, seed=80 + s, shared=s)
+    Ai = oracle.inverse(A.astype(np.float64))
+    Bi = np.stack([oracle.inverse(B[b].astype(np.float64)) for b in range(nb)])
+    Xd = wl.bf16_bits_to_f32(wl.random_bf16((6, 32 * nb), seed=81 + s)).astype(np.float64)
+    Y = oracle.transform_vals_f64(Xd, A, B)
+    P = scipy.linalg.block_diag(*[np.kron(B[b].astype(np.float64), A.astype(np.float64))
+                                  for b in range(nb)])
+    # the factors are passed as fp32; compare against the fp32-rounded inverse factors' block
+    Pi = scipy.linalg.block_diag(*[np.kron(Bi[b].astype(np.float32).astype(np.float64),
+                                           Ai.astype(np.float32).astype(np.float64)) for b in range(nb)])
+    back = oracle.transform_vals_f64(Y, Ai.astype(np.float32), Bi.astype(np.float32))
+    assert np.allclose(back, Y @ Pi, rtol=0, atol=1e-12 * np.abs(Y).max())
+    assert np.allclose(np.linalg.inv(P), Pi, atol=1e-5)
+    assert np.max(np.abs(back - Xd)) <= 1e-5 * np.max(np.abs(Xd))
+
+
+def _mxfp8_rtn(x: np.ndarray):
+    rows, K = x.shape
+    blocks = x.reshape(rows, K // 32, 32).astype(np.float64)
+    amax = np.abs(blocks).max(axis=2)
+    with np.errstate(divide="ignore"):
+        e = np.where(amax > 0, np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - 8, -127)
+    e = np.clip(e, -127, 127)
+    v = (blocks / np.exp2(e)[..., None]).astype(np.float32).reshape(rows, K)
+    v = np.where(v == 0, np.float32(0.0), v)
+    return _e4m3_by_binade(v), (e + 127).astype(np.uint8)
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e2m1"])
+def test_kv_identity_is_rtn_and_scatter(fmt):
+    """Identity factors, no clip: each head vector is plain MX RTN (KV8 / KV4), stored at
+    its slot; slot -1 and slots no token names keep their old contents."""
+    T, H, D, S = 5, 3, 64, 9
+    kv = wl.random_bf16((T, H, D), seed=90, scale=2.0)
+    A = np.eye(8, dtype=np.float32)
+    B = np.repeat(np.eye(4, dtype=np.float32)[None], D // 32, axis=0)
+    slots = np.array([4, -1, 0, 8, 2])
+    cc = np.full((S, H, D), 0x5A, np.uint8)
+    cs = np.full((S, H, D // 32), 0xA5, np.uint8)
+    oracle.kv_quantize(kv, A, B, None, None, fmt, slots, cc, cs)
+    x = wl.bf16_bits_to_f32(kv).reshape(T * H, D)
+    rc, rs = _mxfp8_rtn(x) if fmt == "e4m3" else _rtn_mxfp4(x)
+    rc, rs = rc.reshape(T, H, D), rs.reshape(T, H, D // 32)
+    for t, sl in enumerate(slots):
+        if sl >= 0:
+            assert np.array_equal(cc[sl], rc[t]) and np.array_equal(cs[sl], rs[t])
+    for sl in (1, 3, 5, 6, 7):
+        assert np.all(cc[sl] == 0x5A) and np.all(cs[sl] == 0xA5)
+
+
+def test_kv_head_locality():
+    """Changing one head of one token changes only that head's cache entry."""
+    T, H, D = 4, 4, 128
+    kv = wl.random_bf16((T, H, D), seed=91)
+    A, B, g_lo, g_hi = wl.random_factors(D // 32, seed=92)
+    slots = np.arange(T)
+    c0 = np.zeros((T, H, D), np.uint8); s0 = np.zeros((T, H, D // 32), np.uint8)
+    c1 = c0.copy(); s1 = s0.copy()
+    oracle.kv_quantize(kv, A, B, g_lo, g_hi, "e4m3", slots, c0, s0)
+    kv2 = kv.copy()
+    kv2[2, 1] = wl.random_bf16((D,), seed=93, scale=10.0)
+    oracle.kv_quantize(kv2, A, B, g_lo, g_hi, "e4m3", slots, c1, s1)
+    diff = np.any(c0 != c1, axis=2) | np.any(s0 != s1, axis=2)
+    assert diff[2, 1] and diff.sum() == 1
+
+
+def test_kv_roundtrip_with_inverse_factors():
+    """Dequantizing the cache through B^-1 (x) A^-1 gives back K within the MX error;
+    the transposed inverse (a plausible orientation slip) does not."""
+    T, H, D = 16, 2, 128
+    kv = wl.random_bf16((T, H, D), seed=94, scale=1.5)
+    A, B, _, _ = wl.random_factors(D // 32, seed=95)
+    Ai = oracle.inverse(A.astype(np.float64)).astype(np.float32)
+    Bi = np.stack([oracle.inverse(b.astype(np.float64)) for b in B]).astype(np.float32)
+    x = wl.bf16_bits_to_f32(kv).astype(np.float64)
+    for fmt, tol in (("e4m3", 0.05), ("e2m1", 0.25)):
+        cc = np.zeros((T, H, D), np.uint8); cs = np.zeros((T, H, D // 32), np.uint8)
+        oracle.kv_quantize(kv, A, B, None, None, fmt, np.arange(T), cc, cs)
+        back = oracle.kv_dequantize(cc, cs, np.arange(T), fmt, Ai, Bi)
+        rel = np.linalg.norm(back - x) / np.linalg.norm(x)
+        assert rel < tol, (fmt, rel)
+        wrong = oracle.kv_dequantize(cc, cs, np.arange(T), fmt, Ai.T.copy(),
+                                     np.ascontiguousarray(Bi.transpose(0, 2, 1)))
+        assert np.linalg.norm(wrong - x) / np.linalg.norm(x) > 2 * rel
