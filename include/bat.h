@@ -233,6 +233,61 @@ BAT_API bat_status_t bat_w4a8_gemm(const bat_mxfp8_t* Xq, const bat_mxfp4_t* Wq,
                                    bat_out_dtype_t out_dtype, void* stream);
 
 /*
+ * KV-cache path (the BATQuant note, Key Designs 4 "Equivalent Transformer
+ * integration": transform sets on the per-head key and value cache paths; the KV8
+ * and KV4 settings of Loss & Training store the cache in MXFP8 / MXFP4).
+ *
+ * Every head vector of D = head_dim channels (D % 32 == 0, 32 <= D <= 256) goes
+ * through the block transform x_b (B_b (x) A) with the same factors for every head
+ * (A: device fp32 [s][s]; B: device fp32 [D/32][32/s][32/s], one per 32-channel
+ * block of the head; s as in bat_quantize_act_gpk), the block clip with logits
+ * g_lo, g_hi (device fp32 [D/32], shared by heads and tokens; both NULL for no
+ * clip), and MX quantization (reading of bat_quantize_act for KV4, of
+ * bat_quantize_act_mxfp8 for KV8). The transform is computed in fp32.
+ *
+ * Cache layout (caller-owned device buffers of num_slots rows):
+ *   codes : [num_slots][H][D] E4M3 bytes (BAT_KV_MXFP8) or [num_slots][H][D/2]
+ *           packed E2M1 (BAT_KV_MXFP4, element 2i in the low nibble), 16-byte aligned;
+ *   scales: [num_slots][H][D/32] UE8M0 bytes, plain row-major.
+ * A paged cache is the same buffers indexed by slot = page * page_size + offset.
+ */
+typedef enum { BAT_KV_MXFP8 = 0, BAT_KV_MXFP4 = 1 } bat_kv_format_t;
+
+/* Buffer sizes of a cache of num_slots rows (0 for an invalid shape or format). */
+BAT_API size_t bat_kv_codes_bytes(int64_t num_slots, int64_t H, int64_t D, bat_kv_format_t fmt);
+BAT_API size_t bat_kv_scales_bytes(int64_t num_slots, int64_t H, int64_t D);
+
+/*
+ * Quantize T new tokens' K (or V) into the cache.
+ *   kv    : device bf16 [T][H][D], 16-byte aligned.
+ *   slots : device int64 [T], 8-byte aligned: cache row of token t; -1 skips the
+ *           token. A slot >= num_slots is skipped and sets the device error word
+ *           (bat_device_error), since it cannot be checked on the host without a copy.
+ *   y_out : optional device fp32 [T][H][D] trace of the transformed values (NULL to skip).
+ * Errors: BAT_ERR_UNSUPPORTED (s), BAT_ERR_SHAPE (D), BAT_ERR_INVALID_ARG (null
+ * pointers, sizes < 1, one clip logit array only), BAT_ERR_ALIGN.
+ */
+BAT_API bat_status_t bat_kv_quantize(const void* kv, int64_t T, int64_t H, int64_t D,
+                                     const float* A, int shared, const float* B,
+                                     const float* g_lo, const float* g_hi, const int64_t* slots,
+                                     bat_kv_format_t fmt, void* cache_codes, void* cache_scales,
+                                     int64_t num_slots, float* y_out, void* stream);
+
+/*
+ * Read T cache rows back: out[t][h][:] = the dequantized values of row slots[t]
+ * (E4M3 / E2M1 element times 2^(scale - 127)), and, when A and B are given, those
+ * values multiplied per 32-channel block by B_b (x) A (pass the inverse factors
+ * A^-1 and B_b^-1, split s, to undo the transform). out: device [T][H][D] in
+ * out_dtype, 16-byte aligned. A slot outside [0, num_slots) gives zeros and sets
+ * the device error word. Errors as bat_kv_quantize.
+ */
+BAT_API bat_status_t bat_kv_dequantize(const void* cache_codes, const void* cache_scales,
+                                       int64_t num_slots, int64_t H, int64_t D,
+                                       bat_kv_format_t fmt, const int64_t* slots, int64_t T,
+                                       const float* A, int shared, const float* B, void* out,
+                                       bat_out_dtype_t out_dtype, void* stream);
+
+/*
  * Block-scaled MXFP4 GEMM on the 5th-generation tensor cores (tcgen05,
  * kind::mxf4, fp32 accumulation in tensor memory):
  *   Y[m][n] = sum_b 2^(eX[m][b] + eW[n][b]) * sum_{j<32} x[m][32b+j] * w[n][32b+j]

@@ -529,3 +529,120 @@ def test_w4a8_errors(bat):
         bat.bat_w4a8_gemm(Xq, Wq)  # K % 128 != 0
     assert e.value.status == 2
     assert bat.bat_device_error() == 0
+
+
+# ---------------------------------------------------------------- KV-cache path
+def _kv_host(cache, fmt):
+    S, H, D = cache.num_slots, cache.H, cache.D
+    raw = cache.codes.cpu().numpy()
+    codes = raw.reshape(S, H, D) if fmt == "mxfp8" else \
+        formats.unpack_codes(raw.reshape(S * H, D // 2)).reshape(S, H, D)
+    return codes, cache.scales.cpu().numpy().reshape(S, H, D // 32)
+
+
+def _kv_case(bat, T, H, D, S, fmt, s=8, clip=True, seed=0):
+    kv = wl.random_bf16((T, H, D), seed=seed + 100, scale=2.0)
+    A, B, g_lo, g_hi = wl.random_factors(D // 32, seed=seed + 101, shared=s)
+    if not clip:
+        g_lo = g_hi = None
+    rng = np.random.default_rng(seed)
+    slots = rng.permutation(S)[:T].astype(np.int64)
+    slots[rng.random(T) < 0.2] = -1
+    cache = bat.KVCache.empty(S, H, D, fmt)
+    cache.codes.fill_(0x5A)
+    cache.scales.fill_(0xA5)
+    y = torch.empty(T, H, D, dtype=torch.float32, device="cuda")
+    Ad, Bd = _dev_f32(A), _dev_f32(B)
+    gl = None if g_lo is None else _dev_f32(g_lo)
+    gh = None if g_hi is None else _dev_f32(g_hi)
+    sd = torch.from_numpy(slots).cuda()
+    bat.bat_kv_quantize(_dev_bf16(kv), Ad, Bd, sd, cache, gl, gh, y_out=y)
+    torch.cuda.synchronize()
+    return kv, A, B, g_lo, g_hi, slots, cache, y.cpu().numpy(), sd
+
+
+@pytest.mark.parametrize("fmt", ["mxfp8", "mxfp4"])
+@pytest.mark.parametrize("T,H,D,S,s", [(1, 8, 128, 4, 8), (37, 8, 128, 64, 8), (5, 3, 64, 9, 4),
+                                       (4, 2, 96, 7, 2), (3, 2, 256, 5, 16), (16, 4, 128, 20, 1),
+                                       (6, 2, 128, 8, 32)])
+def test_kv_quantize_parity(bat, fmt, T, H, D, S, s):
+    kv, A, B, g_lo, g_hi, slots, cache, y_gpu, _ = _kv_case(bat, T, H, D, S, fmt, s, seed=T + D)
+    nb = D // 32
+    _check_transform(y_gpu.reshape(T * H, D), oracle.transform(kv.reshape(T * H, D), A, B))
+    r_lo = oracle.clip_ratios(g_lo, nb)
+    r_hi = oracle.clip_ratios(g_hi, nb)
+    ofmt = "e4m3" if fmt == "mxfp8" else "e2m1"
+    oc, os_, bad = oracle.quantize(y_gpu.reshape(T * H, D), r_lo, r_hi, fmt=ofmt)
+    assert bad == 0
+    oc, os_ = oc.reshape(T, H, D), os_.reshape(T, H, nb)
+    codes, scales = _kv_host(cache, fmt)
+    for t in range(T):
+        if slots[t] >= 0:
+            assert np.array_equal(codes[slots[t]], oc[t]), t
+            assert np.array_equal(scales[slots[t]], os_[t]), t
+    untouched = np.setdiff1d(np.arange(S), slots[slots >= 0])
+    raw = cache.codes.cpu().numpy().reshape(S, -1)
+    assert np.all(raw[untouched] == 0x5A)
+    assert np.all(scales[untouched] == 0xA5)
+    assert bat.bat_device_error() == 0
+
+
+@pytest.mark.parametrize("fmt", ["mxfp8", "mxfp4"])
+def test_kv_dequantize_parity(bat, fmt):
+    T, H, D, S = 24, 4, 128, 32
+    kv, A, B, g_lo, g_hi, slots, cache, _, _ = _kv_case(bat, T, H, D, S, fmt, seed=7)
+    read = np.array([sl for sl in slots if sl >= 0] + [slots[slots >= 0][0]], np.int64)
+    rd = torch.from_numpy(read).cuda()
+    ofmt = "e4m3" if fmt == "mxfp8" else "e2m1"
+    codes, scales = _kv_host(cache, fmt)
+    # values as stored: exact (fp32 of the fp64 value)
+    v = bat.bat_kv_dequantize(cache, rd).cpu().numpy()
+    ref = oracle.kv_dequantize(codes, scales, read, ofmt)
+    assert np.array_equal(v, ref.astype(np.float32))
+    vb = bat.bat_kv_dequantize(cache, rd, out_dtype=torch.bfloat16).float().cpu().numpy()
+    assert np.array_equal(vb, torch.from_numpy(v).to(torch.bfloat16).float().numpy())
+    # through the inverse factors: back to K / V up to the quantization error
+    Ai = oracle.inverse(A.astype(np.float64)).astype(np.float32)
+    Bi = np.stack([oracle.inverse(b.astype(np.float64)) for b in B]).astype(np.float32)
+    w = bat.bat_kv_dequantize(cache, rd, _dev_f32(Ai), _dev_f32(Bi)).cpu().numpy()
+    refw = oracle.kv_dequantize(codes, scales, read, ofmt, Ai, Bi)
+    _check_transform(w.reshape(-1, D), refw.reshape(-1, D))
+    assert bat.bat_device_error() == 0
+
+
+def test_kv_bad_slot_is_skipped_and_reported(bat):
+    T, H, D, S = 3, 2, 64, 4
+    kv = _dev_bf16(wl.random_bf16((T, H, D), seed=1))
+    A, B, _, _ = wl.random_factors(D // 32, seed=2)
+    cache = bat.KVCache.empty(S, H, D, "mxfp8")
+    cache.codes.fill_(0x5A)
+    slots = torch.tensor([0, S + 5, 2], dtype=torch.int64, device="cuda")
+    bat.bat_kv_quantize(kv, _dev_f32(A), _dev_f32(B), slots, cache)
+    torch.cuda.synchronize()
+    assert bat.bat_device_error() != 0
+    assert bat.bat_device_error() == 0  # read and cleared
+    raw = cache.codes.cpu().numpy().reshape(S, -1)
+    assert np.all(raw[1] == 0x5A) and np.all(raw[3] == 0x5A)
+    out = bat.bat_kv_dequantize(cache, torch.tensor([1, -1, S], dtype=torch.int64, device="cuda"))
+    torch.cuda.synchronize()
+    assert bat.bat_device_error() != 0
+    assert torch.all(out[1:] == 0)
+
+
+@pytest.mark.parametrize("fmt", ["mxfp8", "mxfp4"])
+def test_kv_prefill_size(bat, fmt):
+    """A 4096-token prefill of 8 KV heads x 128 (Qwen3-8B-like), checked on sampled tokens."""
+    T, H, D = 4096, 8, 128
+    kv, A, B, g_lo, g_hi, slots, cache, y_gpu, _ = _kv_case(bat, T, H, D, T, fmt, seed=11)
+    pick = _sample(T, 64, 5)
+    nb = D // 32
+    _check_transform(y_gpu[pick].reshape(-1, D), oracle.transform(kv[pick].reshape(-1, D), A, B))
+    ofmt = "e4m3" if fmt == "mxfp8" else "e2m1"
+    oc, os_, _ = oracle.quantize(y_gpu[pick].reshape(-1, D), oracle.clip_ratios(g_lo, nb),
+                                 oracle.clip_ratios(g_hi, nb), fmt=ofmt)
+    oc, os_ = oc.reshape(len(pick), H, D), os_.reshape(len(pick), H, nb)
+    codes, scales = _kv_host(cache, fmt)
+    for i, t in enumerate(pick):
+        if slots[t] >= 0:
+            assert np.array_equal(codes[slots[t]], oc[i]) and np.array_equal(scales[slots[t]], os_[i])
+    assert bat.bat_device_error() == 0

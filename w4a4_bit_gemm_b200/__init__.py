@@ -71,6 +71,10 @@ def lib() -> ctypes.CDLL:
         "bat_quantize_act_mxfp8": (S, [P, I64, I64, P, S, P, P, P, SP, P, P]),
         "bat_e4m3_encode": (S, [P, I64, P, P]),
         "bat_w4a8_gemm": (S, [SP, SP, P, S, P]),
+        "bat_kv_codes_bytes": (ctypes.c_size_t, [I64, I64, I64, S]),
+        "bat_kv_scales_bytes": (ctypes.c_size_t, [I64, I64, I64]),
+        "bat_kv_quantize": (S, [P, I64, I64, I64, P, S, P, P, P, P, S, P, P, I64, P, P]),
+        "bat_kv_dequantize": (S, [P, P, I64, I64, I64, S, P, I64, P, S, P, P, S, P]),
         "bat_mxfp4_gemm": (S, [SP, SP, P, S, P]),
         "bat_linear_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
         "bat_linear": (S, [P, I64, SP, P, P, P, P, P, S, P, ctypes.c_size_t, P]),
@@ -422,3 +426,69 @@ def bat_linear_noalloc(X, Wq: MXFP4, A, B, g_lo=None, g_hi=None, Y: Optional[tor
 
 def bat_device_error() -> int:
     return lib().bat_device_error()
+
+
+# ---------------------------------------------------------------- KV cache
+BAT_KV_MXFP8, BAT_KV_MXFP4 = 0, 1
+_KV_FMT = {"mxfp8": BAT_KV_MXFP8, "mxfp4": BAT_KV_MXFP4}
+
+
+@dataclass
+class KVCache:
+    """One K (or V) cache: codes [S][H][D] E4M3 or [S][H][D/2] packed E2M1, scales [S][H][D/32]."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    num_slots: int
+    H: int
+    D: int
+    fmt: str
+
+    @staticmethod
+    def empty(num_slots: int, H: int, D: int, fmt: str = "mxfp8", device="cuda") -> "KVCache":
+        f = _KV_FMT[fmt]
+        cb = lib().bat_kv_codes_bytes(num_slots, H, D, f)
+        sb = lib().bat_kv_scales_bytes(num_slots, H, D)
+        if cb == 0 or sb == 0:
+            raise ValueError(f"invalid KV cache shape {num_slots}x{H}x{D}")
+        return KVCache(torch.zeros(cb, dtype=torch.uint8, device=device),
+                       torch.zeros(sb, dtype=torch.uint8, device=device), num_slots, H, D, fmt)
+
+
+def bat_kv_quantize(kv, A, B, slots, cache: KVCache, g_lo=None, g_hi=None,
+                    y_out: Optional[torch.Tensor] = None, stream=None) -> KVCache:
+    """Transform, clip and quantize kv [T][H][D] (bf16) into cache rows slots[t] (-1 skips)."""
+    T, H, D = kv.shape
+    _need(kv, torch.bfloat16, "kv")
+    s = _gpk_factors(A, B, D)
+    _need(slots, torch.int64, "slots", (T,))
+    if (g_lo is None) != (g_hi is None):
+        raise ValueError("g_lo and g_hi must both be given or both be None")
+    if g_lo is not None:
+        _need(g_lo, torch.float32, "g_lo", (D // 32,))
+        _need(g_hi, torch.float32, "g_hi", (D // 32,))
+    if y_out is not None:
+        _need(y_out, torch.float32, "y_out", (T, H, D))
+    if cache.H != H or cache.D != D:
+        raise ValueError("cache shape does not match kv")
+    _check(lib().bat_kv_quantize(_ptr(kv), T, H, D, _ptr(A), s, _ptr(B), _ptr(g_lo), _ptr(g_hi),
+                                 _ptr(slots), _KV_FMT[cache.fmt], _ptr(cache.codes),
+                                 _ptr(cache.scales), cache.num_slots, _ptr(y_out),
+                                 _stream(stream)), "bat_kv_quantize")
+    return cache
+
+
+def bat_kv_dequantize(cache: KVCache, slots, A=None, B=None, out: Optional[torch.Tensor] = None,
+                      out_dtype: torch.dtype = torch.float32, stream=None) -> torch.Tensor:
+    """Values of cache rows slots[t] as [T][H][D]; with A, B also multiplied by B_b (x) A."""
+    T = slots.shape[0]
+    _need(slots, torch.int64, "slots", (T,))
+    s = 8
+    if A is not None:
+        s = _gpk_factors(A, B, cache.D)
+    code = _out_code(out_dtype)
+    out = torch.empty(T, cache.H, cache.D, dtype=out_dtype, device=cache.codes.device) if out is None else out
+    _need(out, out_dtype, "out", (T, cache.H, cache.D))
+    _check(lib().bat_kv_dequantize(_ptr(cache.codes), _ptr(cache.scales), cache.num_slots, cache.H,
+                                   cache.D, _KV_FMT[cache.fmt], _ptr(slots), T, _ptr(A), s, _ptr(B),
+                                   _ptr(out), code, _stream(stream)), "bat_kv_dequantize")
+    return out

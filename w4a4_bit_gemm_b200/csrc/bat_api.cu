@@ -14,6 +14,7 @@
 #include "../../include/bat.h"
 #include "bat_common.cuh"
 #include "bat_gemm.cuh"
+#include "bat_kv.cuh"
 #include "bat_prologue.cuh"
 
 namespace {
@@ -554,6 +555,124 @@ bat_status_t bat_quantize_act_mxfp8(const void* X, int64_t M, int64_t K, const f
   if (y_out && !aligned16(y_out)) return BAT_ERR_ALIGN;
   return launch_prologue(X, M, K, A, B, g_lo, g_hi, false, Xq, y_out,
                          static_cast<cudaStream_t>(stream), ls, true);
+}
+
+size_t bat_kv_codes_bytes(int64_t num_slots, int64_t H, int64_t D, bat_kv_format_t fmt) {
+  if (num_slots < 1 || H < 1 || D < 32 || D % 32 != 0) return 0;
+  if (fmt != BAT_KV_MXFP8 && fmt != BAT_KV_MXFP4) return 0;
+  const size_t n = static_cast<size_t>(num_slots) * static_cast<size_t>(H) * static_cast<size_t>(D);
+  return fmt == BAT_KV_MXFP8 ? n : n / 2;
+}
+
+size_t bat_kv_scales_bytes(int64_t num_slots, int64_t H, int64_t D) {
+  if (num_slots < 1 || H < 1 || D < 32 || D % 32 != 0) return 0;
+  return static_cast<size_t>(num_slots) * static_cast<size_t>(H) * static_cast<size_t>(D / 32);
+}
+
+static bat_status_t kv_shape_check(int64_t T, int64_t H, int64_t D, int64_t num_slots, int shared,
+                                   int* ls) {
+  *ls = shared_log2(shared);
+  if (*ls < 0) return BAT_ERR_UNSUPPORTED;
+  if (T < 1 || H < 1 || num_slots < 1) return BAT_ERR_INVALID_ARG;
+  if (D < 32 || D % 32 != 0 || D > 32 * bat::kv::kMaxBlocks) return BAT_ERR_SHAPE;
+  return BAT_OK;
+}
+
+static unsigned kv_grid(int64_t items, int sms) {
+  const int64_t want = (items + bat::kv::kWarps - 1) / bat::kv::kWarps;
+  const int64_t cap = static_cast<int64_t>(sms) * 8;
+  return static_cast<unsigned>(want < cap ? want : cap);
+}
+
+bat_status_t bat_kv_quantize(const void* kv, int64_t T, int64_t H, int64_t D, const float* A,
+                             int shared, const float* B, const float* g_lo, const float* g_hi,
+                             const int64_t* slots, bat_kv_format_t fmt, void* cache_codes,
+                             void* cache_scales, int64_t num_slots, float* y_out, void* stream) {
+  int ls = 0;
+  bat_status_t st = kv_shape_check(T, H, D, num_slots, shared, &ls);
+  if (st != BAT_OK) return st;
+  if (fmt != BAT_KV_MXFP8 && fmt != BAT_KV_MXFP4) return BAT_ERR_INVALID_ARG;
+  if (!kv || !A || !B || !slots || !cache_codes || !cache_scales) return BAT_ERR_INVALID_ARG;
+  if ((g_lo == nullptr) != (g_hi == nullptr)) return BAT_ERR_INVALID_ARG;
+  if (!aligned16(kv) || !aligned16(cache_codes) || !aligned16(A) || !aligned16(B) ||
+      (reinterpret_cast<uintptr_t>(slots) & 7u) != 0 || (y_out && !aligned16(y_out)))
+    return BAT_ERR_ALIGN;
+  int dev = 0, sms = 0;
+  st = current_device(&dev, &sms);
+  if (st != BAT_OK) return st;
+  bat::KvParams p;
+  p.kv = static_cast<const uint16_t*>(kv);
+  p.a = A;
+  p.b = B;
+  p.g_lo = g_lo;
+  p.g_hi = g_hi;
+  p.slots = slots;
+  p.codes = static_cast<uint8_t*>(cache_codes);
+  p.scales = static_cast<uint8_t*>(cache_scales);
+  p.y_out = y_out;
+  p.T = T;
+  p.H = H;
+  p.S = num_slots;
+  p.D = static_cast<int>(D);
+  p.nbh = static_cast<int>(D / 32);
+  p.groups = (p.nbh + 3) / 4;
+  p.ls = ls;
+  const unsigned grid = kv_grid(T * H * p.groups, sms);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool fp8 = fmt == BAT_KV_MXFP8;
+  if (fp8)
+    (y_out ? bat::bat_kv_quantize_kernel<true, true> : bat::bat_kv_quantize_kernel<true, false>)
+        <<<grid, bat::kv::kThreads, 0, s>>>(p);
+  else
+    (y_out ? bat::bat_kv_quantize_kernel<false, true> : bat::bat_kv_quantize_kernel<false, false>)
+        <<<grid, bat::kv::kThreads, 0, s>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
+bat_status_t bat_kv_dequantize(const void* cache_codes, const void* cache_scales,
+                               int64_t num_slots, int64_t H, int64_t D, bat_kv_format_t fmt,
+                               const int64_t* slots, int64_t T, const float* A, int shared,
+                               const float* B, void* out, bat_out_dtype_t out_dtype,
+                               void* stream) {
+  int ls = 0;
+  bat_status_t st = kv_shape_check(T, H, D, num_slots, shared, &ls);
+  if (st != BAT_OK) return st;
+  if (fmt != BAT_KV_MXFP8 && fmt != BAT_KV_MXFP4) return BAT_ERR_INVALID_ARG;
+  if (out_dtype != BAT_OUT_BF16 && out_dtype != BAT_OUT_F32) return BAT_ERR_INVALID_ARG;
+  if (!cache_codes || !cache_scales || !slots || !out) return BAT_ERR_INVALID_ARG;
+  if ((A == nullptr) != (B == nullptr)) return BAT_ERR_INVALID_ARG;
+  if (!aligned16(cache_codes) || !aligned16(out) || (reinterpret_cast<uintptr_t>(slots) & 7u) != 0 ||
+      (A && (!aligned16(A) || !aligned16(B))))
+    return BAT_ERR_ALIGN;
+  int dev = 0, sms = 0;
+  st = current_device(&dev, &sms);
+  if (st != BAT_OK) return st;
+  bat::KvReadParams p;
+  p.codes = static_cast<const uint8_t*>(cache_codes);
+  p.scales = static_cast<const uint8_t*>(cache_scales);
+  p.slots = slots;
+  p.a = A;
+  p.b = B;
+  p.out = out;
+  p.T = T;
+  p.H = H;
+  p.S = num_slots;
+  p.D = static_cast<int>(D);
+  p.nbh = static_cast<int>(D / 32);
+  p.groups = (p.nbh + 3) / 4;
+  p.ls = ls;
+  const unsigned grid = kv_grid(T * H * p.groups, sms);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void (*k)(bat::KvReadParams);
+  const bool fp8 = fmt == BAT_KV_MXFP8, xf = A != nullptr, f32 = out_dtype == BAT_OUT_F32;
+  if (fp8)
+    k = xf ? (f32 ? bat::bat_kv_dequantize_kernel<true, true, true> : bat::bat_kv_dequantize_kernel<true, true, false>)
+           : (f32 ? bat::bat_kv_dequantize_kernel<true, false, true> : bat::bat_kv_dequantize_kernel<true, false, false>);
+  else
+    k = xf ? (f32 ? bat::bat_kv_dequantize_kernel<false, true, true> : bat::bat_kv_dequantize_kernel<false, true, false>)
+           : (f32 ? bat::bat_kv_dequantize_kernel<false, false, true> : bat::bat_kv_dequantize_kernel<false, false, false>);
+  k<<<grid, bat::kv::kThreads, 0, s>>>(p);
+  return cuda_status(cudaGetLastError());
 }
 
 bat_status_t bat_w4a8_gemm(const bat_mxfp8_t* Xq, const bat_mxfp4_t* Wq, void* Y,

@@ -20,7 +20,14 @@ enum DevError : unsigned int {
   kErrWaitEmpty = 2u,
   kErrWaitTmemFull = 4u,
   kErrWaitTmemEmpty = 8u,
+  kErrBadIndex = 16u,  // a cache slot index outside [0, num_slots) (the access is skipped)
 };
+
+// fp32(sigma(g)) evaluated in fp64; +inf gives exactly 1.
+__device__ __forceinline__ float clip_ratio(float g) {
+  if (isinf(g) && g > 0.0f) return 1.0f;
+  return static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(g))));
+}
 
 // ---------------------------------------------------------------- small helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -1,0 +1,244 @@
+// KV-cache path of the BATQuant transformer integration (BATQuant note,
+// en.papernotes.org, Method > Key Designs 4 "Equivalent Transformer integration":
+// one transform set on the per-head key cache path and one on the value path;
+// the KV8 / KV4 settings of Loss & Training store the cache in MXFP8 (E4M3) /
+// MXFP4).
+//
+// Every head's D-vector (D = head_dim, a multiple of 32) goes through the block
+// transform y_b = x_b (B_b (x) A) with the same factors for all heads (A s x s
+// shared, B_b (32/s) x (32/s) for each 32-channel block of the head), the
+// block clip with per-block logits shared by heads and tokens, and MX
+// quantization; the codes and the scale byte go to the token's cache slot.
+//
+// The work per element is small (one 32 x 32 block product) and the step is
+// usually a decode step of a few tokens, so this is a CUDA-core kernel sized for
+// latency: a warp takes one (token, head, group of four blocks); lane l holds
+// elements 4(l%8) .. 4(l%8)+3 of block l/8; the block's 32 inputs are exchanged
+// with shuffles and multiplied by the fp32 block P_b, which each CTA builds once
+// in shared memory. Block min/max come from an 8-lane butterfly.
+#pragma once
+
+#include "bat_common.cuh"
+
+namespace bat {
+
+namespace kv {
+constexpr int kWarps = 8;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kMaxBlocks = 8;     // D <= 256: P blocks staged in shared memory (32 KB)
+constexpr int kFacFloats = 2112;  // A and B staged for the build when they fit (s >= 2)
+}  // namespace kv
+
+struct KvParams {
+  const uint16_t* kv;     // bf16 [T][H][D]
+  const float* a;         // [s][s]
+  const float* b;         // [D/32][t][t]
+  const float* g_lo;      // [D/32] clip logits, or null (no clip)
+  const float* g_hi;
+  const int64_t* slots;   // [T]: cache row of token t, -1 to skip
+  uint8_t* codes;         // cache codes [S][H][D] (E4M3) or [S][H][D/2] (E2M1)
+  uint8_t* scales;        // cache scales [S][H][D/32]
+  float* y_out;           // optional fp32 [T][H][D] trace of the transformed values
+  int64_t T, H, S;
+  int D, nbh, groups, ls; // nbh = D/32, groups = ceil(nbh/4), ls = log2 s
+};
+
+struct KvReadParams {
+  const uint8_t* codes;   // cache codes
+  const uint8_t* scales;  // cache scales [S][H][D/32]
+  const int64_t* slots;   // [T]: cache rows to read
+  const float* a;         // optional output factors (null: values as stored)
+  const float* b;
+  void* out;              // [T][H][D] fp32 or bf16
+  int64_t T, H, S;
+  int D, nbh, groups, ls;
+};
+
+// P_b[k][n] = B_b[k/s][n/s] * A[k%s][n%s] in fp32 for the head's nbh blocks. A and B
+// are first copied to `fac` with coalesced loads when they fit (every split but s = 1,
+// whose 32 x 32 private factors are read where they are). Ends with a CTA barrier.
+__device__ __forceinline__ void kv_build_p(float* sp, float* fac, const float* a, const float* b,
+                                           int nbh, int ls) {
+  const int sm = (1 << ls) - 1, t = 32 >> ls;
+  const int na = 1 << (2 * ls), nbf = nbh << (10 - 2 * ls);
+  const bool staged = (na + 3) / 4 * 4 + nbf <= kv::kFacFloats;
+  const float* sa = a;
+  const float* sb = b;
+  if (staged) {
+    float* fb = fac + (na + 3) / 4 * 4;
+    for (int i = threadIdx.x; i < na; i += blockDim.x) fac[i] = a[i];
+    for (int i = threadIdx.x; i < nbf; i += blockDim.x) fb[i] = b[i];
+    __syncthreads();
+    sa = fac;
+    sb = fb;
+  }
+  for (int i = threadIdx.x; i < nbh * 1024; i += blockDim.x) {
+    const int blk = i >> 10, k = (i >> 5) & 31, n = i & 31;
+    sp[i] = __fmul_rn(sb[(blk * t + (k >> ls)) * t + (n >> ls)], sa[((k & sm) << ls) + (n & sm)]);
+  }
+  __syncthreads();
+}
+
+// y[0..3] = outputs 4u..4u+3 of the lane's block: sum over k of x[k] * P[k][n],
+// x[k] held by lane (l & ~7) + k/4 as its element k%4; k ascending.
+__device__ __forceinline__ void kv_block_product(const float* pblk, const float (&x)[4], int lane,
+                                                 float (&y)[4]) {
+  const int base = lane & ~7, u = lane & 7;
+  y[0] = y[1] = y[2] = y[3] = 0.0f;
+#pragma unroll
+  for (int src = 0; src < 8; ++src) {
+    float xs[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) xs[i] = __shfl_sync(0xffffffffu, x[i], base + src);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 pr = *reinterpret_cast<const float4*>(pblk + (4 * src + i) * 32 + 4 * u);
+      y[0] = __fmaf_rn(xs[i], pr.x, y[0]);
+      y[1] = __fmaf_rn(xs[i], pr.y, y[1]);
+      y[2] = __fmaf_rn(xs[i], pr.z, y[2]);
+      y[3] = __fmaf_rn(xs[i], pr.w, y[3]);
+    }
+  }
+}
+
+template <bool kFp8, bool kTrace>
+__global__ void __launch_bounds__(kv::kThreads)
+    bat_kv_quantize_kernel(const KvParams p) {
+  __shared__ __align__(16) float sp[kv::kMaxBlocks * 1024];
+  __shared__ __align__(16) float fac[kv::kFacFloats];
+  __shared__ float ratio[2 * kv::kMaxBlocks];
+  if (threadIdx.x < 2 * p.nbh) {  // clip ratios of the head's blocks: lo, then hi
+    const float* g = threadIdx.x < p.nbh ? p.g_lo : p.g_hi;
+    ratio[threadIdx.x] = g ? clip_ratio(g[threadIdx.x % p.nbh]) : 1.0f;
+  }
+  kv_build_p(sp, fac, p.a, p.b, p.nbh, p.ls);
+  const int lane = threadIdx.x & 31;
+  const int u = lane & 7;
+  const int64_t items = p.T * p.H * p.groups;
+  const int64_t wstride = static_cast<int64_t>(gridDim.x) * kv::kWarps;
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * kv::kWarps + (threadIdx.x >> 5); it < items;
+       it += wstride) {
+    const int g = static_cast<int>(it % p.groups);
+    const int64_t th = it / p.groups;  // token * H + head
+    const int64_t t = th / p.H;
+    const int blk = 4 * g + (lane >> 3);
+    const bool has = blk < p.nbh;  // lanes of a missing fourth block idle (shuffles stay full)
+    const int64_t slot = p.slots[t];
+    if (slot >= p.S) {
+      if (lane == 0) atomicOr(&g_dev_error, kErrBadIndex);
+      continue;
+    }
+    float x[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const int64_t e0 = th * p.D + blk * kG + 4 * u;
+    if (has) {
+      const uint2 w = *reinterpret_cast<const uint2*>(p.kv + e0);
+      x[0] = bf16lo(w.x);
+      x[1] = bf16hi(w.x);
+      x[2] = bf16lo(w.y);
+      x[3] = bf16hi(w.y);
+    }
+    float y[4];
+    kv_block_product(sp + (has ? blk : 0) * 1024, x, lane, y);
+    if (kTrace && has)
+      *reinterpret_cast<float4*>(p.y_out + e0) = make_float4(y[0], y[1], y[2], y[3]);
+    // block min / max over the block's 8 lanes
+    float mn = fminf(fminf(y[0], y[1]), fminf(y[2], y[3]));
+    float mx = fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if (!has || slot < 0) continue;
+    const float r_lo = ratio[blk];
+    const float r_hi = ratio[p.nbh + blk];
+    const float lo = __fmul_rn(r_lo, mn);
+    const float hi = __fmul_rn(r_hi, mx);
+    const float amax = fmaxf(fabsf(fminf(fmaxf(mn, lo), hi)), fabsf(fminf(fmaxf(mx, lo), hi)));
+    constexpr int kEmax = kFp8 ? 8 : 2;
+    const int efield = static_cast<int>(__float_as_uint(amax) >> 23);
+    const int sbyte = efield > kEmax ? efield - kEmax : 0;  // e + 127
+    const float inv_scale = __uint_as_float(static_cast<uint32_t>(254 - sbyte) << 23);  // 2^-e
+    float v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = __fmaf_rn(fminf(fmaxf(y[i], lo), hi), inv_scale, 0.0f);
+    const int64_t crow = (slot * p.H + th % p.H) * p.D + blk * kG + 4 * u;  // element index
+    if (kFp8) {
+      *reinterpret_cast<uint32_t*>(p.codes + crow) = e4m3x4(v[0], v[1], v[2], v[3]);
+    } else {
+      const uint32_t c = e2m1x2(v[0], v[1]) | (e2m1x2(v[2], v[3]) << 8);
+      *reinterpret_cast<uint16_t*>(p.codes + crow / 2) = static_cast<uint16_t>(c);
+    }
+    if (u == 0) p.scales[(slot * p.H + th % p.H) * p.nbh + blk] = static_cast<uint8_t>(sbyte);
+  }
+}
+
+// E4M3 / E2M1 code -> value (exact in fp32).
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+  const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+  if ((c & 0x7Fu) == 0x7Fu) return __uint_as_float(0x7FC00000u);
+  const float mag = e == 0 ? static_cast<float>(m) * 0x1p-9f
+                           : __uint_as_float(((e + 120u) << 23) | (m << 20));
+  return (c & 0x80u) ? -mag : mag;
+}
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+  const uint32_t i = c & 7u;
+  // 0, 0.5, 1, 1.5 (i < 4) then 2, 3, 4, 6
+  const float mag = i < 4 ? 0.5f * static_cast<float>(i) : static_cast<float>((i & 1 ? 3 : 2) << ((i - 4) >> 1));
+  return (c & 8u) ? -mag : mag;
+}
+
+template <bool kFp8, bool kXform, bool kF32Out>
+__global__ void __launch_bounds__(kv::kThreads)
+    bat_kv_dequantize_kernel(const KvReadParams p) {
+  __shared__ __align__(16) float sp[kXform ? kv::kMaxBlocks * 1024 : 4];
+  __shared__ __align__(16) float fac[kXform ? kv::kFacFloats : 4];
+  if (kXform) kv_build_p(sp, fac, p.a, p.b, p.nbh, p.ls);
+  const int lane = threadIdx.x & 31;
+  const int u = lane & 7;
+  const int64_t items = p.T * p.H * p.groups;
+  const int64_t wstride = static_cast<int64_t>(gridDim.x) * kv::kWarps;
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * kv::kWarps + (threadIdx.x >> 5); it < items;
+       it += wstride) {
+    const int g = static_cast<int>(it % p.groups);
+    const int64_t th = it / p.groups;
+    const int64_t t = th / p.H;
+    const int blk = 4 * g + (lane >> 3);
+    const bool has = blk < p.nbh;
+    const int64_t slot = p.slots[t];
+    const bool ok = slot >= 0 && slot < p.S;
+    if (!ok && lane == 0) atomicOr(&g_dev_error, kErrBadIndex);
+    float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (has && ok) {
+      const int64_t crow = (slot * p.H + th % p.H) * p.D + blk * kG + 4 * u;
+      const uint32_t sb = p.scales[(slot * p.H + th % p.H) * p.nbh + blk];
+      const float sc = sb == 255u ? __uint_as_float(0x7FC00000u)
+                                  : (sb == 0u ? 0x1p-127f : __uint_as_float(sb << 23));
+      if (kFp8) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(p.codes + crow);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = e4m3_value((w >> (8 * i)) & 0xFFu) * sc;
+      } else {
+        const uint32_t w = *reinterpret_cast<const uint16_t*>(p.codes + crow / 2);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = e2m1_value((w >> (4 * i)) & 0xFu) * sc;
+      }
+    }
+    float y[4] = {v[0], v[1], v[2], v[3]};
+    if (kXform) kv_block_product(sp + (has ? blk : 0) * 1024, v, lane, y);
+    if (!has) continue;
+    const int64_t e0 = th * p.D + blk * kG + 4 * u;
+    if (kF32Out) {
+      *reinterpret_cast<float4*>(static_cast<float*>(p.out) + e0) = make_float4(y[0], y[1], y[2], y[3]);
+    } else {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(y[0], y[1]);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(y[2], y[3]);
+      uint2 w;
+      w.x = *reinterpret_cast<uint32_t*>(&lo);
+      w.y = *reinterpret_cast<uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.out) + e0) = w;
+    }
+  }
+}
+
+}  // namespace bat

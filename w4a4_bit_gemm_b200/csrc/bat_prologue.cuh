@@ -88,11 +88,6 @@ struct PrologueParams {
   int ls;                // log2 of the shared factor's size: 0..5 (3 is the 8 x 8 / 4 x 4 split)
 };
 
-// fp32(sigma(g)) evaluated in fp64; +inf gives exactly 1.
-__device__ __forceinline__ float clip_ratio(float g) {
-  if (isinf(g) && g > 0.0f) return 1.0f;
-  return static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(g))));
-}
 
 __device__ __forceinline__ int64_t scale_offset(int64_t m, int64_t b, int nbp4) {
   return ((m >> 7) * nbp4 + (b >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (b & 3);
