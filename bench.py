@@ -244,6 +244,158 @@ def run_reference(args, w, inp):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- KV-cache store
+KV_HEADS, KV_DIM = 8, 128  # Qwen3-8B-class attention: 8 KV heads of 128 channels
+
+
+def kv_inputs(T: int, seed: int):
+    """K and V [T][8][128] bf16: N(0,1) with 2 % of the head channels x20 in K (the
+    channel outliers of keys), and the K- and V-path factors and clip logits."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    k = rng.standard_normal((T, KV_HEADS, KV_DIM)).astype(np.float32)
+    ch = rng.choice(KV_DIM, size=max(1, KV_DIM // 50), replace=False)
+    k[:, :, ch] *= 20.0
+    v = rng.standard_normal((T, KV_HEADS, KV_DIM)).astype(np.float32)
+    fk = wl.random_factors(KV_DIM // 32, seed=seed + 1)
+    fv = wl.random_factors(KV_DIM // 32, seed=seed + 2)
+    return wl.f32_to_bf16_bits(k), wl.f32_to_bf16_bits(v), fk, fv
+
+
+def run_kv(args, rank, world, local):
+    import torch
+    import w4a4_bit_gemm_b200 as bat
+    bat.lib()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+    T = args.kv_tokens
+    k_host, v_host, fk, fv = kv_inputs(T, seed=rank_batch_seed(rank))
+
+    def bf16(bits):
+        return torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(dev)
+
+    def f32(a):
+        return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev)
+
+    K, V = bf16(k_host), bf16(v_host)
+    Ak, Bk, glk, ghk = (f32(a) for a in fk)
+    Av, Bv, glv, ghv = (f32(a) for a in fv)
+    S = 2 * T  # a paged cache twice the batch: the tokens land on scattered rows
+    slots = torch.from_numpy(np.random.default_rng(3).permutation(S)[:T].astype(np.int64)).to(dev)
+    ck = bat.KVCache.empty(S, KV_HEADS, KV_DIM, args.kv_format, dev)
+    cv = bat.KVCache.empty(S, KV_HEADS, KV_DIM, args.kv_format, dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_view = flush.view(torch.int32)
+
+    def step(Kin, Vin):
+        bat.bat_kv_quantize(Kin, Ak, Bk, slots, ck, glk, ghk, stream=stream)
+        bat.bat_kv_quantize(Vin, Av, Bv, slots, cv, glv, ghv, stream=stream)
+
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        flush_view.amax()
+        step(K, V)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    if not args.no_clocks and rank == 0:
+        sampler.start()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        flush_view.amax()
+        ev[i][0].record(stream)
+        step(K, V)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    clocks = sampler.stop() if (not args.no_clocks and rank == 0) else None
+    t = max_over_ranks(pg, [sum(e0.elapsed_time(e1) * 1e-3 for e0, e1 in ev)], dev)[0]
+    assert bat.bat_device_error() == 0, "a kernel reported a failure"
+    elems = 2 * T * KV_HEADS * KV_DIM
+    per_elt = 2.0 + (1.0 if args.kv_format == "mxfp8" else 0.5) + 1.0 / 32.0
+    gbs = per_elt * elems * args.steps * world / t / 1e9
+    peaks, peak_src = load_peaks()
+
+    e2e = None
+    if not args.no_e2e:
+        kh = torch.from_numpy(k_host.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+        vh = torch.from_numpy(v_host.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+        ch_codes = torch.empty_like(ck.codes, device="cpu").pin_memory()
+        Kd, Vd = torch.empty_like(K), torch.empty_like(V)
+
+        def e2e_step():
+            Kd.copy_(kh, non_blocking=True)
+            Vd.copy_(vh, non_blocking=True)
+            step(Kd, Vd)
+            ch_codes.copy_(ck.codes, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = max_over_ranks(pg, [e0.elapsed_time(e1) * 1e-3], dev)[0]
+        e2e = {"value": per_elt * elems * args.e2e_steps * world / te / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": int(2 * K.numel() * 2),
+               "d2h_bytes_per_step": int(ck.codes.numel())}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        rng = np.random.default_rng(0)
+        n, dt = 0, 0.0
+        while dt < args.cpu_budget_s and n < T:
+            rows = rng.choice(T, size=min(64, T), replace=False)
+            cc = np.zeros((len(rows), KV_HEADS, KV_DIM), np.uint8)
+            cs = np.zeros((len(rows), KV_HEADS, KV_DIM // 32), np.uint8)
+            t0 = time.perf_counter()
+            ofmt = "e4m3" if args.kv_format == "mxfp8" else "e2m1"
+            oracle.kv_quantize(k_host[rows], *fk, ofmt, np.arange(len(rows)), cc, cs)
+            oracle.kv_quantize(v_host[rows], *fv, ofmt, np.arange(len(rows)), cc, cs)
+            dt += time.perf_counter() - t0
+            n += len(rows)
+        cpu = {"value": per_elt * 2 * n * KV_HEADS * KV_DIM / dt / 1e9, "unit": "GB/s",
+               "cores": oracle.num_threads(), "kind": "oracle",
+               "sample": f"{n} random tokens of K and V (8 heads x 128), batches of 64",
+               "seconds": round(dt, 2)}
+
+    if rank == 0:
+        line = {
+            "metric": f"BAT KV-cache store GB/s (% HBM), {args.kv_format}",
+            "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": args.kv_format, "data": "synthetic",
+            "config": {"workload": f"kv_store T={T}", "tokens": T, "kv_heads": KV_HEADS,
+                       "head_dim": KV_DIM, "cache_rows": S, "format": args.kv_format,
+                       "l2": "flushed between steps (256 MiB write + read outside the timed events)",
+                       "parallelism": f"replicas x{world} (independent token batches)"},
+            "gpu_launches": 2 * args.steps * world,
+            "roofline": {"bound": "hbm", "achieved": gbs / world, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": gbs / world / peaks["hbm_gbs"], "traffic": None,
+                         "kernel": "bat_kv_quantize_kernel", "peak_source": peak_src},
+            "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
 # ---------------------------------------------------------------- GPU leg
 def main():
     ap = argparse.ArgumentParser()
@@ -262,6 +414,10 @@ def main():
                     help="size s of the shared transform factor (A s x s, each B_b 32/s x 32/s)")
     ap.add_argument("--act", default="mxfp4", choices=["mxfp4", "mxfp8"],
                     help="activation format: MXFP4 (W4A4) or MXFP8 E4M3 (W4A8)")
+    ap.add_argument("--path", default="linear", choices=["linear", "kv"],
+                    help="linear layer (default) or the KV-cache store (K and V of --kv-tokens tokens)")
+    ap.add_argument("--kv-tokens", type=int, default=16384)
+    ap.add_argument("--kv-format", default="mxfp8", choices=["mxfp8", "mxfp4"])
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -272,6 +428,9 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             run_reference(args, w, wl.make_inputs(w.name, seed=0))
+        return
+    if args.path == "kv":
+        run_kv(args, rank, world, local)
         return
 
     import torch

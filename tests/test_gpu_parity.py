@@ -120,7 +120,7 @@ def test_quantize_act_workloads(bat, name):
 
 
 @pytest.mark.parametrize("M,K", [(1, 32), (1, 4096), (17, 96), (130, 160), (3, 1056), (129, 4128),
-                                 (64, 1024 + 96)])
+                                 (64, 1024 + 96), (65, 4128), (16, 12288), (2, 262144)])
 def test_quantize_act_ragged(bat, M, K):
     X = wl.random_bf16((M, K), seed=M * 7 + K, scale=3.0)
     A, B, g_lo, g_hi = wl.random_factors(K // 32, seed=K)
@@ -324,7 +324,10 @@ def _gemm_check(bat, Xq, Wq, M, N, K, rows=None, cols=None):
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 256), (64, 128, 256), (1, 8, 32), (17, 200, 96),
                                    (130, 300, 160), (256, 512, 1024), (200, 264, 4128),
-                                   (300, 1000, 2048)])
+                                   (300, 1000, 2048),
+                                   # one row of tiles: split-K over a cluster per tile
+                                   (1, 256, 2048), (100, 520, 1024), (128, 1000, 768),
+                                   (33, 300, 2080), (16, 6144, 4096)])
 def test_gemm_shapes(bat, M, N, K):
     X = wl.random_bf16((M, K), seed=M + 3 * K, scale=2.0)
     W = wl.random_bf16((N, K), seed=N + 5 * K, scale=0.02)
@@ -479,7 +482,8 @@ def _w4a8_check(bat, Xq, Wq, M, N, K, rows=None, cols=None):
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 128), (1, 8, 128), (17, 200, 256), (130, 300, 512),
-                                   (256, 512, 1024), (200, 264, 4096), (300, 1000, 2048)])
+                                   (256, 512, 1024), (200, 264, 4096), (300, 1000, 2048),
+                                   (16, 2048, 1024), (3, 300, 768)])
 def test_w4a8_gemm_shapes(bat, M, N, K):
     X = wl.random_bf16((M, K), seed=M + 7 * K, scale=2.0)
     W = wl.random_bf16((N, K), seed=N + 9 * K, scale=0.02)
@@ -564,7 +568,10 @@ def _kv_case(bat, T, H, D, S, fmt, s=8, clip=True, seed=0):
 @pytest.mark.parametrize("fmt", ["mxfp8", "mxfp4"])
 @pytest.mark.parametrize("T,H,D,S,s", [(1, 8, 128, 4, 8), (37, 8, 128, 64, 8), (5, 3, 64, 9, 4),
                                        (4, 2, 96, 7, 2), (3, 2, 256, 5, 16), (16, 4, 128, 20, 1),
-                                       (6, 2, 128, 8, 32)])
+                                       (6, 2, 128, 8, 32), (511, 8, 128, 600, 8),
+                                       # from 4096 (token, head) rows: the tensor-core prologue
+                                       (512, 8, 128, 600, 8), (2048, 2, 96, 2100, 4),
+                                       (4100, 1, 256, 4200, 16), (700, 8, 64, 800, 1)])
 def test_kv_quantize_parity(bat, fmt, T, H, D, S, s):
     kv, A, B, g_lo, g_hi, slots, cache, y_gpu, _ = _kv_case(bat, T, H, D, S, fmt, s, seed=T + D)
     nb = D // 32
@@ -629,6 +636,22 @@ def test_kv_bad_slot_is_skipped_and_reported(bat):
     assert torch.all(out[1:] == 0)
 
 
+def test_kv_bad_slot_prefill_path(bat):
+    T, H, D, S = 1024, 8, 128, 1100
+    kv = _dev_bf16(wl.random_bf16((T, H, D), seed=3))
+    A, B, _, _ = wl.random_factors(D // 32, seed=4)
+    cache = bat.KVCache.empty(S, H, D, "mxfp4")
+    cache.codes.fill_(0x5A)
+    sl = np.arange(T, dtype=np.int64)
+    sl[5] = S + 1
+    bat.bat_kv_quantize(kv, _dev_f32(A), _dev_f32(B), torch.from_numpy(sl).cuda(), cache)
+    torch.cuda.synchronize()
+    assert bat.bat_device_error() != 0
+    raw = cache.codes.cpu().numpy().reshape(S, -1)
+    assert np.all(raw[5] == 0x5A) and np.all(raw[T:] == 0x5A)
+    assert not np.all(raw[4] == 0x5A)
+
+
 @pytest.mark.parametrize("fmt", ["mxfp8", "mxfp4"])
 def test_kv_prefill_size(bat, fmt):
     """A 4096-token prefill of 8 KV heads x 128 (Qwen3-8B-like), checked on sampled tokens."""
@@ -645,4 +668,19 @@ def test_kv_prefill_size(bat, fmt):
     for i, t in enumerate(pick):
         if slots[t] >= 0:
             assert np.array_equal(codes[slots[t]], oc[i]) and np.array_equal(scales[slots[t]], os_[i])
+    assert bat.bat_device_error() == 0
+
+
+def test_split_k_is_deterministic(bat):
+    """The decode shape runs split-K over clusters; partials are summed in a fixed order."""
+    M, N, K = 16, 6144, 4096
+    X = wl.random_bf16((M, K), seed=21, scale=2.0)
+    W = wl.random_bf16((N, K), seed=22, scale=0.02)
+    A, B, g_lo, g_hi = wl.random_factors(K // 32, seed=23)
+    Ad, Bd = _dev_f32(A), _dev_f32(B)
+    Xq = bat.bat_quantize_act(_dev_bf16(X), Ad, Bd, _dev_f32(g_lo), _dev_f32(g_hi))
+    Wq = bat.bat_prepare_weight(_dev_bf16(W), Ad, Bd)
+    ys = [bat.bat_mxfp4_gemm(Xq, Wq, out_dtype=torch.float32) for _ in range(3)]
+    torch.cuda.synchronize()
+    assert all(torch.equal(ys[0], y) for y in ys[1:])
     assert bat.bat_device_error() == 0

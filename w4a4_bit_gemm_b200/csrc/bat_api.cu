@@ -32,6 +32,7 @@ struct DeviceInfo {
   std::atomic<int> sms{0};
   std::atomic<int> gemm_attr{0};    // bit 0: W4A4 GEMM, bit 1: W4A8 GEMM attribute set
   std::atomic<int> pro_attr{0};     // bit t: the prologue variant t has its smem attribute set
+  std::atomic<int> max_clusters[2][9];  // [W4A8][cluster size]: clusters resident at once, 0 unknown
 };
 DeviceInfo g_dev[64];
 
@@ -231,14 +232,67 @@ bat_status_t check_act_args(const void* X, int64_t M, int64_t K, const float* A,
   return check_mxfp4(Xq, M, K);
 }
 
+// The CUDA-core row quantizer: activation rows (slots == null: codes [rows][D(/2)], tiled
+// scales) or KV-cache rows (token row / H stored at cache slot slots[token]).
+bat_status_t launch_rows(const void* x, int64_t rows, int64_t H, int64_t S,
+                                const int64_t* slots, int64_t D, const float* A, const float* B,
+                                const float* g_lo, const float* g_hi, int ls, bool fp8,
+                                uint8_t* codes, uint8_t* scales, float* y_out, int sms,
+                                cudaStream_t s) {
+  bat::RowQuantParams p;
+  p.x = static_cast<const uint16_t*>(x);
+  p.a = A;
+  p.b = B;
+  p.g_lo = g_lo;
+  p.g_hi = g_hi;
+  p.codes = codes;
+  p.scales = scales;
+  p.y_out = y_out;
+  p.slots = slots;
+  p.rows = rows;
+  p.H = H;
+  p.S = S;
+  p.D = static_cast<int>(D);
+  p.nb = static_cast<int>(D / 32);
+  p.groups = (p.nb + 3) / 4;
+  p.ls = ls;
+  p.nbp4 = (p.nb + 3) / 4;
+  // about 16 warps per SM in all, each group of blocks over a stride of R rows
+  int64_t R = static_cast<int64_t>(sms) * 16 / p.groups;
+  if (R > rows) R = rows;
+  if (R < 1) R = 1;
+  p.R = static_cast<int>(R);
+  const int64_t warps = static_cast<int64_t>(p.groups) * R;
+  const unsigned grid = static_cast<unsigned>((warps + bat::kv::kWarps - 1) / bat::kv::kWarps);
+  const bool kv = slots != nullptr, tr = y_out != nullptr;
+  void (*k)(bat::RowQuantParams);
+  if (kv)
+    k = fp8 ? (tr ? bat::bat_rows_quantize_kernel<true, true, true> : bat::bat_rows_quantize_kernel<true, false, true>)
+            : (tr ? bat::bat_rows_quantize_kernel<false, true, true> : bat::bat_rows_quantize_kernel<false, false, true>);
+  else
+    k = fp8 ? (tr ? bat::bat_rows_quantize_kernel<true, true, false> : bat::bat_rows_quantize_kernel<true, false, false>)
+            : (tr ? bat::bat_rows_quantize_kernel<false, true, false> : bat::bat_rows_quantize_kernel<false, false, false>);
+  k<<<grid, bat::kv::kThreads, 0, s>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
+// Activation batches of at most this many rows run on the CUDA-core row quantizer
+// (its latency is a few microseconds; the tensor-core prologue's set-up costs more).
+constexpr int64_t kRowsCudaCore = 64;
+
 bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float* A,
                              const float* B, const float* g_lo, const float* g_hi, bool per_row,
                              const bat_mxfp4_t* out, float* y_out, cudaStream_t stream,
-                             int ls = 3, bool fp8 = false) {
+                             int ls = 3, bool fp8 = false, const int64_t* kv_slots = nullptr,
+                             int64_t kv_heads = 0, int64_t kv_nslots = 0) {
   int dev = 0, sms = 0;
   bat_status_t st = current_device(&dev, &sms);
   if (st != BAT_OK) return st;
   if (rows >= (int64_t{1} << 31)) return BAT_ERR_SHAPE;  // TMA row coordinates are int32
+  if (!per_row && kv_slots == nullptr && rows <= kRowsCudaCore)
+    return launch_rows(X, rows, 1, 0, nullptr, K, A, B, g_lo, g_hi, ls, fp8,
+                       static_cast<uint8_t*>(out->codes), static_cast<uint8_t*>(out->scales), y_out,
+                       sms, stream);
   CUtensorMap tx;
   if (!make_act_map(&tx, X, rows, K)) return BAT_ERR_CUDA;
   bat::PrologueParams p;
@@ -253,6 +307,9 @@ bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float
   p.K = K;
   p.nb = static_cast<int>(K / 32);
   p.ls = ls;
+  p.slots = kv_slots;
+  p.kv_heads = kv_heads;
+  p.kv_slots = kv_nslots;
   p.nbp2 = (p.nb + 1) / 2;
   p.nbp4 = (p.nb + 3) / 4;
   p.mtiles = (rows + bat::pro::kTok - 1) / bat::pro::kTok;
@@ -266,14 +323,23 @@ bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float
     p.cps = cps < 1 ? 1 : cps;
   }
   void (*kern)(CUtensorMap, bat::PrologueParams);
-  if (fp8)  // activations only: clip logits per block
+  const bool kv = kv_slots != nullptr;
+  if (kv) {  // KV-cache store: rows are (token, head), codes and scales go to cache slots
+    if (fp8)
+      kern = y_out ? bat::bat_prologue_kernel<true, false, true, true>
+                   : bat::bat_prologue_kernel<false, false, true, true>;
+    else
+      kern = y_out ? bat::bat_prologue_kernel<true, false, false, true>
+                   : bat::bat_prologue_kernel<false, false, false, true>;
+  } else if (fp8)  // activations only: clip logits per block
     kern = y_out ? bat::bat_prologue_kernel<true, false, true> : bat::bat_prologue_kernel<false, false, true>;
   else if (per_row)
     kern = y_out ? bat::bat_prologue_kernel<true, true> : bat::bat_prologue_kernel<false, true>;
   else
     kern = y_out ? bat::bat_prologue_kernel<true, false> : bat::bat_prologue_kernel<false, false>;
   DeviceInfo& d = g_dev[dev];
-  const int variant_bit = 1 << ((fp8 ? 4 : (per_row ? 2 : 0)) + (y_out ? 1 : 0));
+  const int variant_bit =
+      1 << ((kv ? 6 + (fp8 ? 2 : 0) : (fp8 ? 4 : (per_row ? 2 : 0))) + (y_out ? 1 : 0));
   if (!(d.pro_attr.load() & variant_bit)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              bat::pro::kSmemBytes) != cudaSuccess)
@@ -317,6 +383,11 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
   void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, bat::GemmParams) =
       a8 ? bat::bat_mxf4_gemm_kernel<true> : bat::bat_mxf4_gemm_kernel<false>;
   const int smem = a8 ? bat::gemm::Cfg<true>::kSmemBytes : bat::gemm::Cfg<false>::kSmemBytes;
+  const int64_t m_tiles = (p.M + bat::gemm::kBM - 1) / bat::gemm::kBM;
+  const int64_t tiles = m_tiles * ((p.N + bat::gemm::kBN - 1) / bat::gemm::kBN);
+  // Split-K over a cluster per tile when one row of tiles leaves most SMs idle (decode
+  // shapes): up to 8 CTAs per tile, at least one K stage each.
+  const int64_t k_stages = (p.K + (a8 ? 127 : 255)) / (a8 ? 128 : 256);
   DeviceInfo& d = g_dev[dev];
   const int variant_bit = a8 ? 2 : 1;
   if (!(d.gemm_attr.load() & variant_bit)) {
@@ -325,9 +396,36 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
     if (ae != cudaSuccess) return cuda_status(ae);
     d.gemm_attr.fetch_or(variant_bit);
   }
-  const int64_t tiles = ((p.M + bat::gemm::kBM - 1) / bat::gemm::kBM) *
-                        ((p.N + bat::gemm::kBN - 1) / bat::gemm::kBN);
-  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  int64_t splits = 1;
+  if (m_tiles == 1 && 2 * tiles <= sms) {
+    splits = sms / tiles;
+    if (splits > 8) splits = 8;
+    if (splits > k_stages) splits = k_stages;
+    // the largest cluster size whose clusters all fit on the GPU at once (one wave)
+    for (; splits > 1; --splits) {
+      std::atomic<int>& mc = d.max_clusters[a8 ? 1 : 0][splits];
+      int n = mc.load();
+      if (n == 0) {
+        cudaLaunchConfig_t oc = {};
+        oc.gridDim = dim3(static_cast<unsigned>(tiles * splits));
+        oc.blockDim = dim3(bat::gemm::kThreads);
+        oc.dynamicSmemBytes = smem;
+        cudaLaunchAttribute ca[1];
+        ca[0].id = cudaLaunchAttributeClusterDimension;
+        ca[0].val.clusterDim.x = static_cast<unsigned>(splits);
+        ca[0].val.clusterDim.y = 1;
+        ca[0].val.clusterDim.z = 1;
+        oc.attrs = ca;
+        oc.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &oc) != cudaSuccess || n < 1) n = -1;
+        mc.store(n);
+      }
+      if (n >= tiles) break;
+    }
+  }
+  p.splits = static_cast<int>(splits);
+  const int grid = splits > 1 ? static_cast<int>(tiles * splits)
+                              : static_cast<int>(tiles < sms ? tiles : sms);
   // Programmatic stream serialization: the kernel's set-up may overlap the previous
   // kernel on the stream; it waits for that kernel's completion (griddepcontrol.wait)
   // before touching the operands or Y, so the stream order of results is unchanged.
@@ -336,11 +434,15 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
   cfg.blockDim = dim3(bat::gemm::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(splits);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = splits > 1 ? 2 : 1;
   return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, p));
 }
 
@@ -578,6 +680,10 @@ static bat_status_t kv_shape_check(int64_t T, int64_t H, int64_t D, int64_t num_
   return BAT_OK;
 }
 
+// (token, head) rows from which bat_kv_quantize runs the tensor-core prologue
+// instead of the CUDA-core kernel
+constexpr int64_t kKvTensorRows = 4096;
+
 static unsigned kv_grid(int64_t items, int sms) {
   const int64_t want = (items + bat::kv::kWarps - 1) / bat::kv::kWarps;
   const int64_t cap = static_cast<int64_t>(sms) * 8;
@@ -600,33 +706,22 @@ bat_status_t bat_kv_quantize(const void* kv, int64_t T, int64_t H, int64_t D, co
   int dev = 0, sms = 0;
   st = current_device(&dev, &sms);
   if (st != BAT_OK) return st;
-  bat::KvParams p;
-  p.kv = static_cast<const uint16_t*>(kv);
-  p.a = A;
-  p.b = B;
-  p.g_lo = g_lo;
-  p.g_hi = g_hi;
-  p.slots = slots;
-  p.codes = static_cast<uint8_t*>(cache_codes);
-  p.scales = static_cast<uint8_t*>(cache_scales);
-  p.y_out = y_out;
-  p.T = T;
-  p.H = H;
-  p.S = num_slots;
-  p.D = static_cast<int>(D);
-  p.nbh = static_cast<int>(D / 32);
-  p.groups = (p.nbh + 3) / 4;
-  p.ls = ls;
-  const unsigned grid = kv_grid(T * H * p.groups, sms);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool fp8 = fmt == BAT_KV_MXFP8;
-  if (fp8)
-    (y_out ? bat::bat_kv_quantize_kernel<true, true> : bat::bat_kv_quantize_kernel<true, false>)
-        <<<grid, bat::kv::kThreads, 0, s>>>(p);
-  else
-    (y_out ? bat::bat_kv_quantize_kernel<false, true> : bat::bat_kv_quantize_kernel<false, false>)
-        <<<grid, bat::kv::kThreads, 0, s>>>(p);
-  return cuda_status(cudaGetLastError());
+  if (T * H >= kKvTensorRows) {
+    // a prefill-sized batch: the tensor-core prologue over the (token, head) rows
+    if (T * H >= (int64_t{1} << 31)) return BAT_ERR_SHAPE;
+    bat_mxfp4_t out;
+    out.codes = cache_codes;
+    out.scales = cache_scales;
+    out.rows = T * H;
+    out.k = D;
+    return launch_prologue(kv, T * H, D, A, B, g_lo, g_hi, false, &out, y_out, s, ls, fp8, slots,
+                           H, num_slots);
+  }
+  return launch_rows(kv, T * H, H, num_slots, slots, D, A, B, g_lo, g_hi, ls, fp8,
+                     static_cast<uint8_t*>(cache_codes), static_cast<uint8_t*>(cache_scales), y_out,
+                     sms, s);
 }
 
 bat_status_t bat_kv_dequantize(const void* cache_codes, const void* cache_scales,

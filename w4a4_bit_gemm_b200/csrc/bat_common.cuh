@@ -29,6 +29,10 @@ __device__ __forceinline__ float clip_ratio(float g) {
   return static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(g))));
 }
 
+__device__ __forceinline__ int64_t scale_offset(int64_t m, int64_t b, int nbp4) {
+  return ((m >> 7) * nbp4 + (b >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (b & 3);
+}
+
 // ---------------------------------------------------------------- small helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -13,18 +13,32 @@
 //               Writing them from registers keeps the copies off the tensor
 //               pipe, where tcgen05.cp would queue behind the MMAs;
 //   warp 8      TMA producer: code tiles through 2-D tensor maps (128-byte
-//               swizzle), scale tiles through 1-D bulk copies, into a ring of
-//               kStages shared-memory stages guarded by mbarriers;
+//               swizzle) into a ring of kStages shared-memory stages guarded by
+//               mbarriers;
 //   warp 9      TMEM owner and MMA issuer: tcgen05.mma kind::mxf4.block_scale
 //               (M=128, N=256, K=64) accumulating in TMEM;
 //               with MXFP8 activations (W4A8, kA8), kind::mxf8f6f4.block_scale
 //               (E4M3 x E2M1, K=32), the weights' packed E2M1 codes unpacked by
 //               the TMA load into the 16-bytes-per-16-elements layout that MMA reads;
-//   warps 10,11 idle (they complete the third warpgroup).
+//   warp 10     scale producer: the stage's scale tiles as 1-D bulk copies (the code
+//               tiles' producer and this warp split a stage's copy instructions);
+//   warp 11     idle (it completes the third warpgroup).
 // Every wait is bounded (see mbar_wait) and reports through the error word.
 // Launched with programmatic stream serialization, so barrier set-up and the TMEM
 // allocation overlap the end of the kernel before it (normally the quantizer).
+//
+// Split-K for a single row of tiles (M <= 128, few N tiles: the decode shapes).
+// With splits = C > 1 the grid is launched in clusters of C CTAs, one cluster per
+// tile; CTA r of a cluster takes K stages [r*ks/C, (r+1)*ks/C) and leaves its fp32
+// partial tile (valid rows only) in its own shared memory (the drained stage
+// buffers). After a cluster barrier each CTA sums, in rank order, one share of the
+// tile's 32-column chunks over the C partials it reads through distributed shared
+// memory, and writes that share of Y. The sum order is fixed, so the result does
+// not depend on timing; a second cluster barrier keeps every partial alive until all
+// readers are done.
 #pragma once
+
+#include <cooperative_groups.h>
 
 #include "bat_common.cuh"
 
@@ -40,6 +54,9 @@ constexpr int kChunk = 512;                  // one 128-row x 4-scale block of t
 constexpr int kThreads = 384;
 constexpr uint32_t kRegsEpi = 248;   // after setmaxnreg: 128 x 248 + 256 x 56 <= 384 x 168
 constexpr uint32_t kRegsOther = 56;
+// split-K partial tile in shared memory: fp32 rows of 256 columns, padded to 260 floats
+// so that the epilogue's row-per-lane stores spread over the banks
+constexpr int kPartStride = kBN + 4;
 // bf16 output staging for the TMA store: one box of 128 rows x 64 columns (128 bytes,
 // 128-byte swizzle); the epilogue holds its whole bf16 tile in registers and
 // streams it through this box one 64-column slice at a time.
@@ -74,6 +91,7 @@ struct GemmParams {
   int out_f32;         // 1: fp32 output, 0: bf16
   int vec_ok;          // rows of Y are 16-byte aligned for vector stores
   int tma_store;       // bf16 output written through the staged TMA store
+  int splits;          // K splits = cluster size (1: persistent, whole K per tile)
 };
 
 __device__ __forceinline__ uint4 lds_v4_u32(uint32_t addr) {
@@ -161,6 +179,65 @@ __device__ __forceinline__ void store_chunk(const GemmParams& p, int64_t row, in
 // kA8 = false: Xq MXFP4 (tmap_a over packed codes [M][K/2] bytes).
 // kA8 = true:  Xq MXFP8 E4M3 (tmap_a over codes [M][K] bytes) and tmap_b over Wq's packed
 //              E2M1 codes with the 16-elements-per-16-bytes shared-memory expansion.
+// Sum of the cluster's partial tiles for this CTA's share of the 32-column chunks
+// (chunks rank, rank + C, ...), rows of the tile that exist; partials are added in
+// rank order 0 .. C-1.
+__device__ __forceinline__ void split_reduce(const GemmParams& p, uint8_t* base_ptr,
+                                             cooperative_groups::cluster_group& cluster,
+                                             int64_t mt, int64_t nt, int rank) {
+  using namespace gemm;
+  const int C = p.splits;
+  const int64_t rows = min(static_cast<int64_t>(kBM), p.M - mt * kBM);
+  const int nch = (kBN / 32 - rank + C - 1) / C;  // chunks of this rank
+  const int64_t work = rows * nch * 8;             // float4 items
+  const float* part = reinterpret_cast<const float*>(base_ptr);
+  for (int64_t i = threadIdx.x; i < work; i += blockDim.x) {
+    const int64_t row = i / (nch * 8);
+    const int j = static_cast<int>(i % (nch * 8));
+    const int col = (rank + (j >> 3) * C) * 32 + (j & 7) * 4;  // column within the tile
+    const int64_t off = row * kPartStride + col;
+    // all C remote loads first (independent, so their latencies overlap), then the sum
+    float4 v[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (q < C) v[q] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(part + off, q));
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (q < C) {
+        acc.x += v[q].x;
+        acc.y += v[q].y;
+        acc.z += v[q].z;
+        acc.w += v[q].w;
+      }
+    const int64_t m = mt * kBM + row;
+    const int64_t n0 = nt * kBN + col;
+    const float a[4] = {acc.x, acc.y, acc.z, acc.w};
+    if (p.out_f32) {
+      float* dst = static_cast<float*>(p.y) + m * p.N + n0;
+      if (p.vec_ok && n0 + 4 <= p.N) {
+        *reinterpret_cast<float4*>(dst) = acc;
+      } else {
+        for (int c = 0; c < 4; ++c)
+          if (n0 + c < p.N) dst[c] = a[c];
+      }
+    } else {
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.y) + m * p.N + n0;
+      __nv_bfloat162 lo = __floats2bfloat162_rn(a[0], a[1]);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(a[2], a[3]);
+      if (p.vec_ok && n0 + 4 <= p.N) {
+        uint2 w;
+        w.x = *reinterpret_cast<uint32_t*>(&lo);
+        w.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(dst) = w;
+      } else {
+        for (int c = 0; c < 4; ++c)
+          if (n0 + c < p.N) dst[c] = __float2bfloat16_rn(a[c]);
+      }
+    }
+  }
+}
+
 template <bool kA8>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
     bat_mxf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
@@ -219,6 +296,14 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   const int64_t n_tiles = (p.N + kBN - 1) / kBN;
   const int64_t tiles = m_tiles * n_tiles;
   const int k_stages = static_cast<int>((p.K + kBK - 1) / kBK);
+  // the tiles this CTA visits and its K stages [kb, ke): with split-K one tile per
+  // cluster and a slice of K per cluster rank; otherwise a persistent walk over tiles
+  const bool split = p.splits > 1;
+  const int rank = split ? static_cast<int>(blockIdx.x % p.splits) : 0;
+  const int64_t tile0 = split ? blockIdx.x / p.splits : blockIdx.x;
+  const int64_t tstride = split ? tiles : gridDim.x;
+  const int kb = split ? rank * k_stages / p.splits : 0;
+  const int ke = split ? (rank + 1) * k_stages / p.splits : k_stages;
   const int64_t sf_groups_b = (p.N + 127) / 128;
   bool ok = true;
 
@@ -230,11 +315,11 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+      for (int64_t tile = tile0; tile < tiles && ok; tile += tstride) {
         const int64_t mt = tile % m_tiles;
         const int64_t nt = tile / m_tiles;
         const int ngb = (nt * 2 + 1 < sf_groups_b) ? 2 : 1;  // 128-row scale groups of this W tile
-        for (int ks = 0; ks < k_stages; ++ks) {
+        for (int ks = kb; ks < ke; ++ks) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, kErrWaitEmpty)) { ok = false; break; }
           const int c0 = ks * kChunksPerStage;
           const int nch = min(kChunksPerStage, p.nbp4 - c0);
@@ -243,12 +328,34 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
           constexpr uint32_t kBTx = kA8 ? kBBytes / 2 : kBBytes;
           const uint32_t bytes = kABytes + kBTx + static_cast<uint32_t>(nch) * kChunk * (1 + ngb);
           const uint32_t sa = base + stage * kStageBytes;
+          // the expected bytes include the scale copies warp 10 issues (their completions may
+          // come first: the phase still waits for this arrival)
           mbar_expect_tx(full_bar(stage), bytes);
           // x of both maps is 128 per stage: bytes of packed E2M1, E4M3 elements, or
           // (unpacking load) E2M1 elements
           tma_load_2d(sa, &tmap_a, full_bar(stage), ks * 128, static_cast<int32_t>(mt * kBM));
           tma_load_2d(sa + kABytes, &tmap_b, full_bar(stage), ks * 128,
                       static_cast<int32_t>(nt * kBN));
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ scale producer
+    // Each copy instruction costs the issuing thread some 60-120 cycles; the scale copies
+    // go out from this warp so that one stage's copies are issued in about half the time.
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int64_t tile = tile0; tile < tiles && ok; tile += tstride) {
+        const int64_t mt = tile % m_tiles;
+        const int64_t nt = tile / m_tiles;
+        const int ngb = (nt * 2 + 1 < sf_groups_b) ? 2 : 1;
+        for (int ks = kb; ks < ke; ++ks) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, kErrWaitEmpty)) { ok = false; break; }
+          const int c0 = ks * kChunksPerStage;
+          const int nch = min(kChunksPerStage, p.nbp4 - c0);
+          const uint32_t sa = base + stage * kStageBytes;
           bulk_load(sa + kABytes + kBBytes, p.sfa + (mt * p.nbp4 + c0) * kChunk, nch * kChunk,
                     full_bar(stage));
           for (int g = 0; g < ngb; ++g)
@@ -271,10 +378,10 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t acc_phase = 0;
-      for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+      for (int64_t tile = tile0; tile < tiles && ok; tile += tstride) {
         if (!mbar_wait(tmem_empty, acc_phase ^ 1u, kErrWaitTmemEmpty)) { ok = false; break; }
         tc_fence_after();
-        for (int ks = 0; ks < k_stages; ++ks) {
+        for (int ks = kb; ks < ke; ++ks) {
           if (!mbar_wait(full_bar(stage), phase, kErrWaitFull) ||
               !mbar_wait(sf_bar(stage), phase, kErrWaitFull)) { ok = false; break; }
           tc_fence_after();
@@ -282,7 +389,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
           const uint32_t t_sfa = tmem_base + kSfCol0 + kSfStageCols * stage;
           const uint32_t t_sfb = t_sfa + 8;
           const int64_t krem = p.K - static_cast<int64_t>(ks) * kBK;
-          const uint32_t acc0 = (ks != 0) ? 1u : 0u;
+          const uint32_t acc0 = (ks != kb) ? 1u : 0u;
           if constexpr (kA8) {
             // four K=32 MMAs, 32 bytes of each operand apiece; scale byte c of each word
             // (K % 128 == 0, so every stage is full)
@@ -326,8 +433,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     const uint32_t tlane = static_cast<uint32_t>(32 * q) << 16;
     int stage = 0;
     uint32_t phase = 0;
-    for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-      for (int ks = 0; ks < k_stages; ++ks) {
+    for (int64_t tile = tile0; tile < tiles && ok; tile += tstride) {
+      for (int ks = kb; ks < ke; ++ks) {
         if (!mbar_wait(full_bar(stage), phase, kErrWaitFull)) { ok = false; break; }
         const uint32_t ssf = base + stage * kStageBytes + kABytes + kBBytes + lane * 16;
         uint32_t fa[8] = {}, fb[16] = {};
@@ -368,7 +475,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     const int rl = 32 * q + lane;  // row within the tile
     const bool leader = (warp == 0 && lane == 0);
     uint32_t acc_phase = 0;
-    for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+    for (int64_t tile = tile0; tile < tiles && ok; tile += tstride) {
       const int64_t mt = tile % m_tiles;
       const int64_t nt = tile / m_tiles;
       bool got = mbar_wait(tmem_full, acc_phase, kErrWaitTmemFull);
@@ -376,7 +483,26 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
       if (!got) { ok = false; break; }
       tc_fence_after();
       const uint32_t trow = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
-      if (p.tma_store) {
+      if (split) {
+        // partial tile -> this CTA's shared memory (rows of the tile that exist); every
+        // stage has been consumed by the MMAs that tmem_full waited for
+        const bool row_ok = mt * kBM + rl < p.M;
+        const uint32_t prow = base + static_cast<uint32_t>(rl * kPartStride * 4);
+#pragma unroll 1
+        for (int cc = 0; cc < kBN / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(trow + cc * 32, r);
+          tmem_wait_ld();
+          if (row_ok) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              st_shared_v4(prow + (cc * 32 + 4 * j) * 4, r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tmem_empty);
+      } else if (p.tma_store) {
         // 1) drain the accumulator into registers as bf16 pairs and release TMEM at once
         uint32_t h[kBN / 2];
 #pragma unroll
@@ -432,6 +558,14 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (split) {
+    // every CTA of the cluster reaches both barriers, error or not
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();  // all partials written
+    split_reduce(p, base_ptr, cluster, tile0 % m_tiles, tile0 / m_tiles, rank);
+    cluster.sync();  // all partials read
+  }
   if (warp == 9) tmem_dealloc(tmem_base, kTmemCols);
 }
 

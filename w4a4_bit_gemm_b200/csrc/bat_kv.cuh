@@ -1,21 +1,17 @@
-// KV-cache path of the BATQuant transformer integration (BATQuant note,
-// en.papernotes.org, Method > Key Designs 4 "Equivalent Transformer integration":
-// one transform set on the per-head key cache path and one on the value path;
-// the KV8 / KV4 settings of Loss & Training store the cache in MXFP8 (E4M3) /
-// MXFP4).
+// Row quantizer on the CUDA cores and the KV-cache path of the BATQuant transformer
+// integration (BATQuant note, en.papernotes.org, Method > Key Designs 4 "Equivalent
+// Transformer integration": one transform set on the per-head key cache path and one
+// on the value path; the KV8 / KV4 settings of Loss & Training store the cache in
+// MXFP8 (E4M3) / MXFP4).
 //
-// Every head's D-vector (D = head_dim, a multiple of 32) goes through the block
-// transform y_b = x_b (B_b (x) A) with the same factors for all heads (A s x s
-// shared, B_b (32/s) x (32/s) for each 32-channel block of the head), the
-// block clip with per-block logits shared by heads and tokens, and MX
-// quantization; the codes and the scale byte go to the token's cache slot.
-//
-// The work per element is small (one 32 x 32 block product) and the step is
-// usually a decode step of a few tokens, so this is a CUDA-core kernel sized for
-// latency: a warp takes one (token, head, group of four blocks); lane l holds
-// elements 4(l%8) .. 4(l%8)+3 of block l/8; the block's 32 inputs are exchanged
-// with shuffles and multiplied by the fp32 block P_b, which each CTA builds once
-// in shared memory. Block min/max come from an 8-lane butterfly.
+// bat_rows_quantize_kernel handles batches with few rows: decode-sized activations
+// (its output is the tiled MXFP4 / MXFP8 layout the GEMM reads) and KV-cache stores,
+// where every head's D-vector (D = head_dim, a multiple of 32) goes through the block
+// transform y_b = x_b (B_b (x) A) with the same factors for all heads (A s x s shared,
+// B_b (32/s) x (32/s) for each 32-channel block of the head), the block clip with
+// per-block logits shared by heads and tokens, and MX quantization; the codes and
+// the scale byte go to the token's cache slot. Larger batches go to the tensor-core
+// prologue. bat_kv_dequantize_kernel reads cache rows back.
 #pragma once
 
 #include "bat_common.cuh"
@@ -29,19 +25,6 @@ constexpr int kMaxBlocks = 8;     // D <= 256: P blocks staged in shared memory 
 constexpr int kFacFloats = 2112;  // A and B staged for the build when they fit (s >= 2)
 }  // namespace kv
 
-struct KvParams {
-  const uint16_t* kv;     // bf16 [T][H][D]
-  const float* a;         // [s][s]
-  const float* b;         // [D/32][t][t]
-  const float* g_lo;      // [D/32] clip logits, or null (no clip)
-  const float* g_hi;
-  const int64_t* slots;   // [T]: cache row of token t, -1 to skip
-  uint8_t* codes;         // cache codes [S][H][D] (E4M3) or [S][H][D/2] (E2M1)
-  uint8_t* scales;        // cache scales [S][H][D/32]
-  float* y_out;           // optional fp32 [T][H][D] trace of the transformed values
-  int64_t T, H, S;
-  int D, nbh, groups, ls; // nbh = D/32, groups = ceil(nbh/4), ls = log2 s
-};
 
 struct KvReadParams {
   const uint8_t* codes;   // cache codes
@@ -101,75 +84,162 @@ __device__ __forceinline__ void kv_block_product(const float* pblk, const float 
   }
 }
 
-template <bool kFp8, bool kTrace>
-__global__ void __launch_bounds__(kv::kThreads)
-    bat_kv_quantize_kernel(const KvParams p) {
-  __shared__ __align__(16) float sp[kv::kMaxBlocks * 1024];
-  __shared__ __align__(16) float fac[kv::kFacFloats];
-  __shared__ float ratio[2 * kv::kMaxBlocks];
-  if (threadIdx.x < 2 * p.nbh) {  // clip ratios of the head's blocks: lo, then hi
-    const float* g = threadIdx.x < p.nbh ? p.g_lo : p.g_hi;
-    ratio[threadIdx.x] = g ? clip_ratio(g[threadIdx.x % p.nbh]) : 1.0f;
-  }
-  kv_build_p(sp, fac, p.a, p.b, p.nbh, p.ls);
+// ---------------------------------------------------------------- row quantizer
+// Small batches of rows (decode-sized activations, and KV-cache stores) on the CUDA
+// cores: the tensor-core prologue's fixed costs (TMEM, barriers, the P_b build of a
+// whole strip) dominate when there are few rows. Warp w always takes the same group
+// g = w % groups of four 32-channel blocks, so lane l always works on block
+// 4g + l/8 and keeps its four columns 4(l%8) .. 4(l%8)+3 of that block's P_b
+// (32 x 4 fp32, the product B_b[k/s][n/s] * A[k%s][n%s] rounded once) and its clip
+// ratios in registers; rows r0, r0 + R, ... of that group follow. Each row reads the
+// block's 32 inputs directly (the block's eight lanes load the same 64 bytes) and
+// sums x[k] * P_b[k][n] in fp32, k ascending.
+struct RowQuantParams {
+  const uint16_t* x;      // bf16 [rows][D]
+  const float* a;         // [s][s]
+  const float* b;         // [D/32][t][t]: one factor per 32-channel block of a row
+  const float* g_lo;      // [D/32] clip logits, or null (no clip)
+  const float* g_hi;
+  uint8_t* codes;
+  uint8_t* scales;
+  float* y_out;           // optional fp32 [rows][D] trace of the transformed values
+  const int64_t* slots;   // KV mode: cache slot of token row / H (-1 skips); else null
+  int64_t rows;           // KV: tokens x heads; linear: M
+  int64_t H;              // KV: heads per token (linear: 1)
+  int64_t S;              // KV: cache slots
+  int D, nb, groups, ls;  // D = channels per row, nb = D/32, groups = ceil(nb/4), log2 s
+  int R;                  // warps per group: row stride
+  int nbp4;               // linear mode: ceil(nb/4) of the tiled scale layout
+};
+
+template <int kLs>  // kLs >= 0: the split as a constant; -1: read it from `ls`
+__device__ __forceinline__ void rows_build_pc(float (&pc)[32][4], const float* __restrict__ a,
+                                              const float* __restrict__ b, int bq, int u, int ls_rt) {
+  const int ls = kLs >= 0 ? kLs : ls_rt;
+  const int sm = (1 << ls) - 1, tt = 32 >> ls;
+  const float* bb = b + static_cast<int64_t>(bq) * tt * tt;
+#pragma unroll
+  for (int k = 0; k < 32; ++k)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = 4 * u + j;
+      pc[k][j] = __fmul_rn(__ldg(bb + (k >> ls) * tt + (n >> ls)), __ldg(a + ((k & sm) << ls) + (n & sm)));
+    }
+}
+
+// kKv: rows are (token, head) pairs stored into cache slots (codes [slot][H][D] or
+// [slot][H][D/2], scales plain [slot][H][D/32]); otherwise rows of an activation
+// matrix (codes [M][D] or [M][D/2], scales in the GEMM's tiled layout, padding 0).
+template <bool kFp8, bool kTrace, bool kKv>
+__global__ void __launch_bounds__(kv::kThreads, 1)
+    bat_rows_quantize_kernel(const RowQuantParams p) {
+  // a following kernel launched with programmatic serialization (the GEMM) may start
+  // its set-up now; this kernel's inputs come from the kernels before it
+  allow_dependents();
+  grid_dependency_wait();
   const int lane = threadIdx.x & 31;
   const int u = lane & 7;
-  const int64_t items = p.T * p.H * p.groups;
-  const int64_t wstride = static_cast<int64_t>(gridDim.x) * kv::kWarps;
-  for (int64_t it = static_cast<int64_t>(blockIdx.x) * kv::kWarps + (threadIdx.x >> 5); it < items;
-       it += wstride) {
-    const int g = static_cast<int>(it % p.groups);
-    const int64_t th = it / p.groups;  // token * H + head
-    const int64_t t = th / p.H;
+  const int64_t wid = static_cast<int64_t>(blockIdx.x) * kv::kWarps + (threadIdx.x >> 5);
+  if (wid < static_cast<int64_t>(p.groups) * p.R) {
+    const int g = static_cast<int>(wid % p.groups);
     const int blk = 4 * g + (lane >> 3);
-    const bool has = blk < p.nbh;  // lanes of a missing fourth block idle (shuffles stay full)
-    const int64_t slot = p.slots[t];
-    if (slot >= p.S) {
-      if (lane == 0) atomicOr(&g_dev_error, kErrBadIndex);
-      continue;
-    }
-    float x[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    const int64_t e0 = th * p.D + blk * kG + 4 * u;
-    if (has) {
-      const uint2 w = *reinterpret_cast<const uint2*>(p.kv + e0);
-      x[0] = bf16lo(w.x);
-      x[1] = bf16hi(w.x);
-      x[2] = bf16lo(w.y);
-      x[3] = bf16hi(w.y);
-    }
-    float y[4];
-    kv_block_product(sp + (has ? blk : 0) * 1024, x, lane, y);
-    if (kTrace && has)
-      *reinterpret_cast<float4*>(p.y_out + e0) = make_float4(y[0], y[1], y[2], y[3]);
-    // block min / max over the block's 8 lanes
-    float mn = fminf(fminf(y[0], y[1]), fminf(y[2], y[3]));
-    float mx = fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
+    const bool has = blk < p.nb;  // lanes of a missing fourth block idle (shuffles stay full)
+    const int bq = has ? blk : 0;
+    const float r_lo = (has && p.g_lo) ? clip_ratio(p.g_lo[bq]) : 1.0f;
+    const float r_hi = (has && p.g_hi) ? clip_ratio(p.g_hi[bq]) : 1.0f;
+    float pc[32][4];
+    if (p.ls == 3)
+      rows_build_pc<3>(pc, p.a, p.b, bq, u, 3);
+    else
+      rows_build_pc<-1>(pc, p.a, p.b, bq, u, p.ls);
+    for (int64_t row = wid / p.groups; row < p.rows; row += p.R) {
+      int64_t slot = row;
+      if (kKv) {
+        slot = p.slots[row / p.H];
+        if (slot >= p.S) {
+          if (lane == 0) atomicOr(&g_dev_error, kErrBadIndex);
+          continue;
+        }
+      }
+      float x[32];
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(p.x + row * p.D + bq * kG);
 #pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    }
-    if (!has || slot < 0) continue;
-    const float r_lo = ratio[blk];
-    const float r_hi = ratio[p.nbh + blk];
-    const float lo = __fmul_rn(r_lo, mn);
-    const float hi = __fmul_rn(r_hi, mx);
-    const float amax = fmaxf(fabsf(fminf(fmaxf(mn, lo), hi)), fabsf(fminf(fmaxf(mx, lo), hi)));
-    constexpr int kEmax = kFp8 ? 8 : 2;
-    const int efield = static_cast<int>(__float_as_uint(amax) >> 23);
-    const int sbyte = efield > kEmax ? efield - kEmax : 0;  // e + 127
-    const float inv_scale = __uint_as_float(static_cast<uint32_t>(254 - sbyte) << 23);  // 2^-e
-    float v[4];
+        for (int c = 0; c < 4; ++c) {
+          const uint4 w = src[c];
+          x[8 * c + 0] = bf16lo(w.x); x[8 * c + 1] = bf16hi(w.x);
+          x[8 * c + 2] = bf16lo(w.y); x[8 * c + 3] = bf16hi(w.y);
+          x[8 * c + 4] = bf16lo(w.z); x[8 * c + 5] = bf16hi(w.z);
+          x[8 * c + 6] = bf16lo(w.w); x[8 * c + 7] = bf16hi(w.w);
+        }
+      }
+      uint64_t y01 = 0ull, y23 = 0ull;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = __fmaf_rn(fminf(fmaxf(y[i], lo), hi), inv_scale, 0.0f);
-    const int64_t crow = (slot * p.H + th % p.H) * p.D + blk * kG + 4 * u;  // element index
-    if (kFp8) {
-      *reinterpret_cast<uint32_t*>(p.codes + crow) = e4m3x4(v[0], v[1], v[2], v[3]);
-    } else {
-      const uint32_t c = e2m1x2(v[0], v[1]) | (e2m1x2(v[2], v[3]) << 8);
-      *reinterpret_cast<uint16_t*>(p.codes + crow / 2) = static_cast<uint16_t>(c);
+      for (int k = 0; k < 32; ++k) {
+        const uint64_t xx = pack2(x[k], x[k]);
+        y01 = ffma2(xx, pack2(pc[k][0], pc[k][1]), y01);
+        y23 = ffma2(xx, pack2(pc[k][2], pc[k][3]), y23);
+      }
+      float y[4];
+      unpack2(y01, y[0], y[1]);
+      unpack2(y23, y[2], y[3]);
+      const int64_t e0 = row * p.D + blk * kG + 4 * u;
+      if (kTrace && has)
+        *reinterpret_cast<float4*>(p.y_out + e0) = make_float4(y[0], y[1], y[2], y[3]);
+      // block min / max over the block's 8 lanes
+      float mn = fminf(fminf(y[0], y[1]), fminf(y[2], y[3]));
+      float mx = fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      if (!has || slot < 0) continue;
+      const float lo = __fmul_rn(r_lo, mn);
+      const float hi = __fmul_rn(r_hi, mx);
+      const float amax = fmaxf(fabsf(fminf(fmaxf(mn, lo), hi)), fabsf(fminf(fmaxf(mx, lo), hi)));
+      constexpr int kEmax = kFp8 ? 8 : 2;
+      const int efield = static_cast<int>(__float_as_uint(amax) >> 23);
+      const int sbyte = efield > kEmax ? efield - kEmax : 0;  // e + 127
+      const float inv_scale = __uint_as_float(static_cast<uint32_t>(254 - sbyte) << 23);  // 2^-e
+      float v[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = __fmaf_rn(fminf(fmaxf(y[i], lo), hi), inv_scale, 0.0f);
+      // element index of the code: cache row (slot, head) or the activation row
+      const int64_t crow = kKv ? slot * p.H + row % p.H : row;
+      const int64_t ci = crow * p.D + blk * kG + 4 * u;
+      if (kFp8) {
+        *reinterpret_cast<uint32_t*>(p.codes + ci) = e4m3x4(v[0], v[1], v[2], v[3]);
+      } else {
+        const uint32_t c = e2m1x2(v[0], v[1]) | (e2m1x2(v[2], v[3]) << 8);
+        *reinterpret_cast<uint16_t*>(p.codes + ci / 2) = static_cast<uint16_t>(c);
+      }
+      if (u == 0) {
+        if (kKv)
+          p.scales[crow * p.nb + blk] = static_cast<uint8_t>(sbyte);
+        else
+          p.scales[scale_offset(row, blk, p.nbp4)] = static_cast<uint8_t>(sbyte);
+      }
     }
-    if (u == 0) p.scales[(slot * p.H + th % p.H) * p.nbh + blk] = static_cast<uint8_t>(sbyte);
+  }
+  if (!kKv) {
+    // padding of the tiled scale layout: rows [M, 128-row boundary) and blocks
+    // [nb, 4 nbp4) of the real rows are 0 (the GEMM multiplies by 2^(byte-127))
+    const int64_t mpad = (p.rows + 127) / 128 * 128;
+    const int64_t tail = 4 * p.nbp4 - p.nb;  // 0..3 padding blocks per real row
+    const int64_t n_rows_pad = (mpad - p.rows) * p.nbp4;
+    const int64_t total = n_rows_pad + p.rows * tail;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+      if (i < n_rows_pad) {
+        const int64_t m = p.rows + i / p.nbp4;
+        const int64_t c = i % p.nbp4;
+        *reinterpret_cast<uint32_t*>(p.scales + scale_offset(m, 4 * c, p.nbp4)) = 0u;
+      } else {
+        const int64_t j = i - n_rows_pad;
+        p.scales[scale_offset(j / tail, p.nb + j % tail, p.nbp4)] = 0;
+      }
+    }
   }
 }
 

@@ -86,12 +86,14 @@ struct PrologueParams {
   int strips;            // ceil(nbp2 / kStrip)
   int cps;               // CTAs per strip (grid = strips * cps)
   int ls;                // log2 of the shared factor's size: 0..5 (3 is the 8 x 8 / 4 x 4 split)
+  // KV-cache store (kKv): row m = token (m / kv_heads), head (m % kv_heads); its codes go
+  // to cache row slots[token] * kv_heads + head, scales plain [cache row][nb]
+  const int64_t* slots;
+  int64_t kv_heads;
+  int64_t kv_slots;
 };
 
 
-__device__ __forceinline__ int64_t scale_offset(int64_t m, int64_t b, int nbp4) {
-  return ((m >> 7) * nbp4 + (b >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (b & 3);
-}
 
 __device__ __forceinline__ float min3f(float a, float b, float c) {
   float d;
@@ -233,7 +235,8 @@ __device__ __forceinline__ uint32_t quantize_block(const float (&y)[32], float r
 // tmap_x: bf16 X [rows][K], box 64 columns x 128 rows, 128-byte swizzle, zero fill.
 // kPerRowClip: clip logits indexed [row][block] (weight side) instead of [block].
 // kFp8: MXFP8 (E4M3) codes, one byte per element, instead of packed MXFP4.
-template <bool kTrace, bool kPerRowClip, bool kFp8 = false>
+// kKv: rows are (token, head) pairs of a K or V batch, stored into cache slots.
+template <bool kTrace, bool kPerRowClip, bool kFp8 = false, bool kKv = false>
 __global__ void __launch_bounds__(pro::kThreads, 1)
     bat_prologue_kernel(const __grid_constant__ CUtensorMap tmap_x, const PrologueParams p) {
   using namespace pro;
@@ -467,28 +470,55 @@ __global__ void __launch_bounds__(pro::kThreads, 1)
         }
         uint32_t packed[kFp8 ? 8 : 4];
         const uint32_t sbyte = quantize_block<kFp8>(y, r_lo, r_hi, packed);
-        if (valid) {
-          if constexpr (kFp8) {
-            uint4* dst = reinterpret_cast<uint4*>(p.codes + m * p.K + b * kG);
-            dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-            dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-          } else {
-            *reinterpret_cast<uint4*>(p.codes + m * (p.K / 2) + b * (kG / 2)) =
-                make_uint4(packed[0], packed[1], packed[2], packed[3]);
-          }
-          if (kTrace) {
-            float4* dst = reinterpret_cast<float4*>(p.y_out + m * p.K + b * kG);
+        if constexpr (kKv) {
+          if (valid) {
+            const int64_t tok = m / p.kv_heads;
+            const int64_t slot = p.slots[tok];
+            if (slot >= p.kv_slots) {
+              atomicOr(&g_dev_error, kErrBadIndex);
+            } else if (slot >= 0) {
+              const int64_t crow = slot * p.kv_heads + (m - tok * p.kv_heads);
+              if constexpr (kFp8) {
+                uint4* dst = reinterpret_cast<uint4*>(p.codes + crow * p.K + b * kG);
+                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+              } else {
+                *reinterpret_cast<uint4*>(p.codes + crow * (p.K / 2) + b * (kG / 2)) =
+                    make_uint4(packed[0], packed[1], packed[2], packed[3]);
+              }
+              p.scales[crow * p.nb + b] = static_cast<uint8_t>(sbyte);
+            }
+            if (kTrace) {
+              float4* dst = reinterpret_cast<float4*>(p.y_out + m * p.K + b * kG);
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              dst[c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
+              for (int c = 0; c < 8; ++c)
+                dst[c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
+            }
           }
+        } else {
+          if (valid) {
+            if constexpr (kFp8) {
+              uint4* dst = reinterpret_cast<uint4*>(p.codes + m * p.K + b * kG);
+              dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+              dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+            } else {
+              *reinterpret_cast<uint4*>(p.codes + m * (p.K / 2) + b * (kG / 2)) =
+                  make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            }
+            if (kTrace) {
+              float4* dst = reinterpret_cast<float4*>(p.y_out + m * p.K + b * kG);
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                dst[c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
+            }
+          }
+          // rows past M and blocks past nb are padding of the tiled scale buffer: 0;
+          // the last pair also covers the padding blocks [2*nbp2, 4*nbp4)
+          uint8_t* sp = p.scales + scale_offset(m, b, p.nbp4);
+          *sp = static_cast<uint8_t>(valid ? sbyte : 0u);
+          if ((b & 3) < 2 && b + 2 >= 2 * static_cast<int64_t>(p.nbp2) && b + 2 < 4 * static_cast<int64_t>(p.nbp4))
+            sp[2] = 0;
         }
-        // rows past M and blocks past nb are padding of the tiled scale buffer: 0;
-        // the last pair also covers the padding blocks [2*nbp2, 4*nbp4)
-        uint8_t* sp = p.scales + scale_offset(m, b, p.nbp4);
-        *sp = static_cast<uint8_t>(valid ? sbyte : 0u);
-        if ((b & 3) < 2 && b + 2 >= 2 * static_cast<int64_t>(p.nbp2) && b + 2 < 4 * static_cast<int64_t>(p.nbp4))
-          sp[2] = 0;
         // next unit of this set
         pr += kSets;
         while (pr >= npair) { pr -= npair; ++mt; }
