@@ -327,7 +327,10 @@ def _gemm_check(bat, Xq, Wq, M, N, K, rows=None, cols=None):
                                    (300, 1000, 2048),
                                    # one row of tiles: split-K over a cluster per tile
                                    (1, 256, 2048), (100, 520, 1024), (128, 1000, 768),
-                                   (33, 300, 2080), (16, 6144, 4096)])
+                                   (33, 300, 2080), (16, 6144, 4096),
+                                   # CTA pairs: 256 x 256 tiles, ragged rows, columns and K
+                                   (512, 768, 2048), (384, 256, 1056), (129, 136, 32),
+                                   (1000, 1288, 4128)])
 def test_gemm_shapes(bat, M, N, K):
     X = wl.random_bf16((M, K), seed=M + 3 * K, scale=2.0)
     W = wl.random_bf16((N, K), seed=N + 5 * K, scale=0.02)
