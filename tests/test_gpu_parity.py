@@ -687,3 +687,28 @@ def test_split_k_is_deterministic(bat):
     torch.cuda.synchronize()
     assert all(torch.equal(ys[0], y) for y in ys[1:])
     assert bat.bat_device_error() == 0
+
+
+@pytest.mark.parametrize("M,N,K,clip", [(16, 6144, 4096, True), (1, 256, 2048, True),
+                                        (64, 520, 1024, False), (7, 1000, 4128, True),
+                                        (33, 264, 12288, True)])
+def test_fused_decode_linear_equals_unfused(bat, M, N, K, clip):
+    """bat_linear at decode sizes quantizes X inside the split-K GEMM; the codes and the
+    GEMM's summation order are those of bat_quantize_act + bat_mxfp4_gemm, so Y is
+    identical bit for bit (and the unfused path is checked against the oracle above)."""
+    X = wl.random_bf16((M, K), seed=M + K, scale=3.0)
+    W = wl.random_bf16((N, K), seed=N + K, scale=0.02)
+    A, B, g_lo, g_hi = wl.random_factors(K // 32, seed=K + 9)
+    Xd, Ad, Bd = _dev_bf16(X), _dev_f32(A), _dev_f32(B)
+    gl = _dev_f32(g_lo) if clip else None
+    gh = _dev_f32(g_hi) if clip else None
+    Wq = bat.bat_prepare_weight(_dev_bf16(W), Ad, Bd)
+    for dt in (torch.float32, torch.bfloat16):
+        Y = bat.bat_linear(X=Xd, Wq=Wq, A=Ad, B=Bd, g_lo=gl, g_hi=gh, out_dtype=dt)
+        Xq = bat.bat_quantize_act(Xd, Ad, Bd, gl, gh)
+        Y2 = bat.bat_mxfp4_gemm(Xq, Wq, out_dtype=dt)
+        Y3 = bat.bat_linear_noalloc(Xd, Wq, Ad, Bd, gl, gh, out_dtype=dt)
+        torch.cuda.synchronize()
+        assert torch.equal(Y, Y2)
+        assert torch.equal(Y3, Y2)
+    assert bat.bat_device_error() == 0

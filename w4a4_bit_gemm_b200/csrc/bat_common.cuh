@@ -323,6 +323,74 @@ __host__ __device__ constexpr uint32_t idesc_mxf4(int m, int n, uint32_t a_sf_id
          (a_sf_id & 3u) << 29;            // A scale-factor id
 }
 
+// ---------------------------------------------------------------- row quantizer math
+// (shared by the CUDA-core row quantizer and the fused decode linear)
+template <int kLs>  // kLs >= 0: the split as a constant; -1: read it from `ls`
+__device__ __forceinline__ void rows_build_pc(float (&pc)[32][4], const float* __restrict__ a,
+                                              const float* __restrict__ b, int bq, int u, int ls_rt) {
+  const int ls = kLs >= 0 ? kLs : ls_rt;
+  const int sm = (1 << ls) - 1, tt = 32 >> ls;
+  const float* bb = b + static_cast<int64_t>(bq) * tt * tt;
+#pragma unroll
+  for (int k = 0; k < 32; ++k)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = 4 * u + j;
+      pc[k][j] = __fmul_rn(__ldg(bb + (k >> ls) * tt + (n >> ls)), __ldg(a + ((k & sm) << ls) + (n & sm)));
+    }
+}
+
+// The 32 bf16 inputs of one block (64 bytes, 16-byte aligned) as fp32.
+__device__ __forceinline__ void rows_load_block(const uint16_t* src16, float (&x)[32]) {
+  const uint4* src = reinterpret_cast<const uint4*>(src16);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 w = src[c];
+    x[8 * c + 0] = bf16lo(w.x); x[8 * c + 1] = bf16hi(w.x);
+    x[8 * c + 2] = bf16lo(w.y); x[8 * c + 3] = bf16hi(w.y);
+    x[8 * c + 4] = bf16lo(w.z); x[8 * c + 5] = bf16hi(w.z);
+    x[8 * c + 6] = bf16lo(w.w); x[8 * c + 7] = bf16hi(w.w);
+  }
+}
+
+// One block of one row, spread over the eight lanes (l & ~7) .. (l | 7) of the warp:
+// this lane's transformed values y[j] = sum_k x[k] P_b[k][4u + j] (fp32, k ascending),
+// the block clip and the MX scale (min / max over the eight lanes by shuffles, so the
+// whole warp must call it together), and this lane's four codes: E2M1 in the low 16
+// bits (element 4u in the lowest nibble) or E4M3 in 32 bits (4u in the lowest byte).
+template <bool kFp8>
+__device__ __forceinline__ void rows_block_quant(const float (&x)[32], const float (&pc)[32][4],
+                                                 float r_lo, float r_hi, float (&y)[4],
+                                                 uint32_t& code, int& sbyte) {
+  uint64_t y01 = 0ull, y23 = 0ull;
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const uint64_t xx = pack2(x[k], x[k]);
+    y01 = ffma2(xx, pack2(pc[k][0], pc[k][1]), y01);
+    y23 = ffma2(xx, pack2(pc[k][2], pc[k][3]), y23);
+  }
+  unpack2(y01, y[0], y[1]);
+  unpack2(y23, y[2], y[3]);
+  float mn = fminf(fminf(y[0], y[1]), fminf(y[2], y[3]));
+  float mx = fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  const float lo = __fmul_rn(r_lo, mn);
+  const float hi = __fmul_rn(r_hi, mx);
+  const float amax = fmaxf(fabsf(fminf(fmaxf(mn, lo), hi)), fabsf(fminf(fmaxf(mx, lo), hi)));
+  constexpr int kEmax = kFp8 ? 8 : 2;
+  const int efield = static_cast<int>(__float_as_uint(amax) >> 23);
+  sbyte = efield > kEmax ? efield - kEmax : 0;  // e + 127
+  const float inv_scale = __uint_as_float(static_cast<uint32_t>(254 - sbyte) << 23);  // 2^-e
+  float v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = __fmaf_rn(fminf(fmaxf(y[i], lo), hi), inv_scale, 0.0f);
+  code = kFp8 ? e4m3x4(v[0], v[1], v[2], v[3]) : (e2m1x2(v[0], v[1]) | (e2m1x2(v[2], v[3]) << 8));
+}
+
 // Instruction descriptor of kind::mxf8f6f4 with A in E4M3 and B in E2M1 (format codes
 // 0 and 5 of that kind), fp32 accumulation, UE8M0 scales, both operands K-major.
 __host__ __device__ constexpr uint32_t idesc_mxf8f6f4_e4m3_e2m1(int m, int n, uint32_t a_sf_id,

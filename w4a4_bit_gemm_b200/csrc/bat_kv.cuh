@@ -112,21 +112,6 @@ struct RowQuantParams {
   int nbp4;               // linear mode: ceil(nb/4) of the tiled scale layout
 };
 
-template <int kLs>  // kLs >= 0: the split as a constant; -1: read it from `ls`
-__device__ __forceinline__ void rows_build_pc(float (&pc)[32][4], const float* __restrict__ a,
-                                              const float* __restrict__ b, int bq, int u, int ls_rt) {
-  const int ls = kLs >= 0 ? kLs : ls_rt;
-  const int sm = (1 << ls) - 1, tt = 32 >> ls;
-  const float* bb = b + static_cast<int64_t>(bq) * tt * tt;
-#pragma unroll
-  for (int k = 0; k < 32; ++k)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = 4 * u + j;
-      pc[k][j] = __fmul_rn(__ldg(bb + (k >> ls) * tt + (n >> ls)), __ldg(a + ((k & sm) << ls) + (n & sm)));
-    }
-}
-
 // kKv: rows are (token, head) pairs stored into cache slots (codes [slot][H][D] or
 // [slot][H][D/2], scales plain [slot][H][D/32]); otherwise rows of an activation
 // matrix (codes [M][D] or [M][D/2], scales in the GEMM's tiled layout, padding 0).
@@ -162,58 +147,22 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
         }
       }
       float x[32];
-      {
-        const uint4* src = reinterpret_cast<const uint4*>(p.x + row * p.D + bq * kG);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint4 w = src[c];
-          x[8 * c + 0] = bf16lo(w.x); x[8 * c + 1] = bf16hi(w.x);
-          x[8 * c + 2] = bf16lo(w.y); x[8 * c + 3] = bf16hi(w.y);
-          x[8 * c + 4] = bf16lo(w.z); x[8 * c + 5] = bf16hi(w.z);
-          x[8 * c + 6] = bf16lo(w.w); x[8 * c + 7] = bf16hi(w.w);
-        }
-      }
-      uint64_t y01 = 0ull, y23 = 0ull;
-#pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const uint64_t xx = pack2(x[k], x[k]);
-        y01 = ffma2(xx, pack2(pc[k][0], pc[k][1]), y01);
-        y23 = ffma2(xx, pack2(pc[k][2], pc[k][3]), y23);
-      }
+      rows_load_block(p.x + row * p.D + bq * kG, x);
       float y[4];
-      unpack2(y01, y[0], y[1]);
-      unpack2(y23, y[2], y[3]);
+      uint32_t code;
+      int sbyte;
+      rows_block_quant<kFp8>(x, pc, r_lo, r_hi, y, code, sbyte);
       const int64_t e0 = row * p.D + blk * kG + 4 * u;
       if (kTrace && has)
         *reinterpret_cast<float4*>(p.y_out + e0) = make_float4(y[0], y[1], y[2], y[3]);
-      // block min / max over the block's 8 lanes
-      float mn = fminf(fminf(y[0], y[1]), fminf(y[2], y[3]));
-      float mx = fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
-#pragma unroll
-      for (int o = 1; o < 8; o <<= 1) {
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      }
       if (!has || slot < 0) continue;
-      const float lo = __fmul_rn(r_lo, mn);
-      const float hi = __fmul_rn(r_hi, mx);
-      const float amax = fmaxf(fabsf(fminf(fmaxf(mn, lo), hi)), fabsf(fminf(fmaxf(mx, lo), hi)));
-      constexpr int kEmax = kFp8 ? 8 : 2;
-      const int efield = static_cast<int>(__float_as_uint(amax) >> 23);
-      const int sbyte = efield > kEmax ? efield - kEmax : 0;  // e + 127
-      const float inv_scale = __uint_as_float(static_cast<uint32_t>(254 - sbyte) << 23);  // 2^-e
-      float v[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) v[i] = __fmaf_rn(fminf(fmaxf(y[i], lo), hi), inv_scale, 0.0f);
       // element index of the code: cache row (slot, head) or the activation row
       const int64_t crow = kKv ? slot * p.H + row % p.H : row;
       const int64_t ci = crow * p.D + blk * kG + 4 * u;
-      if (kFp8) {
-        *reinterpret_cast<uint32_t*>(p.codes + ci) = e4m3x4(v[0], v[1], v[2], v[3]);
-      } else {
-        const uint32_t c = e2m1x2(v[0], v[1]) | (e2m1x2(v[2], v[3]) << 8);
-        *reinterpret_cast<uint16_t*>(p.codes + ci / 2) = static_cast<uint16_t>(c);
-      }
+      if (kFp8)
+        *reinterpret_cast<uint32_t*>(p.codes + ci) = code;
+      else
+        *reinterpret_cast<uint16_t*>(p.codes + ci / 2) = static_cast<uint16_t>(code);
       if (u == 0) {
         if (kKv)
           p.scales[crow * p.nb + blk] = static_cast<uint8_t>(sbyte);
