@@ -404,7 +404,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="mlp_gate_up", choices=wl.ORDER)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--ref-budget-s", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -503,14 +503,11 @@ def main():
     Y = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     gemm_fn = bat.bat_w4a8_gemm if a8 else bat.bat_mxfp4_gemm
-    # W4A4 with the default factor split: the step is the public bat_linear, which at
-    # decode sizes (at most 64 rows, a split-K shape) quantizes X inside the GEMM in
-    # one launch; otherwise it is the quantizer followed by the GEMM
+    # W4A4 with the default factor split: the step is the public bat_linear (the
+    # quantizer and the GEMM on one stream); otherwise the two calls directly
     use_linear = not a8 and args.shared == 8
     ws_step = torch.empty(bat.bat_linear_workspace_bytes(w.M, w.K), dtype=torch.uint8, device=dev)
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    fused = use_linear and w.M <= 64 and 2 * -(-w.N // 256) <= sms and -(-w.K // 256) >= 2
-    launches_per_step = 1 if fused else 2
+    launches_per_step = 2
 
     def step():
         if use_linear:
@@ -582,30 +579,54 @@ def main():
     # end to end through the public API: pinned host X -> device, linear, Y -> pinned host
     e2e = None
     if not args.no_e2e:
+        # Two lanes (streams, each with its own buffers) take alternate steps, so one
+        # step's host copies overlap the other's kernels and copies in the other
+        # direction, as a serving loop would run them; every step still copies its X
+        # in from pinned host memory and its Y out.
         Xh = torch.from_numpy(X_host.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
-        Yh = torch.empty(w.M, w.N, dtype=torch.bfloat16).pin_memory()
-        Xdev = torch.empty_like(X)
-        ws = torch.empty(bat.bat_linear_workspace_bytes(w.M, w.K), dtype=torch.uint8, device=dev)
+        lanes = []
+        for _ in range(2):
+            lanes.append({
+                "stream": torch.cuda.Stream(dev),
+                "Xdev": torch.empty_like(X),
+                "Y": torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev),
+                "Yh": torch.empty(w.M, w.N, dtype=torch.bfloat16).pin_memory(),
+                "ws": torch.empty(bat.bat_linear_workspace_bytes(w.M, w.K), dtype=torch.uint8,
+                                  device=dev),
+                "Xq": (bat.MXFP8 if a8 else bat.MXFP4).empty(w.M, w.K, dev),
+            })
 
-        def e2e_step():
-            Xdev.copy_(Xh, non_blocking=True)
-            if args.shared == 8 and not a8:
-                bat.bat_linear(Xdev, Wq, A, B, gl, gh, Y=Y, out_dtype=torch.bfloat16,
-                               workspace=ws, stream=stream)
-            else:
-                quantize(Xdev, Xq)
-                gemm_fn(Xq, Wq, Y=Y, out_dtype=torch.bfloat16, stream=stream)
-            Yh.copy_(Y, non_blocking=True)
+        def e2e_step(i):
+            ln = lanes[i % 2]
+            ls = ln["stream"]
+            with torch.cuda.stream(ls):
+                ln["Xdev"].copy_(Xh, non_blocking=True)
+                if args.shared == 8 and not a8:
+                    bat.bat_linear(ln["Xdev"], Wq, A, B, gl, gh, Y=ln["Y"], out_dtype=torch.bfloat16,
+                                   workspace=ln["ws"], stream=ls)
+                elif a8:
+                    bat.bat_quantize_act_mxfp8(ln["Xdev"], A, B, gl, gh, Xq=ln["Xq"], stream=ls)
+                    gemm_fn(ln["Xq"], Wq, Y=ln["Y"], out_dtype=torch.bfloat16, stream=ls)
+                else:
+                    bat.bat_quantize_act_gpk(ln["Xdev"], A, B, gl, gh, Xq=ln["Xq"], stream=ls)
+                    gemm_fn(ln["Xq"], Wq, Y=ln["Y"], out_dtype=torch.bfloat16, stream=ls)
+                ln["Yh"].copy_(ln["Y"], non_blocking=True)
 
-        for _ in range(3):
-            e2e_step()
+        for i in range(4):
+            e2e_step(i)
         torch.cuda.synchronize()
         if pg:
             pg.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
+        for ln in lanes:
+            ln["stream"].wait_event(e0)
+        for i in range(args.e2e_steps):
+            e2e_step(i)
+        for ln in lanes:
+            done = torch.cuda.Event()
+            done.record(ln["stream"])
+            stream.wait_event(done)
         e1.record(stream)
         torch.cuda.synchronize()
         te = max_over_ranks(pg, [e0.elapsed_time(e1) * 1e-3], dev)[0]
@@ -632,8 +653,7 @@ def main():
                                     f"B_b {32 // args.shared}x{32 // args.shared} private",
                        "l2": "flushed between steps (256 MiB write + read outside the timed events)",
                        "parallelism": f"replicas x{world} (independent token batches)"},
-            # the timed pass: quantizer + GEMM per step, or the fused decode linear
-            "gpu_launches": launches_per_step * K_ * world,
+            "gpu_launches": launches_per_step * K_ * world,  # timed pass: quantizer + GEMM
             "roofline": {"bound": "tensor", "achieved": gemm_tf, "peak": fp4_peak,
                          "unit": "TFLOP/s", "frac": gemm_tf / fp4_peak,
                          "traffic": recorded_traffic(gemm_kernel, w.name),

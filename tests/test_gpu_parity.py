@@ -690,12 +690,11 @@ def test_split_k_is_deterministic(bat):
 
 
 @pytest.mark.parametrize("M,N,K,clip", [(16, 6144, 4096, True), (1, 256, 2048, True),
-                                        (64, 520, 1024, False), (7, 1000, 4128, True),
-                                        (33, 264, 12288, True)])
-def test_fused_decode_linear_equals_unfused(bat, M, N, K, clip):
-    """bat_linear at decode sizes quantizes X inside the split-K GEMM; the codes and the
-    GEMM's summation order are those of bat_quantize_act + bat_mxfp4_gemm, so Y is
-    identical bit for bit (and the unfused path is checked against the oracle above)."""
+                                        (16, 520, 1024, False), (7, 1000, 4128, True),
+                                        (64, 520, 1024, True), (33, 264, 12288, True)])
+def test_linear_at_decode_sizes_equals_two_calls(bat, M, N, K, clip):
+    """bat_linear and bat_linear_noalloc at decode sizes (row quantizer, split-K GEMM)
+    equal bat_quantize_act followed by bat_mxfp4_gemm bit for bit."""
     X = wl.random_bf16((M, K), seed=M + K, scale=3.0)
     W = wl.random_bf16((N, K), seed=N + K, scale=0.02)
     A, B, g_lo, g_hi = wl.random_factors(K // 32, seed=K + 9)

@@ -32,7 +32,7 @@ struct DeviceInfo {
   std::atomic<int> sms{0};
   std::atomic<int> gemm_attr{0};    // bit 0: W4A4 GEMM, bit 1: W4A8 GEMM attribute set
   std::atomic<int> pro_attr{0};     // bit t: the prologue variant t has its smem attribute set
-  std::atomic<int> max_clusters[3][9];  // [W4A4, W4A8, fused][cluster size]: clusters at once, 0 unknown
+  std::atomic<int> max_clusters[2][9];  // [W4A8][cluster size]: clusters resident at once, 0 unknown
 };
 DeviceInfo g_dev[64];
 
@@ -353,23 +353,13 @@ bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float
 }
 
 // a8: Xq holds MXFP8 (E4M3) activations and the W4A8 kernel runs; K % 128 == 0 then.
-// Returned by launch_gemm when a fused launch was asked for but the shape does not
-// run split-K (the caller then quantizes and launches the GEMM separately).
-constexpr bat_status_t kNotFused = static_cast<bat_status_t>(100);
-
-// fuse != null: the fused decode linear (W4A4, default factor split), X quantized inside
-// the GEMM from fuse->fx / fa / fb / fg_lo / fg_hi; Xq supplies only rows and k.
 bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
-                         bat_out_dtype_t out_dtype, cudaStream_t stream, bool a8 = false,
-                         const bat::GemmParams* fuse = nullptr) {
+                         bat_out_dtype_t out_dtype, cudaStream_t stream, bool a8 = false) {
   int dev = 0, sms = 0;
   bat_status_t st = current_device(&dev, &sms);
   if (st != BAT_OK) return st;
   CUtensorMap ta, tb, ty;
-  if (fuse) {
-    if (!make_code_map(&tb, Wq->codes, Wq->rows, Wq->k, bat::gemm::kBN)) return BAT_ERR_CUDA;
-    ta = tb;  // the A side is produced in the kernel; the map is never loaded from
-  } else if (a8) {
+  if (a8) {
     if (!make_code8_map(&ta, Xq->codes, Xq->rows, Xq->k, bat::gemm::kBM)) return BAT_ERR_CUDA;
     if (!make_code4_unpack_map(&tb, Wq->codes, Wq->rows, Wq->k, bat::gemm::kBN)) return BAT_ERR_CUDA;
   } else {
@@ -391,18 +381,7 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
   p.tma_store = (!p.out_f32 && p.vec_ok) ? 1 : 0;
   if (p.tma_store && !make_out_map(&ty, Y, p.M, p.N)) return BAT_ERR_CUDA;
   void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, bat::GemmParams) =
-      fuse ? bat::bat_mxf4_gemm_kernel<false, true>
-           : (a8 ? bat::bat_mxf4_gemm_kernel<true> : bat::bat_mxf4_gemm_kernel<false>);
-  if (fuse) {
-    p.fx = fuse->fx;
-    p.fa = fuse->fa;
-    p.fb = fuse->fb;
-    p.fg_lo = fuse->fg_lo;
-    p.fg_hi = fuse->fg_hi;
-  } else {
-    p.fx = nullptr;
-    p.fa = p.fb = p.fg_lo = p.fg_hi = nullptr;
-  }
+      a8 ? bat::bat_mxf4_gemm_kernel<true> : bat::bat_mxf4_gemm_kernel<false>;
   const int smem = a8 ? bat::gemm::Cfg<true>::kSmemBytes : bat::gemm::Cfg<false>::kSmemBytes;
   const int64_t m_tiles = (p.M + bat::gemm::kBM - 1) / bat::gemm::kBM;
   const int64_t tiles = m_tiles * ((p.N + bat::gemm::kBN - 1) / bat::gemm::kBN);
@@ -410,7 +389,7 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
   // shapes): up to 8 CTAs per tile, at least one K stage each.
   const int64_t k_stages = (p.K + (a8 ? 127 : 255)) / (a8 ? 128 : 256);
   DeviceInfo& d = g_dev[dev];
-  const int variant_bit = fuse ? 8 : (a8 ? 2 : 1);
+  const int variant_bit = a8 ? 2 : 1;
   if (!(d.gemm_attr.load() & variant_bit)) {
     const cudaError_t ae =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -424,7 +403,7 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
     if (splits > k_stages) splits = k_stages;
     // the largest cluster size whose clusters all fit on the GPU at once (one wave)
     for (; splits > 1; --splits) {
-      std::atomic<int>& mc = d.max_clusters[fuse ? 2 : (a8 ? 1 : 0)][splits];
+      std::atomic<int>& mc = d.max_clusters[a8 ? 1 : 0][splits];
       int n = mc.load();
       if (n == 0) {
         cudaLaunchConfig_t oc = {};
@@ -445,7 +424,6 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
     }
   }
   p.splits = static_cast<int>(splits);
-  if (fuse && splits < 2) return kNotFused;
   const int grid = splits > 1 ? static_cast<int>(tiles * splits)
                               : static_cast<int>(tiles < sms ? tiles : sms);
   // Programmatic stream serialization: the kernel's set-up may overlap the previous
@@ -466,26 +444,6 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
   cfg.attrs = attr;
   cfg.numAttrs = splits > 1 ? 2 : 1;
   return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, p));
-}
-
-// The decode linear in one launch (rows <= kRowsCudaCore and a split-K GEMM shape):
-// returns kNotFused, having launched nothing, for any other shape.
-bat_status_t launch_linear_fused(const void* X, int64_t M, const float* A, const float* B,
-                                 const float* g_lo, const float* g_hi, const bat_mxfp4_t* Wq,
-                                 void* Y, bat_out_dtype_t out_dtype, cudaStream_t stream) {
-  if (M > kRowsCudaCore) return kNotFused;
-  bat::GemmParams f;
-  f.fx = static_cast<const uint16_t*>(X);
-  f.fa = A;
-  f.fb = B;
-  f.fg_lo = g_lo;
-  f.fg_hi = g_hi;
-  bat_mxfp4_t xq;  // shape only
-  xq.codes = nullptr;
-  xq.scales = nullptr;
-  xq.rows = M;
-  xq.k = Wq->k;
-  return launch_gemm(&xq, Wq, Y, out_dtype, stream, false, &f);
 }
 
 bat_status_t check_gemm_args(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, const void* Y,
@@ -847,8 +805,6 @@ bat_status_t bat_linear(const void* X, int64_t M, const bat_mxfp4_t* Wq, const f
   st = check_gemm_args(&xq, Wq, Y, out_dtype);
   if (st != BAT_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = launch_linear_fused(X, M, A, B, g_lo, g_hi, Wq, Y, out_dtype, s);
-  if (st != kNotFused) return st;
   st = launch_prologue(X, M, K, A, B, g_lo, g_hi, false, &xq, nullptr, s);
   if (st != BAT_OK) return st;
   return launch_gemm(&xq, Wq, Y, out_dtype, s);
@@ -979,8 +935,6 @@ extern "C" bat_status_t bat_linear_noalloc(const void* X, int64_t M, const bat_m
   xq.scales = static_cast<uint8_t*>(scratch) +
               round_up(static_cast<int64_t>(bat_mxfp4_codes_bytes(M, K)), 256);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = launch_linear_fused(X, M, A, B, g_lo, g_hi, Wq, Y, out_dtype, s);
-  if (st != kNotFused) return st;
   st = launch_prologue(X, M, K, A, B, g_lo, g_hi, false, &xq, nullptr, s);
   if (st != BAT_OK) return st;
   return launch_gemm(&xq, Wq, Y, out_dtype, s);

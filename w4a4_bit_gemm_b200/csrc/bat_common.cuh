@@ -324,8 +324,9 @@ __host__ __device__ constexpr uint32_t idesc_mxf4(int m, int n, uint32_t a_sf_id
 }
 
 // ---------------------------------------------------------------- row quantizer math
-// (shared by the CUDA-core row quantizer and the fused decode linear)
-template <int kLs>  // kLs >= 0: the split as a constant; -1: read it from `ls`
+// kLs >= 0: the split as a constant; -1: read it from `ls_rt`. kGlobal: a and b point to
+// global memory (read through the read-only cache); otherwise to shared memory.
+template <int kLs, bool kGlobal = true>
 __device__ __forceinline__ void rows_build_pc(float (&pc)[32][4], const float* __restrict__ a,
                                               const float* __restrict__ b, int bq, int u, int ls_rt) {
   const int ls = kLs >= 0 ? kLs : ls_rt;
@@ -336,7 +337,9 @@ __device__ __forceinline__ void rows_build_pc(float (&pc)[32][4], const float* _
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int n = 4 * u + j;
-      pc[k][j] = __fmul_rn(__ldg(bb + (k >> ls) * tt + (n >> ls)), __ldg(a + ((k & sm) << ls) + (n & sm)));
+      const float* pb = bb + (k >> ls) * tt + (n >> ls);
+      const float* pa = a + ((k & sm) << ls) + (n & sm);
+      pc[k][j] = kGlobal ? __fmul_rn(__ldg(pb), __ldg(pa)) : __fmul_rn(*pb, *pa);
     }
 }
 

@@ -92,12 +92,6 @@ struct GemmParams {
   int vec_ok;          // rows of Y are 16-byte aligned for vector stores
   int tma_store;       // bf16 output written through the staged TMA store
   int splits;          // K splits = cluster size (1: persistent, whole K per tile)
-  // fused decode linear (kFuse): the activation tiles are quantized inside the kernel
-  const uint16_t* fx;  // bf16 X [M][K]
-  const float* fa;     // A [8][8]
-  const float* fb;     // B [K/32][4][4]
-  const float* fg_lo;  // clip logits [K/32], or null
-  const float* fg_hi;
 };
 
 __device__ __forceinline__ uint4 lds_v4_u32(uint32_t addr) {
@@ -241,81 +235,10 @@ __device__ __forceinline__ void split_reduce(const GemmParams& p, uint8_t* base_
   }
 }
 
-// The fused decode linear's A side, run by the four epilogue warps (threads 0..127) of a
-// split-K CTA before its epilogue: for each of the CTA's k-steps, wait for the stage,
-// quantize rows [0, M) of its eight blocks into the stage's A tile (128-byte swizzled
-// rows of packed E2M1) and scale chunks, and arrive on the stage's full barrier. Warp w
-// takes the group of four blocks w & 1 and the rows w >> 1, w >> 1 + 2, ...; rows past
-// M were zeroed once and stay zero.
-template <int kStageBytes>
-__device__ __forceinline__ void fused_a_producer(const GemmParams& p, uint32_t base, uint32_t full0,
-                                                 uint32_t empty0, int kb, int ke, bool& ok) {
-  using namespace gemm;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, u = lane & 7;
-  // zero the A tiles and A scale chunks of every stage
-  constexpr int kZero16 = (kABytes + 2 * kChunk) / 16;  // 16-byte words per stage
-  for (int i = threadIdx.x; i < kStages * kZero16; i += 128) {
-    const int st = i / kZero16;
-    const int off = (i % kZero16) * 16;
-    const uint32_t a = base + st * kStageBytes + (off < kABytes ? off : kABytes + kBBytes + (off - kABytes));
-    st_shared_v4(a, 0u, 0u, 0u, 0u);
-  }
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-  const int nb = static_cast<int>(p.K / 32);
-  const int64_t rows = p.M < kBM ? p.M : kBM;
-  int stage = 0;
-  uint32_t phase = 0;
-  for (int ks = kb; ks < ke && ok; ++ks) {
-    // warp-uniform outcome: the shuffles below need every lane
-    if (!__all_sync(0xffffffffu, mbar_wait(empty0 + 8u * stage, phase ^ 1u, kErrWaitEmpty))) {
-      ok = false;
-      break;
-    }
-    const int jb = 4 * (warp & 1) + (lane >> 3);  // block within the stage
-    const int blk = 8 * ks + jb;
-    const bool has = blk < nb;
-    const int bq = has ? blk : 0;
-    const float r_lo = (has && p.fg_lo) ? clip_ratio(p.fg_lo[bq]) : 1.0f;
-    const float r_hi = (has && p.fg_hi) ? clip_ratio(p.fg_hi[bq]) : 1.0f;
-    float pc[32][4];
-    rows_build_pc<3>(pc, p.fa, p.fb, bq, u, 3);
-    const uint32_t sa = base + stage * kStageBytes;
-    for (int64_t m = warp >> 1; m < rows; m += 2) {
-      float x[32];
-      rows_load_block(p.fx + m * p.K + bq * kG, x);
-      float y[4];
-      uint32_t code;
-      int sbyte;
-      rows_block_quant<false>(x, pc, r_lo, r_hi, y, code, sbyte);
-      if (!has) {  // past K: zero codes and scale, like the zero fill of a tensor-map load
-        code = 0u;
-        sbyte = 0;
-      }
-      const int r = static_cast<int>(m);
-      asm volatile("st.shared.u16 [%0], %1;" ::"r"(sa + r * 128 + ((jb ^ (r & 7)) << 4) + 2 * u),
-                   "h"(static_cast<uint16_t>(code))
-                   : "memory");
-      if (u == 0) {
-        const uint32_t sf = sa + kABytes + kBBytes + (jb >> 2) * kChunk + (r & 31) * 16 +
-                            ((r >> 5) & 3) * 4 + (jb & 3);
-        asm volatile("st.shared.u8 [%0], %1;" ::"r"(sf), "h"(static_cast<uint16_t>(sbyte)) : "memory");
-      }
-    }
-    fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor cores
-    __syncwarp();
-    if (lane == 0) mbar_arrive(full0 + 8u * stage);
-    if (++stage == kStages) { stage = 0; phase ^= 1u; }
-  }
-}
-
 // kA8 = false: Xq MXFP4 (tmap_a over packed codes [M][K/2] bytes).
 // kA8 = true:  Xq MXFP8 E4M3 (tmap_a over codes [M][K] bytes) and tmap_b over Wq's packed
 //              E2M1 codes with the 16-elements-per-16-bytes shared-memory expansion.
-// kFuse (MXFP4, split-K launches of at most 128 rows): no Xq; the epilogue warps, idle
-//              until the accumulator is ready, quantize X into each stage's A tile and
-//              scale chunks with the CUDA-core row quantizer's arithmetic (default
-//              8 x 8 / 4 x 4 split), so the codes equal those of the unfused path.
-template <bool kA8, bool kFuse = false>
+template <bool kA8>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
     bat_mxf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                          const __grid_constant__ CUtensorMap tmap_b,
@@ -346,7 +269,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(full_bar(s), kFuse ? 1 + 4 : 1);  // + the four A-producing warps
+      mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
     mbar_init(tmem_full, 1);
@@ -403,16 +326,14 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
           // the unpacking load of W (kA8) moves 64 bytes per row: its 8-byte gaps in shared
           // memory are not written and count no transaction bytes
           constexpr uint32_t kBTx = kA8 ? kBBytes / 2 : kBBytes;
-          const uint32_t bytes = (kFuse ? 0u : static_cast<uint32_t>(kABytes)) + kBTx +
-                                 static_cast<uint32_t>(nch) * kChunk * ((kFuse ? 0 : 1) + ngb);
+          const uint32_t bytes = kABytes + kBTx + static_cast<uint32_t>(nch) * kChunk * (1 + ngb);
           const uint32_t sa = base + stage * kStageBytes;
           // the expected bytes include the scale copies warp 10 issues (their completions may
           // come first: the phase still waits for this arrival)
           mbar_expect_tx(full_bar(stage), bytes);
           // x of both maps is 128 per stage: bytes of packed E2M1, E4M3 elements, or
           // (unpacking load) E2M1 elements
-          if (!kFuse)
-            tma_load_2d(sa, &tmap_a, full_bar(stage), ks * 128, static_cast<int32_t>(mt * kBM));
+          tma_load_2d(sa, &tmap_a, full_bar(stage), ks * 128, static_cast<int32_t>(mt * kBM));
           tma_load_2d(sa + kABytes, &tmap_b, full_bar(stage), ks * 128,
                       static_cast<int32_t>(nt * kBN));
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -435,9 +356,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
           const int c0 = ks * kChunksPerStage;
           const int nch = min(kChunksPerStage, p.nbp4 - c0);
           const uint32_t sa = base + stage * kStageBytes;
-          if (!kFuse)
-            bulk_load(sa + kABytes + kBBytes, p.sfa + (mt * p.nbp4 + c0) * kChunk, nch * kChunk,
-                      full_bar(stage));
+          bulk_load(sa + kABytes + kBBytes, p.sfa + (mt * p.nbp4 + c0) * kChunk, nch * kChunk,
+                    full_bar(stage));
           for (int g = 0; g < ngb; ++g)
             bulk_load(sa + kABytes + kBBytes + kSfaBytes + g * (kChunksPerStage * kChunk),
                       p.sfb + ((nt * 2 + g) * p.nbp4 + c0) * kChunk, nch * kChunk, full_bar(stage));
@@ -555,7 +475,6 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     const int rl = 32 * q + lane;  // row within the tile
     const bool leader = (warp == 0 && lane == 0);
     uint32_t acc_phase = 0;
-    if constexpr (kFuse) fused_a_producer<kStageBytes>(p, base, full_bar(0), empty_bar(0), kb, ke, ok);
     for (int64_t tile = tile0; tile < tiles && ok; tile += tstride) {
       const int64_t mt = tile % m_tiles;
       const int64_t nt = tile / m_tiles;
