@@ -115,3 +115,34 @@ def test_block_hadamard_factors_host():
                                   (scipy.linalg.hadamard(t) / np.sqrt(t)).astype(np.float32))
     with pytest.raises(bat.BatError):
         bat.bat_block_hadamard_factors(3, 2)
+
+
+def test_kv_and_w4a8_host_validation(L):
+    p = _fake_ptr()
+    # cache sizes
+    assert bat.lib().bat_kv_codes_bytes(10, 8, 128, 0) == 10 * 8 * 128
+    assert bat.lib().bat_kv_codes_bytes(10, 8, 128, 1) == 10 * 8 * 64
+    assert bat.lib().bat_kv_scales_bytes(10, 8, 128) == 10 * 8 * 4
+    assert bat.lib().bat_kv_codes_bytes(10, 8, 100, 0) == 0
+    assert bat.lib().bat_mxfp8_codes_bytes(4, 64) == 256
+    # kv store: bad split, bad head size, null pointers, bad format, misaligned slots
+    args = lambda **kw: [kw.get("kv", p), kw.get("T", 4), kw.get("H", 2), kw.get("D", 64), p,
+                         kw.get("s", 8), p, None, None, kw.get("slots", p), kw.get("fmt", 0), p, p,
+                         kw.get("S", 8), None, None]
+    assert L.bat_kv_quantize(*args(s=3)) == 6
+    assert L.bat_kv_quantize(*args(D=48)) == 2
+    assert L.bat_kv_quantize(*args(D=512)) == 2
+    assert L.bat_kv_quantize(*args(kv=None)) == 1
+    assert L.bat_kv_quantize(*args(fmt=7)) == 1
+    assert L.bat_kv_quantize(*args(T=0)) == 1
+    assert L.bat_kv_quantize(*args(slots=_fake_ptr(4))) == 3
+    assert L.bat_kv_dequantize(p, p, 8, 2, 64, 0, p, 4, None, 8, None, p, 7, None) == 1
+    assert L.bat_kv_dequantize(p, p, 8, 2, 64, 0, p, 4, p, 8, None, p, 0, None) == 1
+    # W4A8 GEMM: K % 128 != 0, misaligned weight codes
+    S = bat.MXFP4Struct
+    x8 = S(0x7F0000100000, 0x7F0000200000, 4, 96)
+    w8 = S(0x7F0000300000, 0x7F0000400000, 8, 96)
+    assert L.bat_w4a8_gemm(ctypes.byref(x8), ctypes.byref(w8), p, 0, None) == 2
+    x8 = S(0x7F0000100000, 0x7F0000200000, 4, 128)
+    w8 = S(0x7F0000300010, 0x7F0000400000, 8, 128)
+    assert L.bat_w4a8_gemm(ctypes.byref(x8), ctypes.byref(w8), p, 0, None) == 3
