@@ -21,15 +21,24 @@
  *   - Tensor pointers are DEVICE pointers owned by the caller. The online entry
  *     points never allocate device memory; the offline bat_prepare_weight(_gpk)
  *     allocates (and frees, stream-ordered) one temporary of about
- *     4*s*s + 4*K*32/s bytes for the inverted factors. No state is kept between calls except a sticky
- *     device error word (see bat_device_error).
+ *     4*s*s + 4*K*32/s bytes for the inverted factors. No state is kept between
+ *     calls except a sticky device error word (see bat_device_error) and, per
+ *     device, cached launch facts (kernel attributes set, how many clusters of a
+ *     given size fit), which do not change results.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
  *     asynchronous on it unless stated otherwise.
  *   - Arguments are validated on the host before any CUDA call; a bad argument
  *     returns an error status and launches nothing. CUDA failures return
  *     BAT_ERR_CUDA. The device must be sm_100 (B200); other devices get
  *     BAT_ERR_UNSUPPORTED.
- *   - Calls are thread-safe (no mutable global state on the host).
+ *   - Calls are thread-safe (the per-device caches are atomics written with
+ *     idempotent values).
+ *   - Shapes and routing: activation batches of at most 64 rows are quantized on
+ *     the CUDA cores, larger ones by the tensor-core prologue (the codes of one
+ *     path are exact with respect to its own fp32 transformed values; the two
+ *     paths' transformed values differ by fp32 rounding). A GEMM with one row of
+ *     128-row tiles that leaves most SMs idle runs split-K over thread-block
+ *     clusters, with a fixed summation order.
  *
  * Storage formats (bat_mxfp4_t):
  *   codes : [rows][k/2] bytes, row-major, two E2M1 codes per byte, element 2i in
