@@ -206,6 +206,10 @@ def run_reference(args, w, inp):
     steps, warm = args.steps, args.warmup
     per_step = max(0.05, min(2.0, args.ref_budget_s / max(1, steps + warm)))
     import oracle
+    a8 = args.act == "mxfp8"
+    fmt = "e4m3" if a8 else "e2m1"
+    if args.shared != 8:
+        inp.A, inp.B, _, _ = wl.random_factors(w.K // 32, seed=1, shared=args.shared)
     _, wc, ws = oracle.prepare_weight(inp.W, inp.A, inp.B)
     Wd = oracle.dequantize(wc, ws)
     rng = np.random.default_rng(1)
@@ -216,8 +220,8 @@ def run_reference(args, w, inp):
         rows = rng.choice(w.M, size=nrows, replace=False)
         cols = np.sort(rng.choice(w.N, size=ncols, replace=False))
         t0 = time.perf_counter()
-        _, xc, xs = oracle.quantize_act(inp.X[rows], inp.A, inp.B, inp.g_lo, inp.g_hi)
-        oracle.gemm_sampled(oracle.dequantize(xc, xs), Wd, None, cols)
+        _, xc, xs = oracle.quantize_act(inp.X[rows], inp.A, inp.B, inp.g_lo, inp.g_hi, fmt=fmt)
+        oracle.gemm_sampled(oracle.dequantize(xc, xs, fmt), Wd, None, cols)
         return time.perf_counter() - t0
 
     step(w.N)  # page in the dequantized weights
@@ -232,7 +236,7 @@ def run_reference(args, w, inp):
     value = flops / total / 1e12
     desc = f"per step: {nrows} random token rows x {ncols} weight rows of {w.name} (K={w.K})"
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "impl": "reference", "metric": METRIC_W4A8 if a8 else METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": steps, "warmup": warm,
         "ms_per_step": 1e3 * total / steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -396,6 +400,53 @@ def run_kv(args, rank, world, local):
         pg.destroy_process_group()
 
 
+def run_reference_kv(args):
+    """The oracle's KV-cache store timed as the reference arm (same metric as --path kv)."""
+    import oracle
+    T = args.kv_tokens
+    k_host, v_host, fk, fv = kv_inputs(T, seed=rank_batch_seed(0))
+    fmt = "e4m3" if args.kv_format == "mxfp8" else "e2m1"
+    per_elt = 2.0 + (1.0 if args.kv_format == "mxfp8" else 0.5) + 1.0 / 32.0
+    rng = np.random.default_rng(0)
+    per_step = max(0.05, min(2.0, args.ref_budget_s / max(1, args.steps + args.warmup)))
+    nt = max(1, min(T, 64))
+    cc = np.zeros((nt, KV_HEADS, KV_DIM), np.uint8)
+    cs = np.zeros((nt, KV_HEADS, KV_DIM // 32), np.uint8)
+
+    def step():
+        n, t = 0, 0.0
+        while t < per_step:
+            rows = rng.choice(T, size=nt, replace=False)
+            t0 = time.perf_counter()
+            oracle.kv_quantize(k_host[rows], *fk, fmt, np.arange(nt), cc, cs)
+            oracle.kv_quantize(v_host[rows], *fv, fmt, np.arange(nt), cc, cs)
+            t += time.perf_counter() - t0
+            n += nt
+        return n, t
+
+    for _ in range(args.warmup):
+        step()
+    tot_n, tot_t = 0, 0.0
+    for _ in range(args.steps):
+        n, t = step()
+        tot_n += n
+        tot_t += t
+    value = per_elt * 2 * tot_n * KV_HEADS * KV_DIM / tot_t / 1e9
+    desc = f"per step: batches of {nt} random tokens of K and V (8 heads x 128) for about {per_step:.2f} s"
+    line = {
+        "impl": "reference", "metric": f"BAT KV-cache store GB/s (% HBM), {args.kv_format}",
+        "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"kv_store T={T}", "tokens": T, "kv_heads": KV_HEADS,
+                   "head_dim": KV_DIM, "format": args.kv_format},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ---------------------------------------------------------------- GPU leg
 def main():
     ap = argparse.ArgumentParser()
@@ -427,7 +478,10 @@ def main():
 
     if args.impl == "reference":
         if rank == 0:
-            run_reference(args, w, wl.make_inputs(w.name, seed=0))
+            if args.path == "kv":
+                run_reference_kv(args)
+            else:
+                run_reference(args, w, wl.make_inputs(w.name, seed=0))
         return
     if args.path == "kv":
         run_kv(args, rank, world, local)
