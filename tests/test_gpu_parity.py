@@ -598,9 +598,10 @@ def test_kv_quantize_parity(bat, fmt, T, H, D, S, s):
 
 
 @pytest.mark.parametrize("fmt", ["mxfp8", "mxfp4"])
-def test_kv_dequantize_parity(bat, fmt):
-    T, H, D, S = 24, 4, 128, 32
-    kv, A, B, g_lo, g_hi, slots, cache, _, _ = _kv_case(bat, T, H, D, S, fmt, seed=7)
+@pytest.mark.parametrize("D,s", [(128, 8), (96, 4), (256, 16)])
+def test_kv_dequantize_parity(bat, fmt, D, s):
+    T, H, S = 24, 4, 32
+    kv, A, B, g_lo, g_hi, slots, cache, _, _ = _kv_case(bat, T, H, D, S, fmt, s=s, seed=7)
     read = np.array([sl for sl in slots if sl >= 0] + [slots[slots >= 0][0]], np.int64)
     rd = torch.from_numpy(read).cuda()
     ofmt = "e4m3" if fmt == "mxfp8" else "e2m1"
