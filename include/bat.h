@@ -358,6 +358,16 @@ BAT_API bat_status_t bat_linear_noalloc(const void* X, int64_t M, const bat_mxfp
                                         void* stream);
 
 /*
+ * Self-test of the failure path every kernel wait uses: one thread waits on an
+ * mbarrier that nothing arrives on, gives up after `limit_ns` nanoseconds
+ * (1 .. 2e9), records the stall in the device error word (bat_device_error then
+ * returns a non-zero code) and sets *waited_out (device uint32) to 1. No trap and
+ * no endless wait; the context stays usable.
+ */
+BAT_API bat_status_t bat_selftest_bounded_wait(uint64_t limit_ns, unsigned int* waited_out,
+                                               void* stream);
+
+/*
  * Text of the last CUDA error that made a call on this host thread return
  * BAT_ERR_CUDA ("no CUDA error" if none). Static storage; per thread.
  */

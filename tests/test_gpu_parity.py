@@ -712,3 +712,15 @@ def test_linear_at_decode_sizes_equals_two_calls(bat, M, N, K, clip):
         assert torch.equal(Y, Y2)
         assert torch.equal(Y3, Y2)
     assert bat.bat_device_error() == 0
+
+
+def test_bounded_wait_reports_and_returns(bat):
+    """A wait on a barrier nothing arrives on runs out after its limit, sets the device
+    error word and returns; the context stays usable (a later call works)."""
+    assert bat.bat_device_error() == 0
+    assert bat.bat_selftest_bounded_wait(20_000_000) == 1
+    assert bat.bat_device_error() != 0
+    assert bat.bat_device_error() == 0
+    r = bat.bat_clip_ratios(None, 4)
+    torch.cuda.synchronize()
+    assert torch.all(r == 1.0)

@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
         "bat_kv_scales_bytes": (ctypes.c_size_t, [I64, I64, I64]),
         "bat_kv_quantize": (S, [P, I64, I64, I64, P, S, P, P, P, P, S, P, P, I64, P, P]),
         "bat_kv_dequantize": (S, [P, P, I64, I64, I64, S, P, I64, P, S, P, P, S, P]),
+        "bat_selftest_bounded_wait": (S, [ctypes.c_uint64, P, P]),
         "bat_mxfp4_gemm": (S, [SP, SP, P, S, P]),
         "bat_linear_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
         "bat_linear": (S, [P, I64, SP, P, P, P, P, P, S, P, ctypes.c_size_t, P]),
@@ -492,3 +493,11 @@ def bat_kv_dequantize(cache: KVCache, slots, A=None, B=None, out: Optional[torch
                                    cache.D, _KV_FMT[cache.fmt], _ptr(slots), T, _ptr(A), s, _ptr(B),
                                    _ptr(out), code, _stream(stream)), "bat_kv_dequantize")
     return out
+
+
+def bat_selftest_bounded_wait(limit_ns: int = 50_000_000, stream=None) -> int:
+    """Run the bounded-wait self-test; returns the device flag (1: the wait ran out)."""
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _check(lib().bat_selftest_bounded_wait(limit_ns, _ptr(flag), _stream(stream)),
+           "bat_selftest_bounded_wait")
+    return int(flag.item())

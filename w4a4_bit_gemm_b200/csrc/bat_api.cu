@@ -825,6 +825,40 @@ int bat_device_error(void) {
 
 }  // extern "C"
 
+// ---------------------------------------------------------------- bounded-wait self-test
+namespace bat {
+// One thread waits on an mbarrier that nothing arrives on, with the kernels' bounded
+// wait pattern but the caller's limit; when the limit runs out it records
+// kErrWaitFull in the device error word and returns (no trap, no endless spin).
+__global__ void bat_selftest_wait_kernel(uint64_t limit_ns, unsigned int* waited_out) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  const uint64_t t0 = globaltimer_ns();
+  bool done = false;
+  while (!done) {
+    if (mbar_try_wait_sleep(b, 0, 100000u)) break;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      atomicOr(&g_dev_error, kErrWaitFull);
+      done = true;
+    }
+  }
+  *waited_out = done ? 1u : 0u;
+  mbar_arrive(b);  // complete the phase before the barrier's memory goes away
+}
+}  // namespace bat
+
+extern "C" bat_status_t bat_selftest_bounded_wait(uint64_t limit_ns, unsigned int* waited_out,
+                                                  void* stream) {
+  if (!waited_out || limit_ns == 0 || limit_ns > 2000000000ull) return BAT_ERR_INVALID_ARG;
+  int dev = 0, sms = 0;
+  bat_status_t st = current_device(&dev, &sms);
+  if (st != BAT_OK) return st;
+  bat::bat_selftest_wait_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, waited_out);
+  return cuda_status(cudaGetLastError());
+}
+
 // ---------------------------------------------------------------- element conversion
 namespace bat {
 __global__ void bat_e2m1_encode_kernel(const float* v, int64_t n, uint8_t* codes) {
