@@ -52,8 +52,9 @@ constexpr int kABytes = kBM * 128;           // 16 KB: 128 bytes of codes per ro
 constexpr int kBBytes = kBN * 128;           // 32 KB
 constexpr int kChunk = 512;                  // one 128-row x 4-scale block of the scale layout
 constexpr int kThreads = 384;
-constexpr uint32_t kRegsEpi = 248;   // after setmaxnreg: 128 x 248 + 256 x 56 <= 384 x 168
-constexpr uint32_t kRegsOther = 56;
+constexpr uint32_t kRegsEpi = 232;   // after setmaxnreg: 128 x 232 + 256 x 80 <= 384 x 168
+constexpr uint32_t kRegsOther = 80;
+static_assert(128 * kRegsEpi + 256 * kRegsOther <= kThreads * 168, "register split");
 // split-K partial tile in shared memory: fp32 rows of 256 columns, padded to 260 floats
 // so that the epilogue's row-per-lane stores spread over the banks
 constexpr int kPartStride = kBN + 4;
