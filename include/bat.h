@@ -33,6 +33,9 @@
  *     BAT_ERR_UNSUPPORTED.
  *   - Calls are thread-safe (the per-device caches are atomics written with
  *     idempotent values).
+ *   - Row limit: every operand has at most 2^30 rows (activations M, weights N,
+ *     KV tokens x heads, cache slots x heads); more returns BAT_ERR_SHAPE. The
+ *     tensor-memory copies address a tile by 32-bit signed coordinates.
  *   - Shapes and routing: activation batches of at most 64 rows are quantized on
  *     the CUDA cores, larger ones by the tensor-core prologue (the codes of one
  *     path are exact with respect to its own fp32 transformed values; the two
@@ -117,7 +120,7 @@ BAT_API int bat_version(void);
  *                Ratios are sigma(g) evaluated in fp64 and rounded to fp32;
  *                g = +inf gives ratio 1.
  *   Xq    : output; Xq->rows must equal M and Xq->k must equal K.
- * Requirements: M >= 1, K >= 32, K % 32 == 0, K <= 262144.
+ * Requirements: 1 <= M <= 2^30, K >= 32, K % 32 == 0, K <= 262144.
  */
 BAT_API bat_status_t bat_quantize_act(const void* X, int64_t M, int64_t K, const float* A, const float* B,
                               const float* g_lo, const float* g_hi, const bat_mxfp4_t* Xq,

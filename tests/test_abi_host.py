@@ -146,3 +146,30 @@ def test_kv_and_w4a8_host_validation(L):
     x8 = S(0x7F0000100000, 0x7F0000200000, 4, 128)
     w8 = S(0x7F0000300010, 0x7F0000400000, 8, 128)
     assert L.bat_w4a8_gemm(ctypes.byref(x8), ctypes.byref(w8), p, 0, None) == 3
+
+
+def test_row_limit(L):
+    """Operands of more than 2^30 rows are rejected before any CUDA call: the tensor-memory
+    copies address tiles by 32-bit signed coordinates."""
+    S = bat.MXFP4Struct
+    p = _fake_ptr()
+    big = 1 << 30
+    over = S(0x7F0000100000, 0x7F0000200000, big + 1, 64)
+    w64 = S(0x7F0000300000, 0x7F0000400000, 8, 64)
+    assert L.bat_quantize_act(p, big + 1, 64, p, p, None, None, ctypes.byref(over), None) == 2
+    assert L.bat_mxfp4_gemm(ctypes.byref(over), ctypes.byref(w64), p, 0, None) == 2
+    assert L.bat_mxfp4_gemm(ctypes.byref(w64), ctypes.byref(over), p, 0, None) == 2
+    assert L.bat_prepare_weight(p, big + 1, 64, p, p, None, None, ctypes.byref(over), None,
+                                None) == 2
+    assert L.bat_linear(p, big + 1, ctypes.byref(w64), p, p, None, None, p, 0, p, 1 << 40,
+                        None) == 2
+    assert L.bat_linear_noalloc(p, big + 1, ctypes.byref(w64), p, p, None, None, p, 0, None) == 2
+    # KV stores: tokens x heads, and cache slots x heads
+    kv = lambda T, H, slots: L.bat_kv_quantize(p, T, H, 64, p, 8, p, None, None, p, 0, p, p,
+                                               slots, None, None)
+    assert kv(big // 2 + 1, 2, 8) == 2
+    assert kv(4, 2, big // 2 + 1) == 2
+    assert kv(4, big + 1, 8) == 2
+    # exactly 2^30 rows passes the shape check: a misaligned X is what fails next
+    at = S(0x7F0000100000, 0x7F0000200000, big, 64)
+    assert L.bat_quantize_act(_fake_ptr(2), big, 64, p, p, None, None, ctypes.byref(at), None) == 3

@@ -20,6 +20,10 @@
 namespace {
 
 constexpr int64_t kMaxK = 262144;
+// Rows of any operand (activations, weights, KV rows and cache slots x heads): the
+// tensor-memory copies address a tile by 32-bit signed coordinates, so every tile
+// origin must stay well below 2^31.
+constexpr int64_t kMaxRows = int64_t(1) << 30;
 constexpr double kMaxCond = 1e6;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -227,7 +231,7 @@ bat_status_t check_act_args(const void* X, int64_t M, int64_t K, const float* A,
   if (!X || !A || !B || !Xq) return BAT_ERR_INVALID_ARG;
   if ((g_lo == nullptr) != (g_hi == nullptr)) return BAT_ERR_INVALID_ARG;
   if (M < 1 || K < 32) return BAT_ERR_INVALID_ARG;
-  if (K % 32 != 0 || K > kMaxK) return BAT_ERR_SHAPE;
+  if (K % 32 != 0 || K > kMaxK || M > kMaxRows) return BAT_ERR_SHAPE;
   if (!aligned16(X) || !aligned16(A) || !aligned16(B)) return BAT_ERR_ALIGN;
   return check_mxfp4(Xq, M, K);
 }
@@ -452,6 +456,7 @@ bat_status_t check_gemm_args(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, const
   if (out_dtype != BAT_OUT_BF16 && out_dtype != BAT_OUT_F32) return BAT_ERR_INVALID_ARG;
   if (Xq->rows < 1 || Wq->rows < 1 || Xq->k < 32) return BAT_ERR_INVALID_ARG;
   if (Xq->k != Wq->k || Xq->k % 32 != 0 || Xq->k > kMaxK) return BAT_ERR_SHAPE;
+  if (Xq->rows > kMaxRows || Wq->rows > kMaxRows) return BAT_ERR_SHAPE;
   if (a8) {
     // the unpacking load of the weights: k % 128 == 0, 32-byte aligned codes
     if (Xq->k % 128 != 0) return BAT_ERR_SHAPE;
@@ -557,7 +562,7 @@ bat_status_t bat_prepare_weight_gpk(const void* W, int64_t N, int64_t K, const f
   if (!W || !A || !B || !Wq) return BAT_ERR_INVALID_ARG;
   if ((gw_lo == nullptr) != (gw_hi == nullptr)) return BAT_ERR_INVALID_ARG;
   if (N < 1 || K < 32) return BAT_ERR_INVALID_ARG;
-  if (K % 32 != 0 || K > kMaxK) return BAT_ERR_SHAPE;
+  if (K % 32 != 0 || K > kMaxK || N > kMaxRows) return BAT_ERR_SHAPE;
   if (!aligned16(W) || !aligned16(A) || !aligned16(B)) return BAT_ERR_ALIGN;
   if (wt_out && !aligned16(wt_out)) return BAT_ERR_ALIGN;
   bat_status_t st = check_mxfp4(Wq, N, K);
@@ -677,6 +682,8 @@ static bat_status_t kv_shape_check(int64_t T, int64_t H, int64_t D, int64_t num_
   if (*ls < 0) return BAT_ERR_UNSUPPORTED;
   if (T < 1 || H < 1 || num_slots < 1) return BAT_ERR_INVALID_ARG;
   if (D < 32 || D % 32 != 0 || D > 32 * bat::kv::kMaxBlocks) return BAT_ERR_SHAPE;
+  // (token, head) rows and cache rows, without forming a product that could overflow
+  if (H > kMaxRows || T > kMaxRows / H || num_slots > kMaxRows / H) return BAT_ERR_SHAPE;
   return BAT_OK;
 }
 
@@ -791,7 +798,7 @@ bat_status_t bat_linear(const void* X, int64_t M, const bat_mxfp4_t* Wq, const f
   if (!Wq) return BAT_ERR_INVALID_ARG;
   const int64_t K = Wq->k;
   if (M < 1 || K < 32) return BAT_ERR_INVALID_ARG;
-  if (K % 32 != 0 || K > kMaxK) return BAT_ERR_SHAPE;
+  if (K % 32 != 0 || K > kMaxK || M > kMaxRows) return BAT_ERR_SHAPE;
   const size_t need = bat_linear_workspace_bytes(M, K);
   if (!workspace || workspace_bytes < need) return BAT_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BAT_ERR_ALIGN;
@@ -943,7 +950,7 @@ extern "C" bat_status_t bat_linear_noalloc(const void* X, int64_t M, const bat_m
   if (!Wq) return BAT_ERR_INVALID_ARG;
   const int64_t K = Wq->k;
   if (M < 1 || K < 32) return BAT_ERR_INVALID_ARG;
-  if (K % 32 != 0 || K > kMaxK) return BAT_ERR_SHAPE;
+  if (K % 32 != 0 || K > kMaxK || M > kMaxRows) return BAT_ERR_SHAPE;
   const size_t need = bat_linear_workspace_bytes(M, K);
   if (need == 0 || need > BAT_NOALLOC_SCRATCH_BYTES) return BAT_ERR_WORKSPACE;
   bat_mxfp4_t xq;
