@@ -3,6 +3,7 @@ header declares, and rejects bad arguments on the host before any CUDA call."""
 from __future__ import annotations
 
 import ctypes
+import os
 
 import pytest
 
@@ -173,3 +174,22 @@ def test_row_limit(L):
     # exactly 2^30 rows passes the shape check: a misaligned X is what fails next
     at = S(0x7F0000100000, 0x7F0000200000, big, 64)
     assert L.bat_quantize_act(_fake_ptr(2), big, 64, p, p, None, None, ctypes.byref(at), None) == 3
+
+
+def test_missing_library_fails_loudly():
+    """The product path has no fallback: without libbat.so every call raises."""
+    import subprocess
+    import sys
+    code = (
+        "import w4a4_bit_gemm_b200 as bat\n"
+        "bat.LIB_PATH = '/nonexistent/libbat.so'\n"
+        "bat._lib = None\n"
+        "try:\n"
+        "    bat.bat_version()\n"
+        "except RuntimeError as e:\n"
+        "    print('raised', 'missing' in str(e))\n"
+        "else:\n"
+        "    print('no error')\n")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                         cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    assert out.stdout.strip() == "raised True", out.stdout + out.stderr
