@@ -384,11 +384,17 @@ def test_argument_errors_launch_nothing(bat):
     X = torch.zeros(4, 64, dtype=torch.bfloat16, device="cuda")
     A = torch.eye(8, device="cuda")
     B = torch.eye(4, device="cuda").repeat(2, 1, 1).contiguous()
-    Xq = bat.MXFP4.empty(4, 64)
-    bad = bat.MXFP4(Xq.codes, Xq.scales, 5, 64)
+    # a 5-row output for 4 rows of X: buffers large enough, so the library's shape check
+    # (not the binding's size check) is what refuses it
+    bad = bat.MXFP4.empty(5, 64)
     with pytest.raises(bat.BatError) as e:
         bat.bat_quantize_act(X, A, B, Xq=bad)
     assert e.value.status == 2
+    # buffers too small for the shape they claim: refused by the binding before any call
+    small = bat.MXFP4.empty(4, 64)
+    with pytest.raises(ValueError):
+        bat.bat_quantize_act(torch.zeros(8, 64, dtype=torch.bfloat16, device="cuda"), A, B,
+                             Xq=bat.MXFP4(small.codes, small.scales, 8, 64))
     st = bat.lib().bat_quantize_act(None, 4, 64, None, None, None, None, None, None)
     assert st == 1
     assert bat.bat_device_error() == 0

@@ -109,11 +109,17 @@ def _stream(stream: Optional[torch.cuda.Stream]):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _need(t: torch.Tensor, dtype: torch.dtype, name: str, shape=None) -> torch.Tensor:
+# The library takes device pointers only: every tensor handed to it must live in GPU memory.
+_DEVICE_TYPE = "cuda"
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, name: str, shape=None, device=None) -> torch.Tensor:
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if t.device.type != "cuda":
+    if t.device.type != _DEVICE_TYPE:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}; every tensor of the call must be on {device}")
     if t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
@@ -121,6 +127,23 @@ def _need(t: torch.Tensor, dtype: torch.dtype, name: str, shape=None) -> torch.T
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
     return t
+
+
+def _need_bytes(t: torch.Tensor, name: str, nbytes: int, device) -> torch.Tensor:
+    """A caller-supplied byte buffer the kernels write or read: large enough for its shape."""
+    _need(t, torch.uint8, name, device=device)
+    if t.numel() < nbytes:
+        raise ValueError(f"{name} holds {t.numel()} bytes; {nbytes} are needed")
+    return t
+
+
+def _on_device(dev: torch.device, stream) -> None:
+    """The kernels run on the current device, on `stream`: the tensors must live there."""
+    if dev.type == "cuda" and dev.index is not None and dev.index != torch.cuda.current_device():
+        raise ValueError(f"the tensors are on {dev} but the current device is "
+                         f"cuda:{torch.cuda.current_device()}; call under torch.cuda.device({dev})")
+    if stream is not None and getattr(stream, "device", dev) != dev:
+        raise ValueError(f"the stream belongs to {stream.device}, the tensors to {dev}")
 
 
 def _check(status: int, where: str) -> None:
@@ -151,6 +174,12 @@ class MXFP4:
     def struct(self) -> MXFP4Struct:
         return MXFP4Struct(self.codes.data_ptr(), self.scales.data_ptr(), self.rows, self.k)
 
+    def check(self, name: str, device) -> "MXFP4":
+        """Both buffers on `device` and large enough for rows x k (before any launch)."""
+        _need_bytes(self.codes, f"{name}.codes", bat_mxfp4_codes_bytes(self.rows, self.k), device)
+        _need_bytes(self.scales, f"{name}.scales", bat_mxfp4_scales_bytes(self.rows, self.k), device)
+        return self
+
 
 @dataclass
 class MXFP8:
@@ -171,6 +200,11 @@ class MXFP8:
 
     def struct(self) -> MXFP4Struct:
         return MXFP4Struct(self.codes.data_ptr(), self.scales.data_ptr(), self.rows, self.k)
+
+    def check(self, name: str, device) -> "MXFP8":
+        _need_bytes(self.codes, f"{name}.codes", bat_mxfp8_codes_bytes(self.rows, self.k), device)
+        _need_bytes(self.scales, f"{name}.scales", bat_mxfp4_scales_bytes(self.rows, self.k), device)
+        return self
 
 
 # ---------------------------------------------------------------- C-ABI wrappers
@@ -196,21 +230,28 @@ def bat_version() -> int:
 
 
 def _act_args(X, A, B, g_lo, g_hi):
-    M, K = X.shape
     _need(X, torch.bfloat16, "X")
-    _need(A, torch.float32, "A", (8, 8))
-    _need(B, torch.float32, "B", (K // 32, 4, 4))
-    if (g_lo is None) != (g_hi is None):
-        raise ValueError("g_lo and g_hi must both be given or both be None")
-    if g_lo is not None:
-        _need(g_lo, torch.float32, "g_lo", (K // 32,))
-        _need(g_hi, torch.float32, "g_hi", (K // 32,))
+    M, K = X.shape
+    dev = X.device
+    _need(A, torch.float32, "A", (8, 8), dev)
+    _need(B, torch.float32, "B", (K // 32, 4, 4), dev)
+    _clip_args(g_lo, g_hi, K // 32, dev)
     return M, K
+
+
+def _clip_args(g_lo, g_hi, nb: int, dev, prefix: str = "g", rows=None):
+    if (g_lo is None) != (g_hi is None):
+        raise ValueError(f"{prefix}_lo and {prefix}_hi must both be given or both be None")
+    if g_lo is not None:
+        shape = (nb,) if rows is None else (rows, nb)
+        _need(g_lo, torch.float32, f"{prefix}_lo", shape, dev)
+        _need(g_hi, torch.float32, f"{prefix}_hi", shape, dev)
 
 
 def bat_quantize_act(X, A, B, g_lo=None, g_hi=None, Xq: Optional[MXFP4] = None, stream=None) -> MXFP4:
     M, K = _act_args(X, A, B, g_lo, g_hi)
-    Xq = MXFP4.empty(M, K, X.device) if Xq is None else Xq
+    Xq = (MXFP4.empty(M, K, X.device) if Xq is None else Xq).check("Xq", X.device)
+    _on_device(X.device, stream)
     st = Xq.struct()
     _check(lib().bat_quantize_act(_ptr(X), M, K, _ptr(A), _ptr(B), _ptr(g_lo), _ptr(g_hi),
                                   ctypes.byref(st), _stream(stream)), "bat_quantize_act")
@@ -220,9 +261,10 @@ def bat_quantize_act(X, A, B, g_lo=None, g_hi=None, Xq: Optional[MXFP4] = None, 
 def bat_quantize_act_trace(X, A, B, g_lo=None, g_hi=None, Xq: Optional[MXFP4] = None,
                            y_out: Optional[torch.Tensor] = None, stream=None):
     M, K = _act_args(X, A, B, g_lo, g_hi)
-    Xq = MXFP4.empty(M, K, X.device) if Xq is None else Xq
+    Xq = (MXFP4.empty(M, K, X.device) if Xq is None else Xq).check("Xq", X.device)
     y_out = torch.empty(M, K, dtype=torch.float32, device=X.device) if y_out is None else y_out
-    _need(y_out, torch.float32, "y_out", (M, K))
+    _need(y_out, torch.float32, "y_out", (M, K), X.device)
+    _on_device(X.device, stream)
     st = Xq.struct()
     _check(lib().bat_quantize_act_trace(_ptr(X), M, K, _ptr(A), _ptr(B), _ptr(g_lo), _ptr(g_hi),
                                         ctypes.byref(st), _ptr(y_out), _stream(stream)),
@@ -234,7 +276,13 @@ def bat_clip_ratios(g: Optional[torch.Tensor], n: Optional[int] = None, r=None, 
     if g is not None:
         _need(g, torch.float32, "g")
         n = g.numel()
-    r = torch.empty(n, dtype=torch.float32, device="cuda") if r is None else r
+    dev = g.device if g is not None else (r.device if isinstance(r, torch.Tensor) else
+                                          torch.device("cuda", torch.cuda.current_device()))
+    r = torch.empty(n, dtype=torch.float32, device=dev) if r is None else r
+    _need(r, torch.float32, "r", None, dev)
+    if r.numel() < n:
+        raise ValueError(f"r holds {r.numel()} values; {n} are needed")
+    _on_device(dev, stream)
     _check(lib().bat_clip_ratios(_ptr(g), n, _ptr(r), _stream(stream)), "bat_clip_ratios")
     return r
 
@@ -242,24 +290,24 @@ def bat_clip_ratios(g: Optional[torch.Tensor], n: Optional[int] = None, r=None, 
 def bat_e2m1_encode(v: torch.Tensor, codes=None, stream=None) -> torch.Tensor:
     _need(v, torch.float32, "v")
     codes = torch.empty(v.numel(), dtype=torch.uint8, device=v.device) if codes is None else codes
+    _need_bytes(codes, "codes", v.numel(), v.device)
+    _on_device(v.device, stream)
     _check(lib().bat_e2m1_encode(_ptr(v), v.numel(), _ptr(codes), _stream(stream)), "bat_e2m1_encode")
     return codes
 
 
 def bat_prepare_weight(W, A, B, gw_lo=None, gw_hi=None, Wq: Optional[MXFP4] = None,
                        wt_out: Optional[torch.Tensor] = None, stream=None) -> MXFP4:
-    N, K = W.shape
     _need(W, torch.bfloat16, "W")
-    _need(A, torch.float32, "A", (8, 8))
-    _need(B, torch.float32, "B", (K // 32, 4, 4))
-    if (gw_lo is None) != (gw_hi is None):
-        raise ValueError("gw_lo and gw_hi must both be given or both be None")
-    if gw_lo is not None:
-        _need(gw_lo, torch.float32, "gw_lo", (N, K // 32))
-        _need(gw_hi, torch.float32, "gw_hi", (N, K // 32))
+    N, K = W.shape
+    dev = W.device
+    _need(A, torch.float32, "A", (8, 8), dev)
+    _need(B, torch.float32, "B", (K // 32, 4, 4), dev)
+    _clip_args(gw_lo, gw_hi, K // 32, dev, "gw", rows=N)
     if wt_out is not None:
-        _need(wt_out, torch.float32, "wt_out", (N, K))
-    Wq = MXFP4.empty(N, K, W.device) if Wq is None else Wq
+        _need(wt_out, torch.float32, "wt_out", (N, K), dev)
+    Wq = (MXFP4.empty(N, K, dev) if Wq is None else Wq).check("Wq", dev)
+    _on_device(dev, stream)
     st = Wq.struct()
     _check(lib().bat_prepare_weight(_ptr(W), N, K, _ptr(A), _ptr(B), _ptr(gw_lo), _ptr(gw_hi),
                                     ctypes.byref(st), _ptr(wt_out), _stream(stream)),
@@ -267,28 +315,26 @@ def bat_prepare_weight(W, A, B, gw_lo=None, gw_hi=None, Wq: Optional[MXFP4] = No
     return Wq
 
 
-def _gpk_factors(A, B, K):
+def _gpk_factors(A, B, K, dev=None):
     s = A.shape[0] if isinstance(A, torch.Tensor) and A.dim() == 2 else 0
     t = 32 // s if s else 0
-    _need(A, torch.float32, "A", (s, s))
-    _need(B, torch.float32, "B", (K // 32, t, t))
+    _need(A, torch.float32, "A", (s, s), dev)
+    _need(B, torch.float32, "B", (K // 32, t, t), dev)
     return s
 
 
 def bat_quantize_act_gpk(X, A, B, g_lo=None, g_hi=None, Xq: Optional[MXFP4] = None,
                          y_out: Optional[torch.Tensor] = None, stream=None) -> MXFP4:
     """Activation side with an s x s shared factor A and (32/s) x (32/s) private B_b."""
-    M, K = X.shape
     _need(X, torch.bfloat16, "X")
-    s = _gpk_factors(A, B, K)
-    if (g_lo is None) != (g_hi is None):
-        raise ValueError("g_lo and g_hi must both be given or both be None")
-    if g_lo is not None:
-        _need(g_lo, torch.float32, "g_lo", (K // 32,))
-        _need(g_hi, torch.float32, "g_hi", (K // 32,))
+    M, K = X.shape
+    dev = X.device
+    s = _gpk_factors(A, B, K, dev)
+    _clip_args(g_lo, g_hi, K // 32, dev)
     if y_out is not None:
-        _need(y_out, torch.float32, "y_out", (M, K))
-    Xq = MXFP4.empty(M, K, X.device) if Xq is None else Xq
+        _need(y_out, torch.float32, "y_out", (M, K), dev)
+    Xq = (MXFP4.empty(M, K, dev) if Xq is None else Xq).check("Xq", dev)
+    _on_device(dev, stream)
     st = Xq.struct()
     _check(lib().bat_quantize_act_gpk(_ptr(X), M, K, _ptr(A), s, _ptr(B), _ptr(g_lo), _ptr(g_hi),
                                       ctypes.byref(st), _ptr(y_out), _stream(stream)),
@@ -299,17 +345,15 @@ def bat_quantize_act_gpk(X, A, B, g_lo=None, g_hi=None, Xq: Optional[MXFP4] = No
 def bat_prepare_weight_gpk(W, A, B, gw_lo=None, gw_hi=None, Wq: Optional[MXFP4] = None,
                            wt_out: Optional[torch.Tensor] = None, stream=None) -> MXFP4:
     """Weight side for the factor split of ``bat_quantize_act_gpk``."""
-    N, K = W.shape
     _need(W, torch.bfloat16, "W")
-    s = _gpk_factors(A, B, K)
-    if (gw_lo is None) != (gw_hi is None):
-        raise ValueError("gw_lo and gw_hi must both be given or both be None")
-    if gw_lo is not None:
-        _need(gw_lo, torch.float32, "gw_lo", (N, K // 32))
-        _need(gw_hi, torch.float32, "gw_hi", (N, K // 32))
+    N, K = W.shape
+    dev = W.device
+    s = _gpk_factors(A, B, K, dev)
+    _clip_args(gw_lo, gw_hi, K // 32, dev, "gw", rows=N)
     if wt_out is not None:
-        _need(wt_out, torch.float32, "wt_out", (N, K))
-    Wq = MXFP4.empty(N, K, W.device) if Wq is None else Wq
+        _need(wt_out, torch.float32, "wt_out", (N, K), dev)
+    Wq = (MXFP4.empty(N, K, dev) if Wq is None else Wq).check("Wq", dev)
+    _on_device(dev, stream)
     st = Wq.struct()
     _check(lib().bat_prepare_weight_gpk(_ptr(W), N, K, _ptr(A), s, _ptr(B), _ptr(gw_lo),
                                         _ptr(gw_hi), ctypes.byref(st), _ptr(wt_out),
@@ -338,8 +382,12 @@ def _out_code(out_dtype: torch.dtype) -> int:
 def bat_mxfp4_gemm(Xq: MXFP4, Wq: MXFP4, Y: Optional[torch.Tensor] = None,
                    out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
     code = _out_code(out_dtype)
-    Y = torch.empty(Xq.rows, Wq.rows, dtype=out_dtype, device=Xq.codes.device) if Y is None else Y
-    _need(Y, out_dtype, "Y", (Xq.rows, Wq.rows))
+    dev = Xq.codes.device
+    Xq.check("Xq", dev)
+    Wq.check("Wq", dev)
+    Y = torch.empty(Xq.rows, Wq.rows, dtype=out_dtype, device=dev) if Y is None else Y
+    _need(Y, out_dtype, "Y", (Xq.rows, Wq.rows), dev)
+    _on_device(dev, stream)
     a, b = Xq.struct(), Wq.struct()
     _check(lib().bat_mxfp4_gemm(ctypes.byref(a), ctypes.byref(b), _ptr(Y), code, _stream(stream)),
            "bat_mxfp4_gemm")
@@ -349,17 +397,15 @@ def bat_mxfp4_gemm(Xq: MXFP4, Wq: MXFP4, Y: Optional[torch.Tensor] = None,
 def bat_quantize_act_mxfp8(X, A, B, g_lo=None, g_hi=None, Xq: Optional[MXFP8] = None,
                            y_out: Optional[torch.Tensor] = None, stream=None) -> MXFP8:
     """W4A8 activation side: transform (any split of A, B), clip, MXFP8 (E4M3) quantize."""
-    M, K = X.shape
     _need(X, torch.bfloat16, "X")
-    s = _gpk_factors(A, B, K)
-    if (g_lo is None) != (g_hi is None):
-        raise ValueError("g_lo and g_hi must both be given or both be None")
-    if g_lo is not None:
-        _need(g_lo, torch.float32, "g_lo", (K // 32,))
-        _need(g_hi, torch.float32, "g_hi", (K // 32,))
+    M, K = X.shape
+    dev = X.device
+    s = _gpk_factors(A, B, K, dev)
+    _clip_args(g_lo, g_hi, K // 32, dev)
     if y_out is not None:
-        _need(y_out, torch.float32, "y_out", (M, K))
-    Xq = MXFP8.empty(M, K, X.device) if Xq is None else Xq
+        _need(y_out, torch.float32, "y_out", (M, K), dev)
+    Xq = (MXFP8.empty(M, K, dev) if Xq is None else Xq).check("Xq", dev)
+    _on_device(dev, stream)
     st = Xq.struct()
     _check(lib().bat_quantize_act_mxfp8(_ptr(X), M, K, _ptr(A), s, _ptr(B), _ptr(g_lo),
                                         _ptr(g_hi), ctypes.byref(st), _ptr(y_out),
@@ -370,6 +416,8 @@ def bat_quantize_act_mxfp8(X, A, B, g_lo=None, g_hi=None, Xq: Optional[MXFP8] = 
 def bat_e4m3_encode(v: torch.Tensor, codes=None, stream=None) -> torch.Tensor:
     _need(v, torch.float32, "v")
     codes = torch.empty(v.numel(), dtype=torch.uint8, device=v.device) if codes is None else codes
+    _need_bytes(codes, "codes", v.numel(), v.device)
+    _on_device(v.device, stream)
     _check(lib().bat_e4m3_encode(_ptr(v), v.numel(), _ptr(codes), _stream(stream)), "bat_e4m3_encode")
     return codes
 
@@ -377,8 +425,12 @@ def bat_e4m3_encode(v: torch.Tensor, codes=None, stream=None) -> torch.Tensor:
 def bat_w4a8_gemm(Xq: MXFP8, Wq: MXFP4, Y: Optional[torch.Tensor] = None,
                   out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
     code = _out_code(out_dtype)
-    Y = torch.empty(Xq.rows, Wq.rows, dtype=out_dtype, device=Xq.codes.device) if Y is None else Y
-    _need(Y, out_dtype, "Y", (Xq.rows, Wq.rows))
+    dev = Xq.codes.device
+    Xq.check("Xq", dev)
+    Wq.check("Wq", dev)
+    Y = torch.empty(Xq.rows, Wq.rows, dtype=out_dtype, device=dev) if Y is None else Y
+    _need(Y, out_dtype, "Y", (Xq.rows, Wq.rows), dev)
+    _on_device(dev, stream)
     a, b = Xq.struct(), Wq.struct()
     _check(lib().bat_w4a8_gemm(ctypes.byref(a), ctypes.byref(b), _ptr(Y), code, _stream(stream)),
            "bat_w4a8_gemm")
@@ -394,12 +446,17 @@ def bat_linear(X, Wq: MXFP4, A, B, g_lo=None, g_hi=None, Y: Optional[torch.Tenso
                stream=None) -> torch.Tensor:
     M, K = _act_args(X, A, B, g_lo, g_hi)
     code = _out_code(out_dtype)
-    Y = torch.empty(M, Wq.rows, dtype=out_dtype, device=X.device) if Y is None else Y
-    _need(Y, out_dtype, "Y", (M, Wq.rows))
+    dev = X.device
+    if Wq.k != K:
+        raise ValueError(f"Wq has k={Wq.k} but X has K={K}")
+    Wq.check("Wq", dev)
+    Y = torch.empty(M, Wq.rows, dtype=out_dtype, device=dev) if Y is None else Y
+    _need(Y, out_dtype, "Y", (M, Wq.rows), dev)
     need = bat_linear_workspace_bytes(M, K)
     if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
-    _need(workspace, torch.uint8, "workspace")
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _need(workspace, torch.uint8, "workspace", None, dev)
+    _on_device(dev, stream)
     b = Wq.struct()
     _check(lib().bat_linear(_ptr(X), M, ctypes.byref(b), _ptr(A), _ptr(B), _ptr(g_lo), _ptr(g_hi),
                             _ptr(Y), code, _ptr(workspace), workspace.numel(), _stream(stream)),
@@ -416,8 +473,13 @@ def bat_linear_noalloc(X, Wq: MXFP4, A, B, g_lo=None, g_hi=None, Y: Optional[tor
     the quantized activations (for callers that cannot allocate device memory)."""
     M, K = _act_args(X, A, B, g_lo, g_hi)
     code = _out_code(out_dtype)
-    Y = torch.empty(M, Wq.rows, dtype=out_dtype, device=X.device) if Y is None else Y
-    _need(Y, out_dtype, "Y", (M, Wq.rows))
+    dev = X.device
+    if Wq.k != K:
+        raise ValueError(f"Wq has k={Wq.k} but X has K={K}")
+    Wq.check("Wq", dev)
+    Y = torch.empty(M, Wq.rows, dtype=out_dtype, device=dev) if Y is None else Y
+    _need(Y, out_dtype, "Y", (M, Wq.rows), dev)
+    _on_device(dev, stream)
     b = Wq.struct()
     _check(lib().bat_linear_noalloc(_ptr(X), M, ctypes.byref(b), _ptr(A), _ptr(B), _ptr(g_lo),
                                     _ptr(g_hi), _ptr(Y), code, _stream(stream)),
@@ -454,23 +516,33 @@ class KVCache:
         return KVCache(torch.zeros(cb, dtype=torch.uint8, device=device),
                        torch.zeros(sb, dtype=torch.uint8, device=device), num_slots, H, D, fmt)
 
+    def check(self, device) -> "KVCache":
+        """Both buffers on `device` and large enough for num_slots x H x D (before any launch)."""
+        if self.fmt not in _KV_FMT:
+            raise ValueError(f"unknown KV format {self.fmt!r}")
+        f = _KV_FMT[self.fmt]
+        _need_bytes(self.codes, "cache.codes",
+                    lib().bat_kv_codes_bytes(self.num_slots, self.H, self.D, f), device)
+        _need_bytes(self.scales, "cache.scales",
+                    lib().bat_kv_scales_bytes(self.num_slots, self.H, self.D), device)
+        return self
+
 
 def bat_kv_quantize(kv, A, B, slots, cache: KVCache, g_lo=None, g_hi=None,
                     y_out: Optional[torch.Tensor] = None, stream=None) -> KVCache:
     """Transform, clip and quantize kv [T][H][D] (bf16) into cache rows slots[t] (-1 skips)."""
-    T, H, D = kv.shape
     _need(kv, torch.bfloat16, "kv")
-    s = _gpk_factors(A, B, D)
-    _need(slots, torch.int64, "slots", (T,))
-    if (g_lo is None) != (g_hi is None):
-        raise ValueError("g_lo and g_hi must both be given or both be None")
-    if g_lo is not None:
-        _need(g_lo, torch.float32, "g_lo", (D // 32,))
-        _need(g_hi, torch.float32, "g_hi", (D // 32,))
+    T, H, D = kv.shape
+    dev = kv.device
+    s = _gpk_factors(A, B, D, dev)
+    _need(slots, torch.int64, "slots", (T,), dev)
+    _clip_args(g_lo, g_hi, D // 32, dev)
     if y_out is not None:
-        _need(y_out, torch.float32, "y_out", (T, H, D))
+        _need(y_out, torch.float32, "y_out", (T, H, D), dev)
     if cache.H != H or cache.D != D:
         raise ValueError("cache shape does not match kv")
+    cache.check(dev)
+    _on_device(dev, stream)
     _check(lib().bat_kv_quantize(_ptr(kv), T, H, D, _ptr(A), s, _ptr(B), _ptr(g_lo), _ptr(g_hi),
                                  _ptr(slots), _KV_FMT[cache.fmt], _ptr(cache.codes),
                                  _ptr(cache.scales), cache.num_slots, _ptr(y_out),
@@ -481,14 +553,19 @@ def bat_kv_quantize(kv, A, B, slots, cache: KVCache, g_lo=None, g_hi=None,
 def bat_kv_dequantize(cache: KVCache, slots, A=None, B=None, out: Optional[torch.Tensor] = None,
                       out_dtype: torch.dtype = torch.float32, stream=None) -> torch.Tensor:
     """Values of cache rows slots[t] as [T][H][D]; with A, B also multiplied by B_b (x) A."""
+    dev = cache.codes.device
+    cache.check(dev)
+    _need(slots, torch.int64, "slots", None, dev)
+    if slots.dim() != 1:
+        raise ValueError("slots must be one-dimensional")
     T = slots.shape[0]
-    _need(slots, torch.int64, "slots", (T,))
     s = 8
     if A is not None:
-        s = _gpk_factors(A, B, cache.D)
+        s = _gpk_factors(A, B, cache.D, dev)
     code = _out_code(out_dtype)
-    out = torch.empty(T, cache.H, cache.D, dtype=out_dtype, device=cache.codes.device) if out is None else out
-    _need(out, out_dtype, "out", (T, cache.H, cache.D))
+    out = torch.empty(T, cache.H, cache.D, dtype=out_dtype, device=dev) if out is None else out
+    _need(out, out_dtype, "out", (T, cache.H, cache.D), dev)
+    _on_device(dev, stream)
     _check(lib().bat_kv_dequantize(_ptr(cache.codes), _ptr(cache.scales), cache.num_slots, cache.H,
                                    cache.D, _KV_FMT[cache.fmt], _ptr(slots), T, _ptr(A), s, _ptr(B),
                                    _ptr(out), code, _stream(stream)), "bat_kv_dequantize")
