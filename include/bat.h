@@ -102,7 +102,8 @@ typedef bat_mxfp4_t bat_mxfp8_t;
 BAT_API size_t bat_mxfp4_codes_bytes(int64_t rows, int64_t k);
 BAT_API size_t bat_mxfp4_scales_bytes(int64_t rows, int64_t k);
 
-/* Human-readable name of a status code (static storage). */
+/* Human-readable name of a status code (static storage; "BAT_ERR_UNKNOWN" for a
+ * value that is not a status). */
 BAT_API const char* bat_status_string(bat_status_t status);
 
 /* Library version, major*10000 + minor*100 + patch. */
@@ -121,6 +122,11 @@ BAT_API int bat_version(void);
  *                g = +inf gives ratio 1.
  *   Xq    : output; Xq->rows must equal M and Xq->k must equal K.
  * Requirements: 1 <= M <= 2^30, K >= 32, K % 32 == 0, K <= 262144.
+ * Errors: BAT_ERR_INVALID_ARG (a NULL pointer, only one of g_lo/g_hi, M < 1 or
+ * K < 32), BAT_ERR_SHAPE (K % 32, K or M over its limit, Xq's rows/k not M/K),
+ * BAT_ERR_ALIGN (X, A, B, Xq->codes or Xq->scales not 16-byte aligned),
+ * BAT_ERR_UNSUPPORTED (not an sm_100 device), BAT_ERR_CUDA (launch failure);
+ * nothing is launched on an argument error.
  */
 BAT_API bat_status_t bat_quantize_act(const void* X, int64_t M, int64_t K, const float* A, const float* B,
                               const float* g_lo, const float* g_hi, const bat_mxfp4_t* Xq,
@@ -130,6 +136,8 @@ BAT_API bat_status_t bat_quantize_act(const void* X, int64_t M, int64_t K, const
  * Same as bat_quantize_act, and also writes the fp32 transformed values y
  * (before clipping) to `y_out` (device fp32 [M][K]). For testing and
  * inspection; slower because of the extra 4 bytes per element.
+ * Errors: as bat_quantize_act; also BAT_ERR_INVALID_ARG for a NULL y_out and
+ * BAT_ERR_ALIGN for a y_out that is not 16-byte aligned.
  */
 BAT_API bat_status_t bat_quantize_act_trace(const void* X, int64_t M, int64_t K, const float* A,
                                     const float* B, const float* g_lo, const float* g_hi,
@@ -139,6 +147,8 @@ BAT_API bat_status_t bat_quantize_act_trace(const void* X, int64_t M, int64_t K,
  * The clip ratios the prologue uses: r[t] = fp32(1 / (1 + exp(-g[t]))) computed
  * in fp64 on the device (g = +inf gives 1; g == NULL gives all ones).
  * g, r: device fp32 [n].
+ * Errors: BAT_ERR_INVALID_ARG (n < 1 or r NULL), BAT_ERR_UNSUPPORTED,
+ * BAT_ERR_CUDA.
  */
 BAT_API bat_status_t bat_clip_ratios(const float* g, int64_t n, float* r, void* stream);
 
@@ -147,6 +157,8 @@ BAT_API bat_status_t bat_clip_ratios(const float* g, int64_t n, float* r, void* 
  * v[t] (round-to-nearest-even, saturating at +-6, sign in bit 3), one code per
  * byte. Values are converted in pairs (2t, 2t+1) exactly as the prologue packs
  * them. v: device fp32 [n]; codes: device uint8 [n].
+ * Errors: BAT_ERR_INVALID_ARG (n < 1 or a NULL pointer), BAT_ERR_UNSUPPORTED,
+ * BAT_ERR_CUDA.
  */
 BAT_API bat_status_t bat_e2m1_encode(const float* v, int64_t n, uint8_t* codes, void* stream);
 
@@ -230,6 +242,8 @@ BAT_API bat_status_t bat_quantize_act_mxfp8(const void* X, int64_t M, int64_t K,
  * E4M3 element conversion exactly as the MXFP8 prologue performs it (values
  * converted in groups of four, round to nearest even, saturating at +-448).
  * v: device fp32 [n]; codes: device uint8 [n].
+ * Errors: BAT_ERR_INVALID_ARG (n < 1 or a NULL pointer), BAT_ERR_UNSUPPORTED,
+ * BAT_ERR_CUDA.
  */
 BAT_API bat_status_t bat_e4m3_encode(const float* v, int64_t n, uint8_t* codes, void* stream);
 
@@ -307,11 +321,16 @@ BAT_API bat_status_t bat_kv_dequantize(const void* cache_codes, const void* cach
  *
  *   Xq : M x K MXFP4 activations; Wq : N x K MXFP4 weights (Xq->k == Wq->k).
  *   Y  : device [M][N] row-major, bf16 or fp32 per `out_dtype`, 16-byte aligned.
+ * Errors: BAT_ERR_INVALID_ARG (a NULL pointer, an unknown out_dtype, rows < 1 or
+ * k < 32), BAT_ERR_SHAPE (Xq->k != Wq->k, k % 32, k or rows over their limits),
+ * BAT_ERR_ALIGN (codes, scales or Y not 16-byte aligned), BAT_ERR_UNSUPPORTED,
+ * BAT_ERR_CUDA; nothing is launched on an argument error.
  */
 BAT_API bat_status_t bat_mxfp4_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
                             bat_out_dtype_t out_dtype, void* stream);
 
-/* Workspace bytes bat_linear needs for M rows of K inputs (the quantized X). */
+/* Workspace bytes bat_linear needs for M rows of K inputs (the quantized X); 0 for
+ * an invalid shape. */
 BAT_API size_t bat_linear_workspace_bytes(int64_t M, int64_t K);
 
 /*
@@ -320,6 +339,9 @@ BAT_API size_t bat_linear_workspace_bytes(int64_t M, int64_t K);
  *   X  : bf16 [M][K]; Wq from bat_prepare_weight (Wq->k == K); A, B, g_lo, g_hi
  *        as in bat_quantize_act; Y: [M][Wq->rows] in `out_dtype`.
  *   workspace : device, >= bat_linear_workspace_bytes(M, K) bytes, 256-byte aligned.
+ * Errors: those of bat_quantize_act and bat_mxfp4_gemm, and BAT_ERR_WORKSPACE
+ * (workspace NULL or smaller than needed) or BAT_ERR_ALIGN (workspace not
+ * 256-byte aligned).
  */
 BAT_API bat_status_t bat_linear(const void* X, int64_t M, const bat_mxfp4_t* Wq, const float* A,
                         const float* B, const float* g_lo, const float* g_hi, void* Y,
