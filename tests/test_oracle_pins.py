@@ -276,6 +276,47 @@ def test_clip_properties():
     assert lo[0, 0] <= blk[0, 0].min() and hi[1, 1] >= blk[1, 1].max()
 
 
+def test_weight_clip_per_row_and_block():
+    """Weight clip (the note, Key Designs 3: weights receive the analogous treatment):
+    one logit pair per (output row, block), written independently here with scipy's
+    logistic, a numpy clamp and the separately written RTN quantizer."""
+    inp = wl.make_inputs("tiny")
+    N, K = inp.W.shape
+    nb = K // 32
+    assert N != nb  # a transposed [block][row] index cannot line up by accident
+    rng = np.random.default_rng(31)
+    gw_lo = rng.uniform(-1.0, 3.0, size=(N, nb)).astype(np.float32)
+    gw_hi = rng.uniform(-1.0, 3.0, size=(N, nb)).astype(np.float32)
+    Wt, codes, scales = oracle.prepare_weight(inp.W, inp.A, inp.B, gw_lo, gw_hi)
+    # the transformed weights themselves are unclipped (pinned by inverse fusion)
+    assert np.array_equal(Wt, oracle.weight_transform_f64(inp.W, inp.A, inp.B).astype(np.float32))
+
+    def rtn_with(r_lo, r_hi):
+        blk = Wt.reshape(N, nb, 32)
+        lo = (r_lo * blk.min(axis=2)).astype(np.float32)
+        hi = (r_hi * blk.max(axis=2)).astype(np.float32)
+        c = np.minimum(np.maximum(blk, lo[..., None]), hi[..., None])
+        return _rtn_mxfp4(c.reshape(N, K))
+
+    r_lo = scipy.special.expit(gw_lo.astype(np.float64)).astype(np.float32)
+    r_hi = scipy.special.expit(gw_hi.astype(np.float64)).astype(np.float32)
+    rc, rs = rtn_with(r_lo, r_hi)
+    assert np.array_equal(codes, rc) and np.array_equal(scales, rs)
+    # the quantizer's per-row branch alone, fed the same ratios
+    qc, qs, bad = oracle.quantize(Wt, r_lo, r_hi, per_row=True)
+    assert bad == 0 and np.array_equal(qc, rc) and np.array_equal(qs, rs)
+    # controls: the plausible index mistakes give other codes, so this test would see them
+    flat_lo, flat_hi = r_lo.reshape(-1), r_hi.reshape(-1)
+    transposed = rtn_with(flat_lo.reshape(nb, N).T, flat_hi.reshape(nb, N).T)  # b * N + m
+    shared = rtn_with(np.broadcast_to(flat_lo[:nb], (N, nb)), np.broadcast_to(flat_hi[:nb], (N, nb)))
+    for wc, ws in (transposed, shared):
+        assert not (np.array_equal(wc, codes) and np.array_equal(ws, scales))
+    # the clip is active: most (row, block) pairs change against the unclipped weights
+    _, uc, _ = oracle.prepare_weight(inp.W, inp.A, inp.B)
+    changed = np.any((uc != codes).reshape(N, nb, 32), axis=2)
+    assert changed.mean() > 0.5
+
+
 def test_sigmoid_ratios():
     g = np.array([0.0, 1.0, 2.5, 4.0, -3.0, 30.0], np.float32)
     r = oracle.clip_ratios(g)
