@@ -6,6 +6,9 @@ GEMM against weights prepared offline. Prints one JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
+The headline workload defaults to prefill_o, the largest; on one GPU the line also
+carries `per_config`, the same figures for the other workloads.
+
 Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of the
 same layer (replicated weights, independent token batches, no collective on the
 data path) -> weak scaling; time = max over ranks.
@@ -154,10 +157,12 @@ class ClockSampler:
             for n, v in zip(names, r[3][1:]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
-        loaded = [r for r in rows if r[2] > 200.0] or rows
+        under = [r for r in rows if r[2] > 200.0]
+        loaded = under or rows
         return {"sm_mhz": statistics.median(r[0] for r in loaded),
                 "sm_max_mhz": max(r[1] for r in rows), "reasons": sorted(reasons),
-                "samples": len(rows), "power_w_max": max(r[2] for r in rows)}
+                "samples": len(rows), "samples_under_load": len(under),
+                "power_w_max": max(r[2] for r in rows)}
 
 
 # ---------------------------------------------------------------- CPU oracle leg
@@ -448,19 +453,295 @@ def run_reference_kv(args):
 
 
 # ---------------------------------------------------------------- GPU leg
+PER_CONFIG_ORDER = ("mlp_gate_up", "mlp_down", "decode_qkv", "prefill_o")
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def oracle_prologue_rate(inp, w, budget_s: float, threads: int, seed: int = 5):
+    """The oracle's activation side (transform + clip + MXFP4 quantize) on random token
+    rows for about `budget_s` seconds with `threads` OpenMP threads; GB/s at the
+    prologue's algorithmic 2.531 bytes per element."""
+    import oracle
+    prev = oracle.num_threads()
+    oracle.set_num_threads(threads)
+    try:
+        rng = np.random.default_rng(seed)
+        per = max(1, min(w.M, 8 * threads))
+        oracle.quantize_act(inp.X[:1], inp.A, inp.B, inp.g_lo, inp.g_hi)  # page in
+        n, dt = 0, 0.0
+        while dt < budget_s and n < 64 * w.M:
+            rows = rng.choice(w.M, size=per, replace=False)
+            t0 = time.perf_counter()
+            oracle.quantize_act(inp.X[rows], inp.A, inp.B, inp.g_lo, inp.g_hi)
+            dt += time.perf_counter() - t0
+            n += per
+        gbs = PROLOGUE_BYTES_PER_ELT * n * w.K / dt / 1e9
+        return {"value": gbs, "unit": "GB/s", "cores": threads, "seconds": round(dt, 2),
+                "sample": f"{n} random token rows of {w.name} (K={w.K}) in batches of {per}"}
+    finally:
+        oracle.set_num_threads(prev)
+
+
+class LinearBench:
+    """One workload of the linear layer on one GPU (and its rank's token batch)."""
+
+    def __init__(self, args, name, rank, dev, stream, pg):
+        import torch
+        import w4a4_bit_gemm_b200 as bat
+        self.torch, self.bat, self.args, self.dev, self.stream, self.pg = torch, bat, args, dev, stream, pg
+        self.w = w = wl.WORKLOADS[name]
+        inp, X_host = rank_inputs(name, rank)
+        self.inp, self.X_host = inp, X_host
+
+        def bf16(bits):
+            return torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(dev)
+
+        def f32(a):
+            return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev)
+
+        self.X = bf16(X_host)
+        self.gl, self.gh = f32(inp.g_lo), f32(inp.g_hi)
+        self.a8 = a8 = args.act == "mxfp8"
+        gl, gh = self.gl, self.gh
+        if args.shared != 8:  # another split: factors of the standard recipe at that size
+            inp.A, inp.B, _, _ = wl.random_factors(w.K // 32, seed=1, shared=args.shared)
+        self.A, self.B = A, B = f32(inp.A), f32(inp.B)
+        if a8:
+            self.quantize = lambda Xin, out, s=stream: bat.bat_quantize_act_mxfp8(
+                Xin, A, B, gl, gh, Xq=out, stream=s)
+            prepare = lambda Win: bat.bat_prepare_weight_gpk(Win, A, B)
+        elif args.shared == 8:
+            self.quantize = lambda Xin, out, s=stream: bat.bat_quantize_act(
+                Xin, A, B, gl, gh, Xq=out, stream=s)
+            prepare = lambda Win: bat.bat_prepare_weight(Win, A, B)
+        else:
+            self.quantize = lambda Xin, out, s=stream: bat.bat_quantize_act_gpk(
+                Xin, A, B, gl, gh, Xq=out, stream=s)
+            prepare = lambda Win: bat.bat_prepare_weight_gpk(Win, A, B)
+        Wdev = bf16(inp.W)
+        prepare(Wdev)  # first call: module load, attributes
+        torch.cuda.synchronize()
+        wp0, wp1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        wp0.record()
+        self.Wq = prepare(Wdev)  # offline weight side, timed for information only
+        wp1.record()
+        torch.cuda.synchronize()
+        self.prep_ms = wp0.elapsed_time(wp1)
+        del Wdev
+        self.Xq = (bat.MXFP8 if a8 else bat.MXFP4).empty(w.M, w.K, dev)
+        self.Y = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)
+        self.gemm_fn = bat.bat_w4a8_gemm if a8 else bat.bat_mxfp4_gemm
+        # W4A4 with the default factor split: the step is the public bat_linear (the
+        # quantizer and the GEMM on one stream); otherwise the two calls directly
+        self.use_linear = not a8 and args.shared == 8
+        self.ws = torch.empty(bat.bat_linear_workspace_bytes(w.M, w.K), dtype=torch.uint8, device=dev)
+        self.flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.flush_view = self.flush.view(torch.int32)
+        self.launches_per_step = 2
+
+    def step(self):
+        if self.use_linear:
+            self.bat.bat_linear(self.X, self.Wq, self.A, self.B, self.gl, self.gh, Y=self.Y,
+                                out_dtype=self.torch.bfloat16, workspace=self.ws, stream=self.stream)
+        else:
+            self.quantize(self.X, self.Xq)
+            self.gemm_fn(self.Xq, self.Wq, Y=self.Y, out_dtype=self.torch.bfloat16, stream=self.stream)
+
+    def flush_l2(self, i):
+        # write, then read, a buffer twice the L2: the next kernel starts with a cold L2
+        # holding only clean lines of unrelated data (no write-back lands on it)
+        self.flush.fill_(i & 0xFF)
+        self.flush_view.amax()
+
+    def timed_pass(self, K_):
+        """K_ steps, an L2 flush before each (outside the events), one event pair per step
+        around the step's kernels. Nothing sits between the two kernels on the stream, so
+        the GEMM (programmatic stream serialization) sets up while the quantizer finishes.
+        Returns the sum of the step times (s)."""
+        torch = self.torch
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_)]
+        if self.pg:
+            self.pg.barrier()
+        torch.cuda.synchronize()
+        for i in range(K_):
+            self.flush_l2(i)
+            ev[i][0].record(self.stream)
+            self.step()
+            ev[i][1].record(self.stream)
+        torch.cuda.synchronize()
+        if self.pg:
+            self.pg.barrier()
+        return sum(e0.elapsed_time(e1) * 1e-3 for e0, e1 in ev)
+
+    def kernel_pass(self, K_):
+        """The same steps with an event between the two kernels (which also keeps them
+        from overlapping): per-launch durations of the quantizer and the GEMM (s)."""
+        torch = self.torch
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K_)]
+        torch.cuda.synchronize()
+        for i in range(K_):
+            self.flush_l2(i)
+            ev[i][0].record(self.stream)
+            self.quantize(self.X, self.Xq)
+            ev[i][1].record(self.stream)
+            self.gemm_fn(self.Xq, self.Wq, Y=self.Y, out_dtype=torch.bfloat16, stream=self.stream)
+            ev[i][2].record(self.stream)
+        torch.cuda.synchronize()
+        return ([e[0].elapsed_time(e[1]) * 1e-3 for e in ev],
+                [e[1].elapsed_time(e[2]) * 1e-3 for e in ev])
+
+    def run(self, steps, warmup, min_timed_s, sampler=None):
+        """Warm-up, then timed passes of exactly `steps` steps until at least
+        `min_timed_s` of timed GPU work has accumulated (so the clock record covers the
+        load); the headline is the median pass, the max over ranks."""
+        torch = self.torch
+        for i in range(warmup):
+            self.flush_l2(i)
+            self.step()
+        torch.cuda.synchronize()
+        if sampler is not None:
+            sampler.start()
+        first = max_over_ranks(self.pg, [self.timed_pass(steps)], self.dev)[0]
+        passes = int(min(400, max(1, np.ceil(min_timed_s / max(first, 1e-9)))))
+        times = [first] + [self.timed_pass(steps) for _ in range(passes - 1)]
+        clocks = sampler.stop() if sampler is not None else None
+        med = float(np.median(times))
+        t_step = max_over_ranks(self.pg, [med], self.dev)[0]
+        # per-kernel durations: passes of the same steps until about a quarter of that time
+        tp, tg = [], []
+        while True:
+            a, b = self.kernel_pass(steps)
+            tp += a
+            tg += b
+            if sum(tp) + sum(tg) >= 0.25 * min_timed_s or len(tp) >= 400 * steps:
+                break
+        mp, mg = max_over_ranks(self.pg, [float(np.mean(tp)), float(np.mean(tg))], self.dev)
+        assert self.bat.bat_device_error() == 0, "a kernel reported a stalled wait"
+        return {"t_pass": t_step, "passes": passes, "timed_s": float(sum(times)),
+                "pro_s": mp, "gemm_s": mg, "clocks": clocks}
+
+    def summary(self, r, steps, world):
+        """Figures of one measured workload (throughput of the whole job)."""
+        w = self.w
+        flop = 2.0 * w.M * w.N * w.K
+        peaks, peak_src = load_peaks()
+        ratio = FP8_OVER_BF16 if self.a8 else FP4_OVER_BF16
+        tc_peak = peaks["bf16_tflops"] * ratio
+        step_s = r["t_pass"] / steps
+        value = job_throughput(flop, steps, world, r["t_pass"]) / 1e12
+        gemm_tf = flop / r["gemm_s"] / 1e12
+        pro_bytes = (PROLOGUE8_BYTES_PER_ELT if self.a8 else PROLOGUE_BYTES_PER_ELT) * w.M * w.K
+        pro_gbs = pro_bytes / r["pro_s"] / 1e9
+        d = {"workload": w.name, "M": w.M, "N": w.N, "K": w.K,
+             "step_us": 1e6 * step_s, "linear_tflops": value / world,
+             "linear_frac": value / world / tc_peak,
+             "gemm_us": 1e6 * r["gemm_s"], "gemm_tflops": gemm_tf, "gemm_frac": gemm_tf / tc_peak,
+             "prologue_us": 1e6 * r["pro_s"], "prologue_gbs": pro_gbs,
+             "prologue_frac": pro_gbs / peaks["hbm_gbs"], "passes": r["passes"],
+             "timed_s": round(r["timed_s"], 3)}
+        if w.M <= 64:  # decode: memory-bound on the weight stream
+            wbytes = w.N * w.K / 2 + w.N * ((w.K // 32 + 3) // 4) * 4
+            d["gemm_weight_stream_gbs"] = wbytes / r["gemm_s"] / 1e9
+            d["gemm_weight_stream_frac"] = d["gemm_weight_stream_gbs"] / peaks["hbm_gbs"]
+        c = r.get("clocks")
+        if c:
+            d["clocks"] = c
+            if c.get("sm_mhz"):
+                d["step_us_x_sm_ghz"] = 1e6 * step_s * c["sm_mhz"] / 1e3
+        return d, value, gemm_tf, tc_peak, pro_gbs, peaks, peak_src, ratio
+
+    def e2e(self, world, e2e_steps):
+        """End to end through the public API: pinned host X -> device, linear, Y -> pinned
+        host. Two lanes (streams, each with its own buffers) take alternate steps, so one
+        step's host copies overlap the other's kernels and copies in the other direction,
+        as a serving loop would run them; every step still copies its X in from pinned
+        host memory and its Y out."""
+        torch, bat, w, args = self.torch, self.bat, self.w, self.args
+        Xh = torch.from_numpy(self.X_host.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+        lanes = []
+        for _ in range(2):
+            lanes.append({
+                "stream": torch.cuda.Stream(self.dev),
+                "Xdev": torch.empty_like(self.X),
+                "Y": torch.empty(w.M, w.N, dtype=torch.bfloat16, device=self.dev),
+                "Yh": torch.empty(w.M, w.N, dtype=torch.bfloat16).pin_memory(),
+                "ws": torch.empty(bat.bat_linear_workspace_bytes(w.M, w.K), dtype=torch.uint8,
+                                  device=self.dev),
+                "Xq": (bat.MXFP8 if self.a8 else bat.MXFP4).empty(w.M, w.K, self.dev),
+            })
+
+        def e2e_step(i):
+            ln = lanes[i % 2]
+            ls = ln["stream"]
+            with torch.cuda.stream(ls):
+                ln["Xdev"].copy_(Xh, non_blocking=True)
+                if self.use_linear:
+                    bat.bat_linear(ln["Xdev"], self.Wq, self.A, self.B, self.gl, self.gh, Y=ln["Y"],
+                                   out_dtype=torch.bfloat16, workspace=ln["ws"], stream=ls)
+                else:
+                    self.quantize(ln["Xdev"], ln["Xq"], ls)
+                    self.gemm_fn(ln["Xq"], self.Wq, Y=ln["Y"], out_dtype=torch.bfloat16, stream=ls)
+                ln["Yh"].copy_(ln["Y"], non_blocking=True)
+
+        for i in range(4):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        if self.pg:
+            self.pg.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        for ln in lanes:
+            ln["stream"].wait_event(e0)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        for ln in lanes:
+            done = torch.cuda.Event()
+            done.record(ln["stream"])
+            self.stream.wait_event(done)
+        e1.record(self.stream)
+        torch.cuda.synchronize()
+        te = max_over_ranks(self.pg, [e0.elapsed_time(e1) * 1e-3], self.dev)[0]
+        flop = 2.0 * w.M * w.N * w.K
+        return {"value": job_throughput(flop, e2e_steps, world, te) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(self.X.numel() * 2),
+                "d2h_bytes_per_step": int(self.Y.numel() * 2)}
+
+    def release(self):
+        for k in ("X", "Wq", "Xq", "Y", "ws", "flush", "flush_view"):
+            setattr(self, k, None)
+        self.torch.cuda.synchronize()
+        self.torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="mlp_gate_up", choices=wl.ORDER)
+    ap.add_argument("--workload", default="prefill_o", choices=wl.ORDER,
+                    help="headline workload (default: the largest, prefill_o)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--cpu-budget-s", type=float, default=8.0)
     ap.add_argument("--ref-budget-s", type=float, default=90.0)
+    ap.add_argument("--min-timed-s", type=float, default=0.5,
+                    help="repeat timed passes of --steps steps until this much timed GPU work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="measure only the headline workload")
     ap.add_argument("--shared", type=int, default=8, choices=[1, 2, 4, 8, 16, 32],
                     help="size s of the shared transform factor (A s x s, each B_b 32/s x 32/s)")
     ap.add_argument("--act", default="mxfp4", choices=["mxfp4", "mxfp8"],
@@ -500,228 +781,82 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
         pg = dist
+    stream = torch.cuda.current_stream(dev)
+    K_ = args.steps
 
     # rank r draws its own token batch; weights and transform factors are shared
-    inp, X_host = rank_inputs(w.name, rank)
+    lb = LinearBench(args, w.name, rank, dev, stream, pg)
+    sampler = ClockSampler(local) if (not args.no_clocks and rank == 0) else None
+    r = lb.run(K_, args.warmup, args.min_timed_s, sampler)
+    head, value, gemm_tf, tc_peak, pro_gbs, peaks, peak_src, ratio = lb.summary(r, K_, world)
+    e2e = None if args.no_e2e else lb.e2e(world, args.e2e_steps)
+    inp, a8 = lb.inp, lb.a8
+    prep_ms = lb.prep_ms
+    lb.release()
 
-    def bf16(bits):
-        return torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(dev)
-
-    def f32(a):
-        return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev)
-
-    X = bf16(X_host)
-    gl, gh = f32(inp.g_lo), f32(inp.g_hi)
-    stream = torch.cuda.current_stream(dev)
-    a8 = args.act == "mxfp8"
-    if a8:
-        # W4A8: MXFP8 activations through the E4M3 quantizer, MXFP4 weights
-        if args.shared != 8:
-            inp.A, inp.B, _, _ = wl.random_factors(w.K // 32, seed=1, shared=args.shared)
-        A, B = f32(inp.A), f32(inp.B)
-
-        def quantize(Xin, out):
-            bat.bat_quantize_act_mxfp8(Xin, A, B, gl, gh, Xq=out, stream=stream)
-
-        def prepare(Win):
-            return bat.bat_prepare_weight_gpk(Win, A, B)
-    elif args.shared == 8:
-        A, B = f32(inp.A), f32(inp.B)
-
-        def quantize(Xin, out):
-            bat.bat_quantize_act(Xin, A, B, gl, gh, Xq=out, stream=stream)
-
-        def prepare(Win):
-            return bat.bat_prepare_weight(Win, A, B)
-    else:
-        # another split of the 32 channels: factors of the standard recipe at that size
-        inp.A, inp.B, _, _ = wl.random_factors(w.K // 32, seed=1, shared=args.shared)
-        A, B = f32(inp.A), f32(inp.B)
-
-        def quantize(Xin, out):
-            bat.bat_quantize_act_gpk(Xin, A, B, gl, gh, Xq=out, stream=stream)
-
-        def prepare(Win):
-            return bat.bat_prepare_weight_gpk(Win, A, B)
-    Wdev = bf16(inp.W)
-    prepare(Wdev)  # first call: module load, attributes
-    torch.cuda.synchronize()
-    wp0, wp1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    wp0.record()
-    Wq = prepare(Wdev)  # offline weight side, timed for information only
-    wp1.record()
-    torch.cuda.synchronize()
-    prep_ms = wp0.elapsed_time(wp1)
-    del Wdev
-    Xq = (bat.MXFP8 if a8 else bat.MXFP4).empty(w.M, w.K, dev)
-    Y = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    gemm_fn = bat.bat_w4a8_gemm if a8 else bat.bat_mxfp4_gemm
-    # W4A4 with the default factor split: the step is the public bat_linear (the
-    # quantizer and the GEMM on one stream); otherwise the two calls directly
-    use_linear = not a8 and args.shared == 8
-    ws_step = torch.empty(bat.bat_linear_workspace_bytes(w.M, w.K), dtype=torch.uint8, device=dev)
-    launches_per_step = 2
-
-    def step():
-        if use_linear:
-            bat.bat_linear(X, Wq, A, B, gl, gh, Y=Y, out_dtype=torch.bfloat16, workspace=ws_step,
-                           stream=stream)
-        else:
-            quantize(X, Xq)
-            gemm_fn(Xq, Wq, Y=Y, out_dtype=torch.bfloat16, stream=stream)
-
-    def flush_l2(i):
-        # write, then read, a buffer twice the L2: the next kernel starts with a cold L2
-        # holding only clean lines of unrelated data (no write-back lands on it)
-        flush.fill_(i & 0xFF)
-        flush_view.amax()
-
-    flush_view = flush.view(torch.int32)
-    for i in range(args.warmup):
-        flush_l2(i)
-        step()
-    torch.cuda.synchronize()
-
-    K_ = args.steps
-    # Pass 1 (the headline): one event pair per step around the step's kernels. Nothing
-    # sits between them on the stream, so the GEMM, launched with programmatic stream
-    # serialization, does its set-up while the quantizer finishes.
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_)]
-    sampler = ClockSampler(local)
-    if not args.no_clocks and rank == 0:
-        sampler.start()
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize()
-    for i in range(K_):
-        flush_l2(i)  # evict L2 between steps (outside the timed events)
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    if pg:
-        pg.barrier()
-    clocks = sampler.stop() if (not args.no_clocks and rank == 0) else None
-    t_steps = [ev[i][0].elapsed_time(ev[i][1]) * 1e-3 for i in range(K_)]
-    # Pass 2 (per-kernel durations for the roofline fields): the same steps with an
-    # event between the two kernels, which also keeps them from overlapping.
-    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K_)]
-    torch.cuda.synchronize()
-    for i in range(K_):
-        flush_l2(i)
-        ev2[i][0].record(stream)
-        quantize(X, Xq)
-        ev2[i][1].record(stream)
-        gemm_fn(Xq, Wq, Y=Y, out_dtype=torch.bfloat16, stream=stream)
-        ev2[i][2].record(stream)
-    torch.cuda.synchronize()
-    t_pro = [ev2[i][0].elapsed_time(ev2[i][1]) * 1e-3 for i in range(K_)]
-    t_gemm = [ev2[i][1].elapsed_time(ev2[i][2]) * 1e-3 for i in range(K_)]
-    t_step, sp, sg = max_over_ranks(pg, [sum(t_steps), sum(t_pro), sum(t_gemm)], dev)
-    assert bat.bat_device_error() == 0, "a kernel reported a stalled wait"
-
-    flop = 2.0 * w.M * w.N * w.K
-    value = job_throughput(flop, K_, world, t_step) / 1e12
-    peaks, peak_src = load_peaks()
-    ratio = FP8_OVER_BF16 if a8 else FP4_OVER_BF16
-    fp4_peak = peaks["bf16_tflops"] * ratio
-    gemm_tf = flop / (sg / K_) / 1e12
-    pro_bytes = (PROLOGUE8_BYTES_PER_ELT if a8 else PROLOGUE_BYTES_PER_ELT) * w.M * w.K
-    pro_gbs = pro_bytes / (sp / K_) / 1e9
-
-    # end to end through the public API: pinned host X -> device, linear, Y -> pinned host
-    e2e = None
-    if not args.no_e2e:
-        # Two lanes (streams, each with its own buffers) take alternate steps, so one
-        # step's host copies overlap the other's kernels and copies in the other
-        # direction, as a serving loop would run them; every step still copies its X
-        # in from pinned host memory and its Y out.
-        Xh = torch.from_numpy(X_host.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
-        lanes = []
-        for _ in range(2):
-            lanes.append({
-                "stream": torch.cuda.Stream(dev),
-                "Xdev": torch.empty_like(X),
-                "Y": torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev),
-                "Yh": torch.empty(w.M, w.N, dtype=torch.bfloat16).pin_memory(),
-                "ws": torch.empty(bat.bat_linear_workspace_bytes(w.M, w.K), dtype=torch.uint8,
-                                  device=dev),
-                "Xq": (bat.MXFP8 if a8 else bat.MXFP4).empty(w.M, w.K, dev),
-            })
-
-        def e2e_step(i):
-            ln = lanes[i % 2]
-            ls = ln["stream"]
-            with torch.cuda.stream(ls):
-                ln["Xdev"].copy_(Xh, non_blocking=True)
-                if args.shared == 8 and not a8:
-                    bat.bat_linear(ln["Xdev"], Wq, A, B, gl, gh, Y=ln["Y"], out_dtype=torch.bfloat16,
-                                   workspace=ln["ws"], stream=ls)
-                elif a8:
-                    bat.bat_quantize_act_mxfp8(ln["Xdev"], A, B, gl, gh, Xq=ln["Xq"], stream=ls)
-                    gemm_fn(ln["Xq"], Wq, Y=ln["Y"], out_dtype=torch.bfloat16, stream=ls)
-                else:
-                    bat.bat_quantize_act_gpk(ln["Xdev"], A, B, gl, gh, Xq=ln["Xq"], stream=ls)
-                    gemm_fn(ln["Xq"], Wq, Y=ln["Y"], out_dtype=torch.bfloat16, stream=ls)
-                ln["Yh"].copy_(ln["Y"], non_blocking=True)
-
-        for i in range(4):
-            e2e_step(i)
-        torch.cuda.synchronize()
-        if pg:
-            pg.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for ln in lanes:
-            ln["stream"].wait_event(e0)
-        for i in range(args.e2e_steps):
-            e2e_step(i)
-        for ln in lanes:
-            done = torch.cuda.Event()
-            done.record(ln["stream"])
-            stream.wait_event(done)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        te = max_over_ranks(pg, [e0.elapsed_time(e1) * 1e-3], dev)[0]
-        e2e = {"value": job_throughput(flop, args.e2e_steps, world, te) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": int(X.numel() * 2), "d2h_bytes_per_step": int(Y.numel() * 2)}
+    # the other workloads, measured the same way (one GPU, rank 0 only)
+    per_config = None
+    if world == 1 and not args.no_per_config:
+        per_config = {}
+        for name in PER_CONFIG_ORDER:
+            if name == w.name:
+                continue
+            o = LinearBench(args, name, rank, dev, stream, None)
+            s_o = ClockSampler(local) if not args.no_clocks else None
+            ro = o.run(K_, args.warmup, 0.25 * args.min_timed_s, s_o)
+            per_config[name] = o.summary(ro, K_, 1)[0]
+            o.release()
+            del o
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
         fl, dt, desc, thr = oracle_sample(inp, w, args.cpu_budget_s,
                                           act_fmt="e4m3" if a8 else "e2m1")
         cpu = {"value": fl / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
-               "sample": desc, "seconds": round(dt, 2)}
+               "sample": desc, "seconds": round(dt, 2), "cpu_model": cpu_model(),
+               "host_cpus": os.cpu_count()}
+        if not a8:
+            budget = max(1.0, 0.25 * args.cpu_budget_s)
+            cpu["prologue_1thread"] = oracle_prologue_rate(inp, w, budget, 1)
+            cpu["prologue_all_cores"] = oracle_prologue_rate(inp, w, budget, oracle.num_threads())
 
     gemm_kernel = "bat_mxf4_gemm_kernel<true> (W4A8)" if a8 else "bat_mxf4_gemm_kernel"
     pro_kernel = "bat_prologue_kernel<..., MXFP8>" if a8 else "bat_prologue_kernel"
+    clocks = r["clocks"]
     if rank == 0:
         line = {
             "metric": METRIC_W4A8 if a8 else METRIC, "value": value, "unit": "TFLOP/s",
-            "n_gpus": world, "steps": K_, "warmup": args.warmup, "ms_per_step": 1e3 * t_step / K_,
+            "n_gpus": world, "steps": K_, "warmup": args.warmup,
+            "ms_per_step": 1e3 * r["t_pass"] / K_,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "mxfp8 x mxfp4" if a8 else "mxfp4", "data": "synthetic",
             "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "out": "bf16",
                        "transform": f"GPK A {args.shared}x{args.shared} shared, "
                                     f"B_b {32 // args.shared}x{32 // args.shared} private",
                        "l2": "flushed between steps (256 MiB write + read outside the timed events)",
+                       "timing": f"median of {r['passes']} passes of {K_} steps "
+                                 f"({r['timed_s']:.3f} s of timed steps)",
                        "parallelism": f"replicas x{world} (independent token batches)"},
-            "gpu_launches": launches_per_step * K_ * world,  # timed pass: quantizer + GEMM
-            "roofline": {"bound": "tensor", "achieved": gemm_tf, "peak": fp4_peak,
-                         "unit": "TFLOP/s", "frac": gemm_tf / fp4_peak,
+            # timed passes: quantizer + GEMM per step
+            "gpu_launches": lb.launches_per_step * K_ * r["passes"] * world,
+            "roofline": {"bound": "tensor", "achieved": gemm_tf, "peak": tc_peak,
+                         "unit": "TFLOP/s", "frac": gemm_tf / tc_peak,
                          "traffic": recorded_traffic(gemm_kernel, w.name),
                          "kernel": gemm_kernel,
                          "peak_source": f"{peak_src} bf16 burst x {ratio:g} (nominal "
                                         f"{'FP8' if a8 else 'FP4'}/BF16)"},
             "prologue": {"bound": "hbm", "achieved": pro_gbs, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": pro_gbs / peaks["hbm_gbs"],
-                         "us_per_launch": 1e6 * sp / K_,
+                         "us_per_launch": head["prologue_us"],
                          "traffic": recorded_traffic(pro_kernel, w.name),
                          "kernel": pro_kernel, "peak_source": peak_src},
-            "gemm_us_per_launch": 1e6 * sg / K_,
+            "linear_frac": head["linear_frac"],
+            "gemm_us_per_launch": head["gemm_us"],
             "prepare_weight_ms": prep_ms,
             "clocks": clocks,
+            "step_us_x_sm_ghz": head.get("step_us_x_sm_ghz"),
+            "per_config": per_config,
             "e2e": e2e,
             "cpu_baseline": cpu,
         }

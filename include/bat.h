@@ -369,7 +369,10 @@ BAT_API bat_status_t bat_linear(const void* X, int64_t M, const bat_mxfp4_t* Wq,
  *     K = 12288); larger calls return BAT_ERR_WORKSPACE and launch nothing.
  *   - The first call on each device looks up the array's device address with
  *     that device current (cudaGetSymbolAddress) and caches it. Make that first
- *     call before any stream capture.
+ *     call before any stream capture. The cached address assumes the device's
+ *     primary context lives until the process exits: after cudaDeviceReset (or
+ *     anything else that destroys and recreates that context) the address is
+ *     stale, so do not call this entry point again in that process.
  *   - All calls share the one array, and it keeps the last call's contents.
  *     Every byte a call reads is written by that same call first, so nothing
  *     needs clearing. Calls that overlap on the GPU (other streams, other host

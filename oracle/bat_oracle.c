@@ -411,3 +411,13 @@ int orc_num_threads(void) {
   return 1;
 #endif
 }
+
+/* Set the thread count of the OpenMP loops (timing only: every output element is
+ * a serial sum, so the results do not depend on it). */
+void orc_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}

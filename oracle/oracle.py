@@ -53,6 +53,7 @@ def lib():
         L.orc_weight_transform_f64_gen.restype = ctypes.c_int
         L.orc_transform_vals_f64.argtypes = [P, I64, I64, P, ctypes.c_int, P, P]
         L.orc_num_threads.restype = ctypes.c_int
+        L.orc_set_num_threads.argtypes = [ctypes.c_int]
         L.orc_e4m3_encode_array.argtypes = [P, I64, P]
         L.orc_e4m3_value.argtypes = [ctypes.c_uint8]
         L.orc_e4m3_value.restype = ctypes.c_double
@@ -256,6 +257,11 @@ def gpk_param_counts(K: int, shared: int = 8, private: int = 4) -> dict:
 def num_threads() -> int:
     """Host threads the oracle's parallel loops use."""
     return int(lib().orc_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Thread count of the oracle's parallel loops (results do not depend on it)."""
+    lib().orc_set_num_threads(int(n))
 
 
 def transform_vals_f64(Xd: np.ndarray, A: np.ndarray, B: np.ndarray) -> np.ndarray:

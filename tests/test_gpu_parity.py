@@ -297,29 +297,37 @@ def test_block_hadamard_mode(bat):
     _gemm_check(bat, outs[2][0], Wq, M, N, K)
 
 # ---------------------------------------------------------------- GEMM
-def _gemm_check(bat, Xq, Wq, M, N, K, rows=None, cols=None):
-    xc, xs, _ = _host(Xq, M, K)
-    wc, ws, _ = _host(Wq, N, K)
-    Xd = oracle.dequantize(xc, xs)
-    Wd = oracle.dequantize(wc, ws)
-    Y32 = bat.bat_mxfp4_gemm(Xq, Wq, out_dtype=torch.float32)
-    Y16 = bat.bat_mxfp4_gemm(Xq, Wq, out_dtype=torch.bfloat16)
-    torch.cuda.synchronize()
-    ref = oracle.gemm_sampled(Xd, Wd, rows, cols)
-    r = np.arange(M) if rows is None else np.asarray(rows)
-    c = np.arange(N) if cols is None else np.asarray(cols)
-    y32 = Y32.cpu().numpy()[np.ix_(r, c)].astype(np.float64)
-    y16 = Y16.float().cpu().numpy()[np.ix_(r, c)].astype(np.float64)
+def _check_outputs(y32, y16, Xd, Wd):
+    """Sampled outputs against the oracle's fp64 product of the same dequantized
+    operands (Xd, Wd: the sampled rows and columns): relative Frobenius error, a
+    per-element bound far inside fp32 accumulation of the absolute terms, and the
+    bf16 output against the bf16-rounded product."""
+    ref = oracle.gemm_sampled(Xd, Wd)
     assert np.all(np.isfinite(y32))
     rel = np.linalg.norm(y32 - ref) / max(np.linalg.norm(ref), 1e-300)
     assert rel <= GEMM_TOL, rel
-    # each output's error is far inside fp32 accumulation of the absolute terms
-    mag = oracle.gemm_sampled(np.abs(Xd), np.abs(Wd), rows, cols)
+    mag = oracle.gemm_sampled(np.abs(Xd), np.abs(Wd))
     assert np.all(np.abs(y32 - ref) <= 1e-5 * mag + 1e-30), np.max(np.abs(y32 - ref) / (mag + 1e-30))
-    ref16 = torch.from_numpy(ref).to(torch.bfloat16).float().numpy().astype(np.float64)
-    rel16 = np.linalg.norm(y16 - ref16) / max(np.linalg.norm(ref16), 1e-300)
-    assert rel16 <= GEMM_TOL, rel16
+    if y16 is not None:
+        ref16 = torch.from_numpy(ref).to(torch.bfloat16).float().numpy().astype(np.float64)
+        rel16 = np.linalg.norm(y16 - ref16) / max(np.linalg.norm(ref16), 1e-300)
+        assert rel16 <= GEMM_TOL, rel16
     return rel
+
+
+def _gemm_check(bat, Xq, Wq, M, N, K, rows=None, cols=None):
+    xc, xs, _ = _host(Xq, M, K)
+    wc, ws, _ = _host(Wq, N, K)
+    r = np.arange(M) if rows is None else np.asarray(rows)
+    c = np.arange(N) if cols is None else np.asarray(cols)
+    Xd = oracle.dequantize(xc[r], xs[r])
+    Wd = oracle.dequantize(wc[c], ws[c])
+    Y32 = bat.bat_mxfp4_gemm(Xq, Wq, out_dtype=torch.float32)
+    Y16 = bat.bat_mxfp4_gemm(Xq, Wq, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    y32 = Y32.cpu().numpy()[np.ix_(r, c)].astype(np.float64)
+    y16 = Y16.float().cpu().numpy()[np.ix_(r, c)].astype(np.float64)
+    return _check_outputs(y32, y16, Xd, Wd)
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 256), (64, 128, 256), (1, 8, 32), (17, 200, 96),
@@ -340,10 +348,17 @@ def test_gemm_shapes(bat, M, N, K):
     _gemm_check(bat, Xq, Wq, M, N, K)
 
 
-def _sample(n, count, seed):
+def _sample(n, count, seed, tile=None):
+    """Edge indices, `count` random ones and, with `tile`, one random index inside
+    every tile of that size (so every output tile of the GEMM is checked)."""
     rng = np.random.default_rng(seed)
     fixed = [0, 1, n // 2, n - 1] + ([127, 128] if n > 128 else [])
-    return np.unique(np.concatenate([fixed, rng.integers(0, n, size=count)]))
+    parts = [fixed, rng.integers(0, n, size=count)]
+    if tile:
+        starts = np.arange(0, n, tile)
+        parts.append(starts + rng.integers(0, tile, size=starts.size) % (n - starts))
+        parts.append(np.minimum(starts + tile - 1, n - 1))  # last row/column of each tile
+    return np.unique(np.concatenate(parts)).astype(np.int64)
 
 
 @pytest.mark.parametrize("name", wl.ORDER)
@@ -360,18 +375,14 @@ def test_linear_workloads(bat, name):
     Y2 = bat.bat_mxfp4_gemm(Xq, Wq, out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert torch.equal(Y, Y2)  # unfused linear == quantize then GEMM, bit for bit
-    rows = None if w.M <= 64 else _sample(w.M, 24, 1)
-    cols = None if w.N <= 512 else _sample(w.N, 200, 2)
-    # oracle path end to end (its own quantizer on its own transform)
+    # a row in every 128-row tile and a column in every 256-column tile, plus edges
+    r = np.arange(w.M) if w.M <= 64 else _sample(w.M, 24, 1, tile=128)
+    c = np.arange(w.N) if w.N <= 512 else _sample(w.N, 200, 2, tile=256)
     x_codes, x_scales, _ = _host(Xq, w.M, w.K)
     w_codes, w_scales, _ = _host(Wq, w.N, w.K)
-    ref = oracle.gemm_sampled(oracle.dequantize(x_codes, x_scales),
-                              oracle.dequantize(w_codes, w_scales), rows, cols)
-    r = np.arange(w.M) if rows is None else rows
-    c = np.arange(w.N) if cols is None else cols
     y = Y.cpu().numpy()[np.ix_(r, c)].astype(np.float64)
-    rel = np.linalg.norm(y - ref) / np.linalg.norm(ref)
-    assert rel <= GEMM_TOL, rel
+    _check_outputs(y, None, oracle.dequantize(x_codes[r], x_scales[r]),
+                   oracle.dequantize(w_codes[c], w_scales[c]))
     # and against the oracle's own quantization of its own transform (same codes almost everywhere)
     if w.M * w.K <= 2048 * 4096:
         _, oc, os_ = oracle.quantize_act(inp.X, inp.A, inp.B, inp.g_lo, inp.g_hi)
@@ -469,25 +480,16 @@ def test_quantize_act_mxfp8_workloads(bat, name):
 def _w4a8_check(bat, Xq, Wq, M, N, K, rows=None, cols=None):
     xc, xs, _ = _host8(Xq, M, K)
     wc, ws, _ = _host(Wq, N, K)
-    Xd = oracle.dequantize(xc, xs, "e4m3")
-    Wd = oracle.dequantize(wc, ws)
+    r = np.arange(M) if rows is None else np.asarray(rows)
+    c = np.arange(N) if cols is None else np.asarray(cols)
+    Xd = oracle.dequantize(xc[r], xs[r], "e4m3")
+    Wd = oracle.dequantize(wc[c], ws[c])
     Y32 = bat.bat_w4a8_gemm(Xq, Wq, out_dtype=torch.float32)
     Y16 = bat.bat_w4a8_gemm(Xq, Wq, out_dtype=torch.bfloat16)
     torch.cuda.synchronize()
-    ref = oracle.gemm_sampled(Xd, Wd, rows, cols)
-    r = np.arange(M) if rows is None else np.asarray(rows)
-    c = np.arange(N) if cols is None else np.asarray(cols)
     y32 = Y32.cpu().numpy()[np.ix_(r, c)].astype(np.float64)
     y16 = Y16.float().cpu().numpy()[np.ix_(r, c)].astype(np.float64)
-    assert np.all(np.isfinite(y32))
-    rel = np.linalg.norm(y32 - ref) / max(np.linalg.norm(ref), 1e-300)
-    assert rel <= GEMM_TOL, rel
-    mag = oracle.gemm_sampled(np.abs(Xd), np.abs(Wd), rows, cols)
-    assert np.all(np.abs(y32 - ref) <= 1e-5 * mag + 1e-30), np.max(np.abs(y32 - ref) / (mag + 1e-30))
-    ref16 = torch.from_numpy(ref).to(torch.bfloat16).float().numpy().astype(np.float64)
-    rel16 = np.linalg.norm(y16 - ref16) / max(np.linalg.norm(ref16), 1e-300)
-    assert rel16 <= GEMM_TOL, rel16
-    return rel
+    return _check_outputs(y32, y16, Xd, Wd)
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 128), (1, 8, 128), (17, 200, 256), (130, 300, 512),
@@ -504,7 +506,7 @@ def test_w4a8_gemm_shapes(bat, M, N, K):
     assert bat.bat_device_error() == 0
 
 
-@pytest.mark.parametrize("name", ["mlp_gate_up", "prefill_o", "decode_qkv"])
+@pytest.mark.parametrize("name", ["mlp_gate_up", "mlp_down", "prefill_o", "decode_qkv"])
 def test_w4a8_linear_workloads(bat, name):
     """W4A8 at the full workload sizes: sampled outputs against the oracle, and the
     error of the layer against the unquantized product below W4A4's."""
@@ -515,8 +517,8 @@ def test_w4a8_linear_workloads(bat, name):
     Xd = _dev_bf16(inp.X)
     Wq = bat.bat_prepare_weight(_dev_bf16(inp.W), Ad, Bd)
     Xq8 = bat.bat_quantize_act_mxfp8(Xd, Ad, Bd, gl, gh)
-    rows = None if w.M <= 64 else _sample(w.M, 24, 3)
-    cols = None if w.N <= 512 else _sample(w.N, 200, 4)
+    rows = None if w.M <= 64 else _sample(w.M, 24, 3, tile=128)
+    cols = None if w.N <= 512 else _sample(w.N, 200, 4, tile=256)
     _w4a8_check(bat, Xq8, Wq, w.M, w.N, w.K, rows, cols)
     Xq4 = bat.bat_quantize_act(Xd, Ad, Bd, gl, gh)
     Y4 = bat.bat_mxfp4_gemm(Xq4, Wq, out_dtype=torch.float32)

@@ -5,9 +5,9 @@ workspace from their framework, for example a plugin running under an allocator
 that already holds all device memory, or a serving loop that must not allocate
 once it is running. It keeps the quantized activations in the library's own
 static device scratch instead of a caller workspace. Its results must equal
-those of bat_linear, the entry point that takes a workspace. Two calls in a
-row, with different inputs, show that stale scratch contents from an earlier
-call do not leak into the next one.
+those of bat_linear, the entry point that takes a workspace, bit for bit. Calls
+in a row, with different inputs and a smaller call after a larger one, show that
+stale scratch contents from an earlier call do not leak into the next one.
 
 This file is collected last on purpose, so a failure here comes after every
 other GPU test has run.
@@ -52,6 +52,28 @@ def test_linear_noalloc_matches_linear_two_calls():
         torch.cuda.synchronize()
         assert torch.isfinite(got.float()).all()
         assert _rel(got.float(), ref.float()) <= GEMM_TOL, call
+        # the same kernels on the same bytes: equal bit for bit
+        assert torch.equal(got, ref), call
+    assert bat.bat_device_error() == 0
+
+
+def test_linear_noalloc_smaller_call_after_larger():
+    """A large call leaves its codes and scales in the shared scratch; smaller ragged
+    calls after it (rows inside the earlier call's 128-row groups, the tensor-core and
+    the CUDA-core quantizer paths, K with padding blocks) must not see them."""
+    import w4a4_bit_gemm_b200 as bat
+
+    N, K = 264, 1056  # 33 blocks: the tiled scales carry padding blocks 33..35
+    A, B, g_lo, g_hi = wl.random_factors(K // 32, seed=41)
+    Ad, Bd, gl, gh = _dev_f32(A), _dev_f32(B), _dev_f32(g_lo), _dev_f32(g_hi)
+    Wq = bat.bat_prepare_weight(_dev_bf16(wl.random_bf16((N, K), seed=42, scale=0.02)), Ad, Bd)
+    for i, M in enumerate([1000, 70, 5, 1000, 129]):
+        X = _dev_bf16(wl.random_bf16((M, K), seed=43 + i, scale=1.0 + 3.0 * (i % 2)))
+        ref = bat.bat_linear(X, Wq, Ad, Bd, gl, gh, out_dtype=torch.float32)
+        got = bat.bat_linear_noalloc(X, Wq, Ad, Bd, gl, gh, out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        assert torch.isfinite(got).all(), M
+        assert torch.equal(got, ref), M
     assert bat.bat_device_error() == 0
 
 
