@@ -24,12 +24,17 @@
 // that consecutive copies read adjacent 128-byte pieces of the same 128 rows.
 //   warp 0      producer: TMA copies of the units' boxes into a ring of kStages
 //               shared-memory stages;
-//   warp 1      TMEM owner and MMA issuer: per unit, two blocks x two K-steps of
-//               M=128, N=96, K=16 into one of two 192-column accumulators;
+//   warps 1, 18 MMA issuers, taking alternate units (unit n uses accumulator n % 2):
+//               per unit, two blocks x two K-steps of M=128, N=96, K=16 into one of
+//               two 192-column accumulators. The issuing thread waits about 150
+//               cycles on each MMA (the tensor pipe takes one M=128, K=16 step at a
+//               time) and some 100 on each barrier wait and commit, so with one issuer
+//               the tensor pipe idles while it waits; with two, one issues while the
+//               other waits. Warp 1 also owns TMEM;
 //   warps 2-17  two quantizer sets of eight warps; set s takes the units whose
 //               index within the CTA is s mod 2, warp (s, j, q) block j of the
 //               pair for the 32 tokens of TMEM lane quarter q.
-// Warps 1-17 build the strip's P terms (and its blocks' clip ratios) while the
+// Warps 1-18 build the strip's P terms (and its blocks' clip ratios) while the
 // producer's first copies are in flight. The issuer waits once per unit for its
 // copy and once for its accumulator, so its chain of waits, MMAs and commits
 // stays inside the copy's time, and each quantizer set has two units' time for
@@ -52,7 +57,8 @@ constexpr int kPPairBytes = kBlk * kPBlockBytes; // 12 KB
 constexpr int kPBytes = kStrip * kPPairBytes;    // one strip: 48 KB
 constexpr int kSets = 2;                         // quantizer sets (alternate units)
 constexpr int kSetWarps = 4 * kBlk;              // lane quarters x blocks
-constexpr int kThreads = 32 * (2 + kSets * kSetWarps);
+constexpr int kIssuers = 2;                      // MMA issuer warps (alternate units)
+constexpr int kThreads = 32 * (1 + kIssuers + kSets * kSetWarps);
 constexpr int kBuilders = kThreads - 32;         // every warp but the producer
 constexpr int kBarBytes = 2048;                  // barriers, TMEM address, clip ratios
 // A and the strip's B_b staged for the P build: s*s + 2*kStrip*(32/s)^2 floats, at most
@@ -64,6 +70,7 @@ constexpr bool fac_fits(int ls) {
 }
 static_assert(fac_fits(1), "the staged factors of every split s >= 2 fit the staging area");
 constexpr int kSmemBytes = kStages * kStageBytes + kPBytes + kBarBytes + 4 * kFacFloats + 1024;
+static_assert(kStages % kIssuers == 0 && kIssuers == 2, "issuer i owns accumulator i and every other stage");
 constexpr int kSlotCols = 96;                    // one block's accumulator: 3 terms x 32 columns
 constexpr uint32_t kAccCols = kBlk * kSlotCols;  // one unit's accumulator: 192 columns
 constexpr uint32_t kTmemCols = 512;              // allocation (power of two) holding 2 x 192
@@ -173,6 +180,30 @@ __device__ __forceinline__ void build_p_row(uint8_t* dst, const float* a, const 
 // Quantize one 32-element block held by this thread: clip to [r_lo*min, r_hi*max],
 // UE8M0 scale, then E2M1 codes (MXFP4: 16 bytes into `packed`) or, with kFp8, OCP
 // E4M3 codes (MXFP8: 32 bytes). Returns the scale byte e + 127.
+//
+// The clip is applied to the codes rather than to the values. The conversion is
+// monotone and symmetric, so the code of a clamped value is the code of the unclamped
+// value with its magnitude capped at the magnitude code of the bound on its side:
+// hi for a positive value, min(lo, hi) for a negative one (lo > hi happens only in a
+// one-signed block, where every value ends at hi). Codes are sign-magnitude with the
+// magnitude's order that of the values, so the cap is an unsigned minimum per code,
+// done on 8 packed E2M1 codes (or 4 E4M3 codes) per 32-bit word with integer ops.
+// This gives the codes of the value-domain clip exactly (the bound values are
+// converted the same way, fma(bound, 2^-e, +0)), with half the per-element work.
+template <int kBits>  // 4: E2M1 nibbles, 8: E4M3 bytes
+__device__ __forceinline__ uint32_t cap_codes(uint32_t w, uint32_t bp, uint32_t bn) {
+  constexpr uint32_t kOnes = kBits == 4 ? 0x11111111u : 0x01010101u;
+  constexpr uint32_t kSign = kOnes << (kBits - 1);       // sign bit of every code
+  constexpr uint32_t kMagMax = (1u << (kBits - 1)) - 1;  // 7 or 0x7f
+  const uint32_t neg = (w >> (kBits - 1)) & kOnes;       // 1 per negative code
+  const uint32_t bp_all = bp * kOnes, bn_all = bn * kOnes;
+  const uint32_t bw = bp_all ^ ((bp_all ^ bn_all) & (neg * ((1u << kBits) - 1)));  // cap per code
+  // per code: (sign bit set | magnitude) - cap >= sign bit  <=>  magnitude >= cap
+  const uint32_t d = (w | kSign) - bw;
+  const uint32_t sel = ((d >> (kBits - 1)) & kOnes) * kMagMax;
+  return (w & ~sel) | (bw & sel);
+}
+
 template <bool kFp8>
 __device__ __forceinline__ uint32_t quantize_block(const float (&y)[32], float r_lo, float r_hi,
                                                    uint32_t (&packed)[kFp8 ? 8 : 4]) {
@@ -201,32 +232,32 @@ __device__ __forceinline__ uint32_t quantize_block(const float (&y)[32], float r
   const int sbyte = efield > kEmax ? efield - kEmax : 0;  // e + 127
   const float inv_scale = __uint_as_float(static_cast<uint32_t>(254 - sbyte) << 23);  // 2^-e
   const uint64_t s2 = pack2(inv_scale, inv_scale);
-  // codes: v = c * 2^-e (+0 turns an exact -0 into +0), round to nearest even; E4M3:
-  // four codes per 32-bit word
+  // magnitude caps: codes of the bounds scaled the same way
+  const float cap_p = __fmaf_rn(hi, inv_scale, 0.0f);
+  const float cap_n = __fmaf_rn(fabsf(fminf(lo, hi)), inv_scale, 0.0f);
+  // codes of the unclipped values v = y * 2^-e (+0 turns an exact -0 into +0), round to
+  // nearest even, then capped
   if constexpr (kFp8) {
+    const uint32_t caps = e4m3x4(cap_p, cap_n, 0.0f, 0.0f);
+    const uint32_t bp = caps & 0x7fu, bn = (caps >> 8) & 0x7fu;
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       float v[4];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const float c0 = fminf(fmaxf(y[4 * c + 2 * h], lo), hi);
-        const float c1 = fminf(fmaxf(y[4 * c + 2 * h + 1], lo), hi);
-        unpack2(ffma2(pack2(c0, c1), s2, 0ull), v[2 * h], v[2 * h + 1]);
-      }
-      packed[c] = e4m3x4(v[0], v[1], v[2], v[3]);
+      for (int h = 0; h < 2; ++h)
+        unpack2(ffma2(pack2(y[4 * c + 2 * h], y[4 * c + 2 * h + 1]), s2, 0ull), v[2 * h], v[2 * h + 1]);
+      packed[c] = cap_codes<8>(e4m3x4(v[0], v[1], v[2], v[3]), bp, bn);
     }
   } else {
-    // E2M1: eight codes per 32-bit word
+    const uint32_t caps = e2m1x2(cap_p, cap_n);
+    const uint32_t bp = caps & 7u, bn = (caps >> 4) & 7u;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       float v[8];
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const float c0 = fminf(fmaxf(y[8 * c + 2 * h], lo), hi);
-        const float c1 = fminf(fmaxf(y[8 * c + 2 * h + 1], lo), hi);
-        unpack2(ffma2(pack2(c0, c1), s2, 0ull), v[2 * h], v[2 * h + 1]);
-      }
-      packed[c] = e2m1x8(v);
+      for (int h = 0; h < 4; ++h)
+        unpack2(ffma2(pack2(y[8 * c + 2 * h], y[8 * c + 2 * h + 1]), s2, 0ull), v[2 * h], v[2 * h + 1]);
+      packed[c] = cap_codes<4>(e2m1x8(v), bp, bn);
     }
   }
   return static_cast<uint32_t>(sbyte);
@@ -252,8 +283,8 @@ __global__ void __launch_bounds__(pro::kThreads, 1)
   auto tfull = [&](uint32_t a) { return bars + 8u * (2 * kStages + a); };
   auto tempty = [&](uint32_t a) { return bars + 8u * (2 * kStages + 2 + a); };
   const uint32_t pfull = bars + 8u * (2 * kStages + 4);
-  const uint32_t done_bar = pfull + 8u;
-  const uint32_t tmem_slot = done_bar + 8u;
+  auto done_bar = [&](int i) { return pfull + 8u * (1 + i); };
+  const uint32_t tmem_slot = pfull + 8u * (1 + kIssuers);
   volatile uint32_t* tmem_slot_ptr =
       reinterpret_cast<volatile uint32_t*>(base_ptr + (tmem_slot - base));
   // clip ratios of the strip's blocks: [2 * kStrip] lo, then [2 * kStrip] hi
@@ -289,7 +320,7 @@ __global__ void __launch_bounds__(pro::kThreads, 1)
       mbar_init(tempty(a), kSetWarps);
     }
     mbar_init(pfull, kBuilders);
-    mbar_init(done_bar, 1);
+    for (int i = 0; i < kIssuers; ++i) mbar_init(done_bar(i), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&tmap_x);
   }
@@ -312,6 +343,7 @@ __global__ void __launch_bounds__(pro::kThreads, 1)
     // that the memory system sees whole row segments rather than lone 128-byte
     // pieces of rows 8 KB apart.
     if (lane == 0) {
+      const uint64_t pol = policy_evict_first();  // X is read once
       int stage = 0;
       uint32_t phase = 0;
       uint32_t inflight = 0;  // bit s: stage s was loaded; bit 16+s: parity of that load
@@ -331,8 +363,8 @@ __global__ void __launch_bounds__(pro::kThreads, 1)
         }
         for (int i = 0; i < cnt && ok; ++i) {
           mbar_expect_tx(full_bar(stage), kStageBytes);
-          tma_load_2d(base + stage * kStageBytes, &tmap_x, full_bar(stage),
-                      (pair_base + pr) * 64, static_cast<int32_t>(mt * kTok));
+          tma_load_2d_hint(base + stage * kStageBytes, &tmap_x, full_bar(stage),
+                           (pair_base + pr) * 64, static_cast<int32_t>(mt * kTok), pol);
           inflight = (inflight & ~(0x10001u << stage)) | (1u << stage) | (phase << (16 + stage));
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
           if (++pr == npair) { pr = 0; ++mt; }
@@ -382,18 +414,22 @@ __global__ void __launch_bounds__(pro::kThreads, 1)
       fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor cores
       mbar_arrive(pfull);
     }
-    if (warp == 1) {
-      // ---------------------------------------------------------- MMA issuer
+    if (warp == 1 || warp >= 2 + kSets * kSetWarps) {
+      // ---------------------------------------------------------- MMA issuers
+      // issuer i takes units n = i, i + kIssuers, ...: accumulator n % 2 = i and stages
+      // of its own (kStages is even)
+      const int iss = warp == 1 ? 0 : warp - (1 + kSets * kSetWarps);
       if (lane == 0 && mbar_wait(pfull, 0, kErrWaitFull)) {
         constexpr uint32_t idesc = idesc_bf16(kTok, kSlotCols);
         // Descriptors differ only in the start-address field (bits 0-13, address / 16).
         const uint64_t adesc0 = smem_desc(base, 16, 1024, 2);
         const uint64_t bdesc0 = smem_desc(pbase, 128, 512, 0);
-        int stage = 0;
+        int stage = iss;
         uint32_t phase = 0;
-        int pr = pr0;
-        uint32_t n = 0;
-        for (int64_t v = v_begin; v < v_end; ++v, ++n) {
+        int pr = pr0 + iss;
+        if (pr >= npair) pr -= npair;
+        uint32_t n = static_cast<uint32_t>(iss);
+        for (int64_t v = v_begin + iss; v < v_end; v += kIssuers, n += kIssuers) {
           const uint32_t a = n & 1u;
           if (!mbar_wait(full_bar(stage), phase, kErrWaitFull)) break;
           if (!mbar_wait(tempty(a), ((n >> 1) & 1u) ^ 1u, kErrWaitTmemEmpty)) break;
@@ -411,12 +447,14 @@ __global__ void __launch_bounds__(pro::kThreads, 1)
                        bd + ((j * kPBlockBytes + ks * 256) >> 4), idesc, static_cast<uint32_t>(ks));
           tc_commit(tfull(a));
           tc_commit(empty_bar(stage));
-          if (++stage == kStages) { stage = 0; phase ^= 1u; }
-          if (++pr == npair) pr = 0;
+          stage += kIssuers;
+          if (stage >= kStages) { stage -= kStages; phase ^= 1u; }
+          pr += kIssuers;
+          while (pr >= npair) pr -= npair;
         }
         // every MMA issued above has finished before TMEM is released
-        tc_commit(done_bar);
-        mbar_wait(done_bar, 0, kErrWaitTmemFull);
+        tc_commit(done_bar(iss));
+        mbar_wait(done_bar(iss), 0, kErrWaitTmemFull);
       }
     } else {
       // ------------------------------------------------------ quantizer sets
