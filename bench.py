@@ -821,7 +821,14 @@ def main():
             cpu["prologue_1thread"] = oracle_prologue_rate(inp, w, budget, 1)
             cpu["prologue_all_cores"] = oracle_prologue_rate(inp, w, budget, oracle.num_threads())
 
-    gemm_kernel = "bat_mxf4_gemm_kernel<true> (W4A8)" if a8 else "bat_mxf4_gemm_kernel"
+    # the library's GEMM routing: CTA pairs on 256 x 256 tiles for MXFP4 activations with
+    # more than one 128-row tile, the one-SM kernel otherwise (W4A8, decode split-K)
+    if a8:
+        gemm_kernel = "bat_mxf4_gemm_kernel<true> (W4A8)"
+    elif w.M > 128:
+        gemm_kernel = "bat_mxf4_gemm_pair_kernel (cta_group::2)"
+    else:
+        gemm_kernel = "bat_mxf4_gemm_kernel"
     pro_kernel = "bat_prologue_kernel<..., MXFP8>" if a8 else "bat_prologue_kernel"
     clocks = r["clocks"]
     if rank == 0:

@@ -14,6 +14,7 @@
 #include "../../include/bat.h"
 #include "bat_common.cuh"
 #include "bat_gemm.cuh"
+#include "bat_gemm2.cuh"
 #include "bat_kv.cuh"
 #include "bat_prologue.cuh"
 
@@ -37,6 +38,8 @@ struct DeviceInfo {
   std::atomic<int> gemm_attr{0};    // bit 0: W4A4 GEMM, bit 1: W4A8 GEMM attribute set
   std::atomic<int> pro_attr{0};     // bit t: the prologue variant t has its smem attribute set
   std::atomic<int> max_clusters[2][9];  // [W4A8][cluster size]: clusters resident at once, 0 unknown
+  std::atomic<int> pair_attr{0};        // the CTA-pair GEMM's smem attribute is set
+  std::atomic<int> max_pairs{0};        // CTA pairs of that GEMM resident at once, 0 unknown
 };
 DeviceInfo g_dev[64];
 
@@ -151,6 +154,21 @@ bool make_out_map(CUtensorMap* map, void* y, int64_t M, int64_t N) {
   cuuint32_t estr[2] = {1u, 1u};
   CUresult r = f(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box, estr,
                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// bf16 Y [M][N] for the CTA-pair GEMM's TMA store: box of 32 columns (64 bytes) x 128 rows,
+// 64-byte swizzle, matching that epilogue's staging layout. Needs N % 8 == 0.
+bool make_out_map64(CUtensorMap* map, void* y, int64_t M, int64_t N) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(N * 2)};
+  cuuint32_t box[2] = {32u, static_cast<cuuint32_t>(bat::gemm2::kRows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = f(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -428,6 +446,54 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
     }
   }
   p.splits = static_cast<int>(splits);
+  if (!a8 && splits == 1 && m_tiles >= 2) {
+    // CTA pairs on 256 x 256 tiles (bat_gemm2.cuh)
+    CUtensorMap pa, pb, py;
+    if (!make_code_map(&pa, Xq->codes, Xq->rows, Xq->k, bat::gemm2::kRows)) return BAT_ERR_CUDA;
+    if (!make_code_map(&pb, Wq->codes, Wq->rows, Wq->k, bat::gemm2::kBN / 2)) return BAT_ERR_CUDA;
+    std::memset(&py, 0, sizeof(py));
+    if (p.tma_store && !make_out_map64(&py, Y, p.M, p.N)) return BAT_ERR_CUDA;
+    void (*pk)(CUtensorMap, CUtensorMap, CUtensorMap, bat::GemmParams) = bat::bat_mxf4_gemm_pair_kernel;
+    if (!d.pair_attr.load()) {
+      const cudaError_t ae = cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  bat::gemm2::kSmemBytes);
+      if (ae != cudaSuccess) return cuda_status(ae);
+      d.pair_attr.store(1);
+    }
+    const int64_t tiles2 = ((p.M + 255) / 256) * ((p.N + bat::gemm2::kBN - 1) / bat::gemm2::kBN);
+    int npair = d.max_pairs.load();
+    if (npair == 0) {
+      cudaLaunchConfig_t oc = {};
+      oc.gridDim = dim3(static_cast<unsigned>(sms & ~1));
+      oc.blockDim = dim3(bat::gemm2::kThreads);
+      oc.dynamicSmemBytes = bat::gemm2::kSmemBytes;
+      cudaLaunchAttribute ca[1];
+      ca[0].id = cudaLaunchAttributeClusterDimension;
+      ca[0].val.clusterDim.x = 2;
+      ca[0].val.clusterDim.y = 1;
+      ca[0].val.clusterDim.z = 1;
+      oc.attrs = ca;
+      oc.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&npair, pk, &oc) != cudaSuccess || npair < 1) npair = sms / 2;
+      d.max_pairs.store(npair);
+    }
+    const int64_t pairs = tiles2 < npair ? tiles2 : npair;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    cfg.blockDim = dim3(bat::gemm2::kThreads);
+    cfg.dynamicSmemBytes = bat::gemm2::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cuda_status(cudaLaunchKernelEx(&cfg, pk, pa, pb, py, p));
+  }
   const int grid = splits > 1 ? static_cast<int>(tiles * splits)
                               : static_cast<int>(tiles < sms ? tiles : sms);
   // Programmatic stream serialization: the kernel's set-up may overlap the previous

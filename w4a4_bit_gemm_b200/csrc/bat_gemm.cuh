@@ -316,6 +316,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      uint32_t inflight = 0;  // bit s: stage s was loaded; bit 16+s: parity of that load
       for (int64_t tile = tile0; tile < tiles && ok; tile += tstride) {
         const int64_t mt = tile % m_tiles;
         const int64_t nt = tile / m_tiles;
@@ -337,9 +338,16 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
           tma_load_2d(sa, &tmap_a, full_bar(stage), ks * 128, static_cast<int32_t>(mt * kBM));
           tma_load_2d(sa + kABytes, &tmap_b, full_bar(stage), ks * 128,
                       static_cast<int32_t>(nt * kBN));
+          inflight = (inflight & ~(0x10001u << stage)) | (1u << stage) | (phase << (16 + stage));
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
       }
+      // No copy may still be writing shared memory when the CTA exits: wait (bounded) for
+      // the last load of every stage. Its phase completes when all five copies of the stage
+      // (this warp's code tiles and warp 10's scale chunks, counted together) have landed,
+      // so this also covers the scale producer's copies of the stage.
+      for (int s = 0; s < kStages; ++s)
+        if ((inflight >> s) & 1u) mbar_wait(full_bar(s), (inflight >> (16 + s)) & 1u, kErrWaitFull);
     }
   } else if (warp == 10) {
     // ------------------------------------------------------------ scale producer
@@ -348,6 +356,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      uint32_t inflight = 0;  // as in the code producer
       for (int64_t tile = tile0; tile < tiles && ok; tile += tstride) {
         const int64_t mt = tile % m_tiles;
         const int64_t nt = tile / m_tiles;
@@ -362,9 +371,13 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
           for (int g = 0; g < ngb; ++g)
             bulk_load(sa + kABytes + kBBytes + kSfaBytes + g * (kChunksPerStage * kChunk),
                       p.sfb + ((nt * 2 + g) * p.nbp4 + c0) * kChunk, nch * kChunk, full_bar(stage));
+          inflight = (inflight & ~(0x10001u << stage)) | (1u << stage) | (phase << (16 + stage));
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
       }
+      // the same bounded drain for this warp's copies
+      for (int s = 0; s < kStages; ++s)
+        if ((inflight >> s) & 1u) mbar_wait(full_bar(s), (inflight >> (16 + s)) & 1u, kErrWaitFull);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
@@ -505,17 +518,21 @@ __global__ void __launch_bounds__(gemm::kThreads, 1)
         if (lane == 0) mbar_arrive(tmem_empty);
       } else if (p.tma_store) {
         // 1) drain the accumulator into registers as bf16 pairs and release TMEM at once
+        //    (four 32-column loads per wait: two round trips instead of eight)
         uint32_t h[kBN / 2];
 #pragma unroll
-        for (int cc = 0; cc < kBN / 32; ++cc) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(trow + cc * 32, r);
+        for (int hh = 0; hh < kBN / 128; ++hh) {
+          uint32_t r[4][32];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) tmem_ld_32x32b_x32(trow + (hh * 4 + i) * 32, r[i]);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1]));
-            h[cc * 16 + c] = *reinterpret_cast<uint32_t*>(&v);
-          }
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(r[i][2 * c]), __uint_as_float(r[i][2 * c + 1]));
+              h[(hh * 4 + i) * 16 + c] = *reinterpret_cast<uint32_t*>(&v);
+            }
         }
         tc_fence_before();
         __syncwarp();
