@@ -336,6 +336,8 @@ def _gemm_check(bat, Xq, Wq, M, N, K, rows=None, cols=None):
                                    # one row of tiles: split-K over a cluster per tile
                                    (1, 256, 2048), (100, 520, 1024), (128, 1000, 768),
                                    (33, 300, 2080), (16, 6144, 4096),
+                                   # decode kernel: eight K stages per CTA, 48 token rows
+                                   (5, 136, 16384), (48, 1000, 4128),
                                    # CTA pairs: 256 x 256 tiles, ragged rows, columns and K
                                    (512, 768, 2048), (384, 256, 1056), (129, 136, 32),
                                    (1000, 1288, 4128)])

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <chrono>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -15,6 +16,7 @@
 #include "bat_common.cuh"
 #include "bat_gemm.cuh"
 #include "bat_gemm2.cuh"
+#include "bat_gemm_dec.cuh"
 #include "bat_kv.cuh"
 #include "bat_prologue.cuh"
 
@@ -40,6 +42,8 @@ struct DeviceInfo {
   std::atomic<int> max_clusters[2][9];  // [W4A8][cluster size]: clusters resident at once, 0 unknown
   std::atomic<int> pair_attr{0};        // the CTA-pair GEMM's smem attribute is set
   std::atomic<int> max_pairs{0};        // CTA pairs of that GEMM resident at once, 0 unknown
+  std::atomic<int> dec_attr{0};         // the decode GEMM's smem attribute is set
+  std::atomic<int> dec_clusters[9];     // [cluster size]: its clusters resident at once, 0 unknown
 };
 DeviceInfo g_dev[64];
 
@@ -256,11 +260,29 @@ bat_status_t check_act_args(const void* X, int64_t M, int64_t K, const float* A,
 
 // The CUDA-core row quantizer: activation rows (slots == null: codes [rows][D(/2)], tiled
 // scales) or KV-cache rows (token row / H stored at cache slot slots[token]).
+// Activation batches of at most this many rows run on the CUDA-core row quantizer
+// (its latency is a few microseconds; the tensor-core prologue's set-up costs more).
+constexpr int64_t kRowsCudaCore = 64;
+// The linear layer at those sizes: room for the row quantizer's per-CTA completion flags
+// (64-bit; its grid is at most 16 warps per SM, two CTAs per SM) and their epochs, unique
+// per call and process (a salted counter), so flags left by earlier calls never match.
+constexpr size_t kDoneFlagBytes = 4096;
+std::atomic<unsigned long long> g_calls{0};
+unsigned long long next_epoch() {
+  static const unsigned long long salt =
+      (static_cast<unsigned long long>(std::chrono::steady_clock::now().time_since_epoch().count()) *
+       0x9E3779B97F4A7C15ull) ^ static_cast<unsigned long long>(reinterpret_cast<uintptr_t>(&g_calls));
+  return (salt + 2 * g_calls.fetch_add(1)) | 1ull;  // odd, so never the 0 of fresh memory
+}
+
+// done_flags (activation rows only): one 64-bit completion flag per CTA, set to `epoch`;
+// *grid_out gets the number of CTAs.
 bat_status_t launch_rows(const void* x, int64_t rows, int64_t H, int64_t S,
                                 const int64_t* slots, int64_t D, const float* A, const float* B,
                                 const float* g_lo, const float* g_hi, int ls, bool fp8,
                                 uint8_t* codes, uint8_t* scales, float* y_out, int sms,
-                                cudaStream_t s) {
+                                cudaStream_t s, unsigned long long* done_flags = nullptr,
+                                unsigned long long epoch = 0, int* grid_out = nullptr) {
   bat::RowQuantParams p;
   p.x = static_cast<const uint16_t*>(x);
   p.a = A;
@@ -279,6 +301,9 @@ bat_status_t launch_rows(const void* x, int64_t rows, int64_t H, int64_t S,
   p.groups = (p.nb + 3) / 4;
   p.ls = ls;
   p.nbp4 = (p.nb + 3) / 4;
+  p.done_flags = slots == nullptr ? done_flags : nullptr;
+  p.epoch = epoch;
+  if (grid_out) *grid_out = 0;
   // about 16 warps per SM in all, each group of blocks over a stride of R rows
   int64_t R = static_cast<int64_t>(sms) * 16 / p.groups;
   if (R > rows) R = rows;
@@ -286,6 +311,8 @@ bat_status_t launch_rows(const void* x, int64_t rows, int64_t H, int64_t S,
   p.R = static_cast<int>(R);
   const int64_t warps = static_cast<int64_t>(p.groups) * R;
   const unsigned grid = static_cast<unsigned>((warps + bat::kv::kWarps - 1) / bat::kv::kWarps);
+  if (grid > kDoneFlagBytes / 8) p.done_flags = nullptr;  // (never at supported sizes)
+  if (grid_out) *grid_out = p.done_flags != nullptr ? static_cast<int>(grid) : 0;
   const bool kv = slots != nullptr, tr = y_out != nullptr;
   void (*k)(bat::RowQuantParams);
   if (kv)
@@ -298,15 +325,13 @@ bat_status_t launch_rows(const void* x, int64_t rows, int64_t H, int64_t S,
   return cuda_status(cudaGetLastError());
 }
 
-// Activation batches of at most this many rows run on the CUDA-core row quantizer
-// (its latency is a few microseconds; the tensor-core prologue's set-up costs more).
-constexpr int64_t kRowsCudaCore = 64;
-
 bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float* A,
                              const float* B, const float* g_lo, const float* g_hi, bool per_row,
                              const bat_mxfp4_t* out, float* y_out, cudaStream_t stream,
                              int ls = 3, bool fp8 = false, const int64_t* kv_slots = nullptr,
-                             int64_t kv_heads = 0, int64_t kv_nslots = 0) {
+                             int64_t kv_heads = 0, int64_t kv_nslots = 0,
+                             unsigned long long* done_flags = nullptr, unsigned long long epoch = 0,
+                             int* rows_grid_out = nullptr) {
   int dev = 0, sms = 0;
   bat_status_t st = current_device(&dev, &sms);
   if (st != BAT_OK) return st;
@@ -314,7 +339,7 @@ bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float
   if (!per_row && kv_slots == nullptr && rows <= kRowsCudaCore)
     return launch_rows(X, rows, 1, 0, nullptr, K, A, B, g_lo, g_hi, ls, fp8,
                        static_cast<uint8_t*>(out->codes), static_cast<uint8_t*>(out->scales), y_out,
-                       sms, stream);
+                       sms, stream, done_flags, epoch, rows_grid_out);
   CUtensorMap tx;
   if (!make_act_map(&tx, X, rows, K)) return BAT_ERR_CUDA;
   bat::PrologueParams p;
@@ -375,8 +400,14 @@ bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float
 }
 
 // a8: Xq holds MXFP8 (E4M3) activations and the W4A8 kernel runs; K % 128 == 0 then.
+// w_static: the kernel before the GEMM on the stream does not write the weights (the
+// linear layer: that kernel is the activation quantizer). q_flags / q_ctas / epoch: that
+// quantizer's completion flags (row quantizer), which the decode GEMM waits on instead of
+// the grid dependency; null otherwise.
 bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
-                         bat_out_dtype_t out_dtype, cudaStream_t stream, bool a8 = false) {
+                         bat_out_dtype_t out_dtype, cudaStream_t stream, bool a8 = false,
+                         bool w_static = false, const unsigned long long* q_flags = nullptr,
+                         int q_ctas = 0, unsigned long long epoch = 0) {
   int dev = 0, sms = 0;
   bat_status_t st = current_device(&dev, &sms);
   if (st != BAT_OK) return st;
@@ -411,6 +442,64 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
   // shapes): up to 8 CTAs per tile, at least one K stage each.
   const int64_t k_stages = (p.K + (a8 ? 127 : 255)) / (a8 ? 128 : 256);
   DeviceInfo& d = g_dev[dev];
+  const int64_t dks = (p.K + bat::gemmd::kBK - 1) / bat::gemmd::kBK;
+  if (!a8 && p.M <= bat::gemmd::kMaxNx && dks <= bat::gemmd::kStages * bat::gemmd::kMaxSplits) {
+    // decode shapes: Y^T = Wq . Xq^T on 128-row W tiles, K split over a cluster of S CTAs
+    // per tile (bat_gemm_dec.cuh): the smallest power of two S that leaves each CTA at most
+    // kStages K stages, doubled while the doubled grid still fits the SMs in one wave
+    const int nx = static_cast<int>((p.M + 15) / 16 * 16);
+    CUtensorMap tw;
+    if (!make_code_map(&tw, Wq->codes, Wq->rows, Wq->k, bat::gemmd::kBM)) return BAT_ERR_CUDA;
+    if (q_ctas <= 0) q_flags = nullptr;
+    void (*dk)(CUtensorMap, bat::GemmParams, const uint8_t*, int, int, const unsigned long long*, int,
+               unsigned long long) = bat::bat_mxf4_gemm_dec_kernel;
+    if (!d.dec_attr.load()) {
+      const cudaError_t ae = cudaFuncSetAttribute(dk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  bat::gemmd::kSmemBytes);
+      if (ae != cudaSuccess) return cuda_status(ae);
+      d.dec_attr.store(1);
+    }
+    const int64_t wt = (p.N + bat::gemmd::kBM - 1) / bat::gemmd::kBM;
+    int S = 1;
+    while (S * bat::gemmd::kStages < dks) S *= 2;
+    while (2 * S <= bat::gemmd::kMaxSplits && 2 * S <= dks && wt * 2 * S <= sms) S *= 2;
+    if (S > 1) {
+      int n = d.dec_clusters[S].load();
+      if (n == 0) {
+        cudaLaunchConfig_t oc = {};
+        oc.gridDim = dim3(static_cast<unsigned>(wt * S));
+        oc.blockDim = dim3(bat::gemmd::kThreads);
+        oc.dynamicSmemBytes = bat::gemmd::kSmemBytes;
+        cudaLaunchAttribute ca[1];
+        ca[0].id = cudaLaunchAttributeClusterDimension;
+        ca[0].val.clusterDim.x = static_cast<unsigned>(S);
+        ca[0].val.clusterDim.y = 1;
+        ca[0].val.clusterDim.z = 1;
+        oc.attrs = ca;
+        oc.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, dk, &oc) != cudaSuccess || n < 1) n = -1;
+        d.dec_clusters[S].store(n);
+      }
+      if (n < 1) return BAT_ERR_UNSUPPORTED;  // clusters of S CTAs cannot be resident
+    }
+    p.splits = S;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(wt * S));
+    cfg.blockDim = dim3(bat::gemmd::kThreads);
+    cfg.dynamicSmemBytes = bat::gemmd::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(S);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = S > 1 ? 2 : 1;
+    return cuda_status(cudaLaunchKernelEx(&cfg, dk, tw, p, static_cast<const uint8_t*>(Xq->codes), nx,
+                                          w_static ? 1 : 0, q_flags, q_ctas, epoch));
+  }
   const int variant_bit = a8 ? 2 : 1;
   if (!(d.gemm_attr.load() & variant_bit)) {
     const cudaError_t ae =
@@ -854,6 +943,10 @@ size_t bat_linear_workspace_bytes(int64_t M, int64_t K) {
   const size_t c = bat_mxfp4_codes_bytes(M, K);
   const size_t s = bat_mxfp4_scales_bytes(M, K);
   if (!c || !s) return 0;
+  // decode sizes (row quantizer): the quantizer's completion flags after the scales
+  if (M <= kRowsCudaCore)
+    return static_cast<size_t>(round_up(static_cast<int64_t>(c), 256) +
+                               round_up(static_cast<int64_t>(s), 256)) + kDoneFlagBytes;
   return static_cast<size_t>(round_up(static_cast<int64_t>(c), 256)) + s;
 }
 
@@ -878,9 +971,22 @@ bat_status_t bat_linear(const void* X, int64_t M, const bat_mxfp4_t* Wq, const f
   st = check_gemm_args(&xq, Wq, Y, out_dtype);
   if (st != BAT_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = launch_prologue(X, M, K, A, B, g_lo, g_hi, false, &xq, nullptr, s);
+  // decode sizes: the row quantizer signals completion through flags after the scales,
+  // which the GEMM waits on (see launch_gemm)
+  unsigned long long* flags = nullptr;
+  unsigned long long epoch = 0;
+  int q_ctas = 0;
+  if (M <= kRowsCudaCore) {
+    flags = reinterpret_cast<unsigned long long*>(
+        static_cast<uint8_t*>(xq.scales) +
+        round_up(static_cast<int64_t>(bat_mxfp4_scales_bytes(M, K)), 256));
+    epoch = next_epoch();
+  }
+  st = launch_prologue(X, M, K, A, B, g_lo, g_hi, false, &xq, nullptr, s, 3, false, nullptr, 0, 0,
+                       flags, epoch, &q_ctas);
   if (st != BAT_OK) return st;
-  return launch_gemm(&xq, Wq, Y, out_dtype, s);
+  // the kernel right before the GEMM is the quantizer, which does not write the weights
+  return launch_gemm(&xq, Wq, Y, out_dtype, s, false, true, flags, q_ctas, epoch);
 }
 
 const char* bat_last_cuda_error(void) {
@@ -1042,7 +1148,20 @@ extern "C" bat_status_t bat_linear_noalloc(const void* X, int64_t M, const bat_m
   xq.scales = static_cast<uint8_t*>(scratch) +
               round_up(static_cast<int64_t>(bat_mxfp4_codes_bytes(M, K)), 256);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = launch_prologue(X, M, K, A, B, g_lo, g_hi, false, &xq, nullptr, s);
+  // decode sizes: the row quantizer signals completion through flags after the scales,
+  // which the GEMM waits on (see launch_gemm)
+  unsigned long long* flags = nullptr;
+  unsigned long long epoch = 0;
+  int q_ctas = 0;
+  if (M <= kRowsCudaCore) {
+    flags = reinterpret_cast<unsigned long long*>(
+        static_cast<uint8_t*>(xq.scales) +
+        round_up(static_cast<int64_t>(bat_mxfp4_scales_bytes(M, K)), 256));
+    epoch = next_epoch();
+  }
+  st = launch_prologue(X, M, K, A, B, g_lo, g_hi, false, &xq, nullptr, s, 3, false, nullptr, 0, 0,
+                       flags, epoch, &q_ctas);
   if (st != BAT_OK) return st;
-  return launch_gemm(&xq, Wq, Y, out_dtype, s);
+  // the kernel right before the GEMM is the quantizer, which does not write the weights
+  return launch_gemm(&xq, Wq, Y, out_dtype, s, false, true, flags, q_ctas, epoch);
 }

@@ -110,6 +110,10 @@ struct RowQuantParams {
   int D, nb, groups, ls;  // D = channels per row, nb = D/32, groups = ceil(nb/4), log2 s
   int R;                  // warps per group: row stride
   int nbp4;               // linear mode: ceil(nb/4) of the tiled scale layout
+  // optional completion flags (linear mode): CTA i stores `epoch` into done_flags[i]
+  // (release, GPU scope) once all its outputs are written; null: none
+  unsigned long long* done_flags;
+  unsigned long long epoch;
 };
 
 // kKv: rows are (token, head) pairs stored into cache slots (codes [slot][H][D] or
@@ -118,10 +122,32 @@ struct RowQuantParams {
 template <bool kFp8, bool kTrace, bool kKv>
 __global__ void __launch_bounds__(kv::kThreads, 1)
     bat_rows_quantize_kernel(const RowQuantParams p) {
+  // per warp (factor split s = 8): A, the group's four B_b, its four pairs of clip logits
+  __shared__ float fac_smem[kv::kWarps][136];
   // a following kernel launched with programmatic serialization (the GEMM) may start
   // its set-up now; this kernel's inputs come from the kernels before it
   allow_dependents();
   grid_dependency_wait();
+  if (!kKv) {
+    // padding of the tiled scale layout: rows [M, 128-row boundary) and blocks
+    // [nb, 4 nbp4) of the real rows are 0 (the GEMM multiplies by 2^(byte-127)); done
+    // first, so these stores overlap the loads below
+    const int64_t mpad = (p.rows + 127) / 128 * 128;
+    const int64_t tail = 4 * p.nbp4 - p.nb;  // 0..3 padding blocks per real row
+    const int64_t n_rows_pad = (mpad - p.rows) * p.nbp4;
+    const int64_t total = n_rows_pad + p.rows * tail;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+      if (i < n_rows_pad) {
+        const int64_t m = p.rows + i / p.nbp4;
+        const int64_t c = i % p.nbp4;
+        *reinterpret_cast<uint32_t*>(p.scales + scale_offset(m, 4 * c, p.nbp4)) = 0u;
+      } else {
+        const int64_t j = i - n_rows_pad;
+        p.scales[scale_offset(j / tail, p.nb + j % tail, p.nbp4)] = 0;
+      }
+    }
+  }
   const int lane = threadIdx.x & 31;
   const int u = lane & 7;
   const int64_t wid = static_cast<int64_t>(blockIdx.x) * kv::kWarps + (threadIdx.x >> 5);
@@ -130,28 +156,52 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
     const int blk = 4 * g + (lane >> 3);
     const bool has = blk < p.nb;  // lanes of a missing fourth block idle (shuffles stay full)
     const int bq = has ? blk : 0;
-    const float r_lo = (has && p.g_lo) ? clip_ratio(p.g_lo[bq]) : 1.0f;
-    const float r_hi = (has && p.g_hi) ? clip_ratio(p.g_hi[bq]) : 1.0f;
+    // the first row's block is requested before the factors, so that its load and theirs
+    // are in flight together
+    int64_t row = wid / p.groups;
+    float x[32];
+    if (row < p.rows) rows_load_block(p.x + row * p.D + bq * kG, x);
+    float r_lo = 1.0f, r_hi = 1.0f;
     float pc[32][4];
-    if (p.ls == 3)
-      rows_build_pc<3>(pc, p.a, p.b, bq, u, 3);
-    else
+    if (p.ls == 3) {
+      // A (8 x 8), the four blocks' B_b (4 x 4 each) and clip logits: one load per lane
+      // or two, all in flight at once, into this warp's shared-memory slice
+      float* f = fac_smem[threadIdx.x >> 5];
+      const int b0 = 4 * g;
+      f[lane] = __ldg(p.a + lane);
+      f[32 + lane] = __ldg(p.a + 32 + lane);
+      if (b0 + (lane >> 4) < p.nb) f[64 + lane] = __ldg(p.b + b0 * 16 + lane);
+      if (b0 + 2 + (lane >> 4) < p.nb) f[96 + lane] = __ldg(p.b + b0 * 16 + 32 + lane);
+      if (lane < 4 && b0 + lane < p.nb) {
+        f[128 + lane] = p.g_lo ? __ldg(p.g_lo + b0 + lane) : 0.0f;
+        f[132 + lane] = p.g_hi ? __ldg(p.g_hi + b0 + lane) : 0.0f;
+      }
+      __syncwarp();
+      const int bl = has ? blk - b0 : 0;  // the lane's block within the four
+      if (has && p.g_lo) r_lo = clip_ratio(f[128 + bl]);
+      if (has && p.g_hi) r_hi = clip_ratio(f[132 + bl]);
+      rows_build_pc<3, false>(pc, f, f + 64, bl, u, 3);
+    } else {
+      if (has && p.g_lo) r_lo = clip_ratio(p.g_lo[bq]);
+      if (has && p.g_hi) r_hi = clip_ratio(p.g_hi[bq]);
       rows_build_pc<-1>(pc, p.a, p.b, bq, u, p.ls);
-    for (int64_t row = wid / p.groups; row < p.rows; row += p.R) {
+    }
+    for (; row < p.rows; row += p.R) {
       int64_t slot = row;
       if (kKv) {
         slot = p.slots[row / p.H];
         if (slot >= p.S) {
           if (lane == 0) atomicOr(&g_dev_error, kErrBadIndex);
+          if (row + p.R < p.rows) rows_load_block(p.x + (row + p.R) * p.D + bq * kG, x);
           continue;
         }
       }
-      float x[32];
-      rows_load_block(p.x + row * p.D + bq * kG, x);
       float y[4];
       uint32_t code;
       int sbyte;
       rows_block_quant<kFp8>(x, pc, r_lo, r_hi, y, code, sbyte);
+      // the next row's block (this one's values are consumed)
+      if (row + p.R < p.rows) rows_load_block(p.x + (row + p.R) * p.D + bq * kG, x);
       const int64_t e0 = row * p.D + blk * kG + 4 * u;
       if (kTrace && has)
         *reinterpret_cast<float4*>(p.y_out + e0) = make_float4(y[0], y[1], y[2], y[3]);
@@ -171,23 +221,13 @@ __global__ void __launch_bounds__(kv::kThreads, 1)
       }
     }
   }
-  if (!kKv) {
-    // padding of the tiled scale layout: rows [M, 128-row boundary) and blocks
-    // [nb, 4 nbp4) of the real rows are 0 (the GEMM multiplies by 2^(byte-127))
-    const int64_t mpad = (p.rows + 127) / 128 * 128;
-    const int64_t tail = 4 * p.nbp4 - p.nb;  // 0..3 padding blocks per real row
-    const int64_t n_rows_pad = (mpad - p.rows) * p.nbp4;
-    const int64_t total = n_rows_pad + p.rows * tail;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-      if (i < n_rows_pad) {
-        const int64_t m = p.rows + i / p.nbp4;
-        const int64_t c = i % p.nbp4;
-        *reinterpret_cast<uint32_t*>(p.scales + scale_offset(m, 4 * c, p.nbp4)) = 0u;
-      } else {
-        const int64_t j = i - n_rows_pad;
-        p.scales[scale_offset(j / tail, p.nb + j % tail, p.nbp4)] = 0;
-      }
+  if (!kKv && p.done_flags != nullptr) {
+    // every thread of the CTA has written its outputs; thread 0 publishes them (the
+    // barrier orders the others' stores before its release)
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      st_release_gpu_u64(p.done_flags + blockIdx.x, p.epoch);
     }
   }
 }
