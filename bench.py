@@ -553,7 +553,8 @@ class LinearBench:
     def step(self):
         if self.use_linear:
             self.bat.bat_linear(self.X, self.Wq, self.A, self.B, self.gl, self.gh, Y=self.Y,
-                                out_dtype=self.torch.bfloat16, workspace=self.ws, stream=self.stream)
+                                out_dtype=self.torch.bfloat16, workspace=self.ws, stream=self.stream,
+                                fused=self.args.fused == 1)
         else:
             self.quantize(self.X, self.Xq)
             self.gemm_fn(self.Xq, self.Wq, Y=self.Y, out_dtype=self.torch.bfloat16, stream=self.stream)
@@ -688,7 +689,8 @@ class LinearBench:
                 ln["Xdev"].copy_(Xh, non_blocking=True)
                 if self.use_linear:
                     bat.bat_linear(ln["Xdev"], self.Wq, self.A, self.B, self.gl, self.gh, Y=ln["Y"],
-                                   out_dtype=torch.bfloat16, workspace=ln["ws"], stream=ls)
+                                   out_dtype=torch.bfloat16, workspace=ln["ws"], stream=ls,
+                                   fused=self.args.fused == 1)
                 else:
                     self.quantize(ln["Xdev"], ln["Xq"], ls)
                     self.gemm_fn(ln["Xq"], self.Wq, Y=ln["Y"], out_dtype=torch.bfloat16, stream=ls)
@@ -742,6 +744,10 @@ def main():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
                     help="measure only the headline workload")
+    ap.add_argument("--fused", type=int, default=0, choices=[0, 1],
+                    help="bat_linear's fused argument: 1 lets the GEMM start on each token tile "
+                         "as the prologue publishes it; 0 (default, the faster as measured) "
+                         "waits for the whole prologue")
     ap.add_argument("--shared", type=int, default=8, choices=[1, 2, 4, 8, 16, 32],
                     help="size s of the shared transform factor (A s x s, each B_b 32/s x 32/s)")
     ap.add_argument("--act", default="mxfp4", choices=["mxfp4", "mxfp8"],
@@ -839,6 +845,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "mxfp8 x mxfp4" if a8 else "mxfp4", "data": "synthetic",
             "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "out": "bf16",
+                       "fused": bool(args.fused) and not a8 and args.shared == 8,
                        "transform": f"GPK A {args.shared}x{args.shared} shared, "
                                     f"B_b {32 // args.shared}x{32 // args.shared} private",
                        "l2": "flushed between steps (256 MiB write + read outside the timed events)",

@@ -329,16 +329,25 @@ BAT_API bat_status_t bat_kv_dequantize(const void* cache_codes, const void* cach
 BAT_API bat_status_t bat_mxfp4_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
                             bat_out_dtype_t out_dtype, void* stream);
 
-/* Workspace bytes bat_linear needs for M rows of K inputs (the quantized X); 0 for
- * an invalid shape. */
+/* Workspace bytes bat_linear needs for M rows of K inputs (the quantized X and, for
+ * M <= 64 or M > 128, the completion flags the two kernels synchronise on); 0 for an
+ * invalid shape. */
 BAT_API size_t bat_linear_workspace_bytes(int64_t M, int64_t K);
 
 /*
  * The whole online linear layer Y = Q(XP) . Q(P^-1 W^T): bat_quantize_act into
- * `workspace`, then bat_mxfp4_gemm, on one stream.
+ * `workspace`, then bat_mxfp4_gemm, on one stream (BATQuant note, en.papernotes.org,
+ * Method > Key Designs 1 for the product, 2 and 3 for the transform and the clip).
  *   X  : bf16 [M][K]; Wq from bat_prepare_weight (Wq->k == K); A, B, g_lo, g_hi
  *        as in bat_quantize_act; Y: [M][Wq->rows] in `out_dtype`.
  *   workspace : device, >= bat_linear_workspace_bytes(M, K) bytes, 256-byte aligned.
+ *   fused : 0 or 1. With 1 and M > 128 the two kernels overlap at tile granularity:
+ *        the quantizer publishes each 128-row token tile's block pairs as it stores
+ *        them, and the GEMM starts on a token tile as soon as that tile is complete
+ *        instead of after the whole quantizer. Codes and Y are the same bytes as with 0
+ *        (the same kernels; only their synchronisation changes). For M <= 128, fused
+ *        changes nothing (at M <= 64 the GEMM always starts on the quantizer's
+ *        completion flags).
  * Errors: those of bat_quantize_act and bat_mxfp4_gemm, and BAT_ERR_WORKSPACE
  * (workspace NULL or smaller than needed) or BAT_ERR_ALIGN (workspace not
  * 256-byte aligned).
@@ -346,7 +355,7 @@ BAT_API size_t bat_linear_workspace_bytes(int64_t M, int64_t K);
 BAT_API bat_status_t bat_linear(const void* X, int64_t M, const bat_mxfp4_t* Wq, const float* A,
                         const float* B, const float* g_lo, const float* g_hi, void* Y,
                         bat_out_dtype_t out_dtype, void* workspace, size_t workspace_bytes,
-                        void* stream);
+                        int fused, void* stream);
 
 /*
  * Allocation-free variant of bat_linear. There is no counterpart on the pages:

@@ -76,8 +76,10 @@ def test_host_validation_returns_before_cuda(L):
     assert L.bat_mxfp4_gemm(ctypes.byref(good), ctypes.byref(w64), p, 7, None) == 1
     assert L.bat_mxfp4_gemm(ctypes.byref(good), ctypes.byref(w64), _fake_ptr(4), 0, None) == 3
     # linear: workspace too small or missing
-    assert L.bat_linear(p, 4, ctypes.byref(w64), p, p, None, None, p, 0, None, 0, None) == 7
-    assert L.bat_linear(p, 4, ctypes.byref(w64), p, p, None, None, p, 0, p, 16, None) == 7
+    assert L.bat_linear(p, 4, ctypes.byref(w64), p, p, None, None, p, 0, None, 0, 0, None) == 7
+    assert L.bat_linear(p, 4, ctypes.byref(w64), p, p, None, None, p, 0, p, 16, 0, None) == 7
+    # linear: the fused flag is 0 or 1
+    assert L.bat_linear(p, 4, ctypes.byref(w64), p, p, None, None, p, 0, p, 1 << 20, 2, None) == 1
     # weight prep: K too large / invalid N
     w_big = S(0x7F0000300000, 0x7F0000400000, 8, 262144 + 32)
     assert L.bat_prepare_weight(p, 8, 262144 + 32, p, p, None, None, ctypes.byref(w_big), None, None) == 2
@@ -163,7 +165,7 @@ def test_row_limit(L):
     assert L.bat_prepare_weight(p, big + 1, 64, p, p, None, None, ctypes.byref(over), None,
                                 None) == 2
     assert L.bat_linear(p, big + 1, ctypes.byref(w64), p, p, None, None, p, 0, p, 1 << 40,
-                        None) == 2
+                        0, None) == 2
     assert L.bat_linear_noalloc(p, big + 1, ctypes.byref(w64), p, p, None, None, p, 0, None) == 2
     # KV stores: tokens x heads, and cache slots x heads
     kv = lambda T, H, slots: L.bat_kv_quantize(p, T, H, 64, p, 8, p, None, None, p, 0, p, p,

@@ -375,8 +375,10 @@ def test_linear_workloads(bat, name):
     Y = bat.bat_linear(Xd, Wq, Ad, Bd, gl, gh, out_dtype=torch.float32)
     Xq = bat.bat_quantize_act(Xd, Ad, Bd, gl, gh)
     Y2 = bat.bat_mxfp4_gemm(Xq, Wq, out_dtype=torch.float32)
+    Y3 = bat.bat_linear(Xd, Wq, Ad, Bd, gl, gh, out_dtype=torch.float32, fused=True)
     torch.cuda.synchronize()
     assert torch.equal(Y, Y2)  # unfused linear == quantize then GEMM, bit for bit
+    assert torch.equal(Y, Y3)  # the tile-level overlap changes only the synchronisation
     # a row in every 128-row tile and a column in every 256-column tile, plus edges
     r = np.arange(w.M) if w.M <= 64 else _sample(w.M, 24, 1, tile=128)
     c = np.arange(w.N) if w.N <= 512 else _sample(w.N, 200, 2, tile=256)
@@ -390,6 +392,30 @@ def test_linear_workloads(bat, name):
         _, oc, os_ = oracle.quantize_act(inp.X, inp.A, inp.B, inp.g_lo, inp.g_hi)
         agree = np.mean(oc == x_codes)
         assert agree > 0.999, agree
+    assert bat.bat_device_error() == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 1000, 2048), (129, 264, 4128), (1000, 1288, 4128),
+                                   (256, 512, 256), (2048, 768, 12288), (777, 520, 96)])
+def test_linear_fused_equals_unfused(bat, M, N, K):
+    """fused=True (the GEMM starts on each token tile as the prologue publishes it) gives
+    the same codes and the same Y bytes as fused=False; one workspace reused across calls
+    and shapes (stale flags of earlier calls must not release a later one)."""
+    X = wl.random_bf16((M, K), seed=M + K, scale=2.0)
+    W = wl.random_bf16((N, K), seed=N + 3 * K, scale=0.02)
+    A, B, g_lo, g_hi = wl.random_factors(K // 32, seed=K + 5)
+    Xd, Ad, Bd, gl, gh = _dev_bf16(X), _dev_f32(A), _dev_f32(B), _dev_f32(g_lo), _dev_f32(g_hi)
+    Wq = bat.bat_prepare_weight(_dev_bf16(W), Ad, Bd)
+    ws = torch.empty(bat.bat_linear_workspace_bytes(M, K) + 4096, dtype=torch.uint8, device="cuda")
+    for dt in (torch.bfloat16, torch.float32):
+        ref = bat.bat_linear(Xd, Wq, Ad, Bd, gl, gh, out_dtype=dt, workspace=ws)
+        codes_ref = ws.clone()
+        for _ in range(3):
+            got = bat.bat_linear(Xd, Wq, Ad, Bd, gl, gh, out_dtype=dt, workspace=ws, fused=True)
+            torch.cuda.synchronize()
+            assert torch.equal(got, ref)
+        n_q = bat.bat_mxfp4_codes_bytes(M, K)
+        assert torch.equal(ws[:n_q], codes_ref[:n_q])  # the same codes
     assert bat.bat_device_error() == 0
 
 

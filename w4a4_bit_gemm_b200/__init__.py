@@ -78,7 +78,7 @@ def lib() -> ctypes.CDLL:
         "bat_selftest_bounded_wait": (S, [ctypes.c_uint64, P, P]),
         "bat_mxfp4_gemm": (S, [SP, SP, P, S, P]),
         "bat_linear_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
-        "bat_linear": (S, [P, I64, SP, P, P, P, P, P, S, P, ctypes.c_size_t, P]),
+        "bat_linear": (S, [P, I64, SP, P, P, P, P, P, S, P, ctypes.c_size_t, S, P]),
         "bat_linear_noalloc": (S, [P, I64, SP, P, P, P, P, P, S, P]),
         "bat_device_error": (S, []),
         "bat_last_cuda_error": (ctypes.c_char_p, []),
@@ -443,7 +443,7 @@ def bat_linear_workspace_bytes(M: int, K: int) -> int:
 
 def bat_linear(X, Wq: MXFP4, A, B, g_lo=None, g_hi=None, Y: Optional[torch.Tensor] = None,
                out_dtype: torch.dtype = torch.bfloat16, workspace: Optional[torch.Tensor] = None,
-               stream=None) -> torch.Tensor:
+               stream=None, fused: bool = False) -> torch.Tensor:
     M, K = _act_args(X, A, B, g_lo, g_hi)
     code = _out_code(out_dtype)
     dev = X.device
@@ -459,7 +459,8 @@ def bat_linear(X, Wq: MXFP4, A, B, g_lo=None, g_hi=None, Y: Optional[torch.Tenso
     _on_device(dev, stream)
     b = Wq.struct()
     _check(lib().bat_linear(_ptr(X), M, ctypes.byref(b), _ptr(A), _ptr(B), _ptr(g_lo), _ptr(g_hi),
-                            _ptr(Y), code, _ptr(workspace), workspace.numel(), _stream(stream)),
+                            _ptr(Y), code, _ptr(workspace), workspace.numel(), 1 if fused else 0,
+                            _stream(stream)),
            "bat_linear")
     return Y
 

@@ -263,9 +263,10 @@ bat_status_t check_act_args(const void* X, int64_t M, int64_t K, const float* A,
 // Activation batches of at most this many rows run on the CUDA-core row quantizer
 // (its latency is a few microseconds; the tensor-core prologue's set-up costs more).
 constexpr int64_t kRowsCudaCore = 64;
-// The linear layer at those sizes: room for the row quantizer's per-CTA completion flags
-// (64-bit; its grid is at most 16 warps per SM, two CTAs per SM) and their epochs, unique
-// per call and process (a salted counter), so flags left by earlier calls never match.
+// The linear layer's per-CTA completion flags (64-bit): the row quantizer's (at most 16
+// warps per SM, two CTAs per SM) or the prologue's (one CTA per SM at most), and their
+// epochs, unique per call and process (a salted counter), so flags left by earlier calls
+// never match.
 constexpr size_t kDoneFlagBytes = 4096;
 std::atomic<unsigned long long> g_calls{0};
 unsigned long long next_epoch() {
@@ -331,7 +332,8 @@ bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float
                              int ls = 3, bool fp8 = false, const int64_t* kv_slots = nullptr,
                              int64_t kv_heads = 0, int64_t kv_nslots = 0,
                              unsigned long long* done_flags = nullptr, unsigned long long epoch = 0,
-                             int* rows_grid_out = nullptr) {
+                             int* rows_grid_out = nullptr, unsigned long long* cta_flags = nullptr,
+                             int* strips_out = nullptr, int* cps_out = nullptr) {
   int dev = 0, sms = 0;
   bat_status_t st = current_device(&dev, &sms);
   if (st != BAT_OK) return st;
@@ -355,6 +357,9 @@ bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float
   p.nb = static_cast<int>(K / 32);
   p.ls = ls;
   p.slots = kv_slots;
+  // unit completion flags: activations of the linear layer only
+  p.cta_flags = (!per_row && kv_slots == nullptr && !fp8) ? cta_flags : nullptr;
+  p.epoch = epoch;
   p.kv_heads = kv_heads;
   p.kv_slots = kv_nslots;
   p.nbp2 = (p.nb + 1) / 2;
@@ -395,6 +400,8 @@ bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float
   }
   // One CTA per (strip, part): about one per SM.
   const int64_t grid = static_cast<int64_t>(p.strips) * p.cps;
+  if (strips_out) *strips_out = p.strips;
+  if (cps_out) *cps_out = p.cps;
   kern<<<static_cast<unsigned>(grid), bat::pro::kThreads, bat::pro::kSmemBytes, stream>>>(tx, p);
   return cuda_status(cudaGetLastError());
 }
@@ -404,10 +411,15 @@ bat_status_t launch_prologue(const void* X, int64_t rows, int64_t K, const float
 // linear layer: that kernel is the activation quantizer). q_flags / q_ctas / epoch: that
 // quantizer's completion flags (row quantizer), which the decode GEMM waits on instead of
 // the grid dependency; null otherwise.
+// cta_flags (CTA-pair kernel): the prologue's per-CTA completion flags (q_strips x q_cps
+// CTAs), waited for tile by tile instead of the grid dependency (the tile-level overlap
+// of the fused linear layer).
 bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
                          bat_out_dtype_t out_dtype, cudaStream_t stream, bool a8 = false,
                          bool w_static = false, const unsigned long long* q_flags = nullptr,
-                         int q_ctas = 0, unsigned long long epoch = 0) {
+                         int q_ctas = 0, unsigned long long epoch = 0,
+                         const unsigned long long* cta_flags = nullptr, int q_strips = 0,
+                         int q_cps = 0) {
   int dev = 0, sms = 0;
   bat_status_t st = current_device(&dev, &sms);
   if (st != BAT_OK) return st;
@@ -420,7 +432,7 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
     if (!make_code_map(&tb, Wq->codes, Wq->rows, Wq->k, bat::gemm::kBN)) return BAT_ERR_CUDA;
   }
   std::memset(&ty, 0, sizeof(ty));
-  bat::GemmParams p;
+  bat::GemmParams p{};
   p.sfa = static_cast<const uint8_t*>(Xq->scales);
   p.sfb = static_cast<const uint8_t*>(Wq->scales);
   p.y = Y;
@@ -537,6 +549,15 @@ bat_status_t launch_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
   p.splits = static_cast<int>(splits);
   if (!a8 && splits == 1 && m_tiles >= 2) {
     // CTA pairs on 256 x 256 tiles (bat_gemm2.cuh)
+    if (cta_flags != nullptr && q_strips > 0 && q_cps > 0) {
+      static_assert(bat::pro::kStrip == 4, "the pair kernel's flag walk assumes 4 pairs per strip");
+      p.cta_flags = cta_flags;
+      p.q_mtiles = (p.M + 127) / 128;
+      p.q_nbp2 = static_cast<int>((p.K / 32 + 1) / 2);
+      p.q_strips = q_strips;
+      p.q_cps = q_cps;
+      p.q_epoch = epoch;
+    }
     CUtensorMap pa, pb, py;
     if (!make_code_map(&pa, Xq->codes, Xq->rows, Xq->k, bat::gemm2::kRows)) return BAT_ERR_CUDA;
     if (!make_code_map(&pb, Wq->codes, Wq->rows, Wq->k, bat::gemm2::kBN / 2)) return BAT_ERR_CUDA;
@@ -947,14 +968,18 @@ size_t bat_linear_workspace_bytes(int64_t M, int64_t K) {
   if (M <= kRowsCudaCore)
     return static_cast<size_t>(round_up(static_cast<int64_t>(c), 256) +
                                round_up(static_cast<int64_t>(s), 256)) + kDoneFlagBytes;
+  // CTA-pair GEMM sizes: the prologue's per-CTA completion flags (fused)
+  if (M > 128)
+    return static_cast<size_t>(round_up(static_cast<int64_t>(c), 256) +
+                               round_up(static_cast<int64_t>(s), 256)) + kDoneFlagBytes;
   return static_cast<size_t>(round_up(static_cast<int64_t>(c), 256)) + s;
 }
 
 bat_status_t bat_linear(const void* X, int64_t M, const bat_mxfp4_t* Wq, const float* A,
                         const float* B, const float* g_lo, const float* g_hi, void* Y,
                         bat_out_dtype_t out_dtype, void* workspace, size_t workspace_bytes,
-                        void* stream) {
-  if (!Wq) return BAT_ERR_INVALID_ARG;
+                        int fused, void* stream) {
+  if (!Wq || (fused != 0 && fused != 1)) return BAT_ERR_INVALID_ARG;
   const int64_t K = Wq->k;
   if (M < 1 || K < 32) return BAT_ERR_INVALID_ARG;
   if (K % 32 != 0 || K > kMaxK || M > kMaxRows) return BAT_ERR_SHAPE;
@@ -976,17 +1001,25 @@ bat_status_t bat_linear(const void* X, int64_t M, const bat_mxfp4_t* Wq, const f
   unsigned long long* flags = nullptr;
   unsigned long long epoch = 0;
   int q_ctas = 0;
+  // fused (more than 128 rows): the prologue publishes each (token tile, block pair) as
+  // it is stored and the CTA-pair GEMM waits for its token tiles only
+  unsigned long long* cta_flags = nullptr;
+  int q_strips = 0, q_cps = 0;
+  uint8_t* after_scales = static_cast<uint8_t*>(xq.scales) +
+                          round_up(static_cast<int64_t>(bat_mxfp4_scales_bytes(M, K)), 256);
   if (M <= kRowsCudaCore) {
-    flags = reinterpret_cast<unsigned long long*>(
-        static_cast<uint8_t*>(xq.scales) +
-        round_up(static_cast<int64_t>(bat_mxfp4_scales_bytes(M, K)), 256));
+    flags = reinterpret_cast<unsigned long long*>(after_scales);
+    epoch = next_epoch();
+  } else if (fused && M > 128) {
+    cta_flags = reinterpret_cast<unsigned long long*>(after_scales);
     epoch = next_epoch();
   }
   st = launch_prologue(X, M, K, A, B, g_lo, g_hi, false, &xq, nullptr, s, 3, false, nullptr, 0, 0,
-                       flags, epoch, &q_ctas);
+                       flags, epoch, &q_ctas, cta_flags, &q_strips, &q_cps);
   if (st != BAT_OK) return st;
   // the kernel right before the GEMM is the quantizer, which does not write the weights
-  return launch_gemm(&xq, Wq, Y, out_dtype, s, false, true, flags, q_ctas, epoch);
+  return launch_gemm(&xq, Wq, Y, out_dtype, s, false, true, flags, q_ctas, epoch, cta_flags,
+                     q_strips, q_cps);
 }
 
 const char* bat_last_cuda_error(void) {

@@ -93,6 +93,13 @@ struct GemmParams {
   int vec_ok;          // rows of Y are 16-byte aligned for vector stores
   int tma_store;       // bf16 output written through the staged TMA store
   int splits;          // K splits = cluster size (1: persistent, whole K per tile)
+  // CTA-pair kernel, tile-level overlap with the prologue: null (wait for the grid
+  // dependency), or the prologue's per-CTA completion flags (q_strips x q_cps CTAs over
+  // q_mtiles token tiles and q_nbp2 block pairs), complete when they hold q_epoch
+  const unsigned long long* cta_flags;
+  int64_t q_mtiles;
+  int q_nbp2, q_strips, q_cps;
+  unsigned long long q_epoch;
 };
 
 __device__ __forceinline__ uint4 lds_v4_u32(uint32_t addr) {

@@ -27,6 +27,14 @@
 // No copy is multicast. Every wait is bounded and reports through the error word; both
 // CTAs meet at a cluster barrier before TMEM is released.
 //
+// Tile-level overlap with the prologue (p.cta_flags set): instead of waiting for the
+// prologue's grid to retire, the code producer warp's lanes 1-31 walk this CTA's tiles
+// ahead of the producers and, for each, poll the completion flags of the prologue CTAs
+// that wrote the 128-row token tile this CTA loads (in every strip, the one or two CTAs
+// whose unit range covers the tile), then publish "tiles ready" in shared memory; the
+// code and scale producers wait for that count before a tile's first X copy.
+// The weights and their scales are not written by the prologue, and neither is Y.
+//
 // Warp roles per CTA: 0-3 epilogue, 4-7 scale writers, 8 code producer, 9 MMA issuer of
 // even k-steps (even CTA) / TMEM owner (both), 10 scale producer, 11 MMA issuer of odd
 // k-steps (even CTA).
@@ -191,7 +199,8 @@ __global__ void __launch_bounds__(gemm2::kThreads, 1)
   const uint32_t tmem_full = bars + 8u * (4 * kStages);                   // both
   const uint32_t tmem_empty = tmem_full + 8u;                             // used in CTA 0
   const uint32_t turn_bar = tmem_empty + 8u;                             // used in CTA 0
-  const uint32_t tmem_slot = turn_bar + 8u;
+  const uint32_t tiles_ready = turn_bar + 8u;  // tile-level overlap: tiles whose X is written
+  const uint32_t tmem_slot = tiles_ready + 8u;
   volatile uint32_t* tmem_slot_ptr =
       reinterpret_cast<volatile uint32_t*>(base_ptr + (tmem_slot - base));
 
@@ -209,6 +218,7 @@ __global__ void __launch_bounds__(gemm2::kThreads, 1)
     }
     mbar_init(tmem_full, 2);         // the multicast commits of the two issuers
     mbar_init(turn_bar, 1);          // the issuer of the k-step just issued
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(tiles_ready), "r"(0u) : "memory");
     mbar_init(tmem_empty, 8);        // four epilogue warps in each CTA
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&tmap_a);
@@ -223,8 +233,9 @@ __global__ void __launch_bounds__(gemm2::kThreads, 1)
   cluster_sync_all();  // both CTAs' barriers exist before either signals the other's
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot_ptr;
-  // Everything above is local setup; the operands (and Y) belong to the kernels before.
-  grid_dependency_wait();
+  // Everything above is local setup; the operands (and Y) belong to the kernels before
+  // (with p.cta_flags, X and its scales are waited for tile by tile below instead).
+  if (p.cta_flags == nullptr) grid_dependency_wait();
 
   const int64_t m_tiles = (p.M + 2 * kRows - 1) / (2 * kRows);  // 256-row tiles
   const int64_t n_tiles = (p.N + kBN - 1) / kBN;
@@ -236,6 +247,24 @@ __global__ void __launch_bounds__(gemm2::kThreads, 1)
   const int64_t sf_groups_b = (p.N + 127) / 128;
   bool ok = true;
 
+  // (tile-level overlap) the producers' wait for the i-th tile of this CTA's walk
+  auto wait_tile_ready = [&](uint32_t i) -> bool {
+    if (p.cta_flags == nullptr) return true;
+    if (ld_acquire_cta_u32(tiles_ready) <= i) {
+      const uint64_t t0 = globaltimer_ns();
+      while (ld_acquire_cta_u32(tiles_ready) <= i) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          atomicOr(&g_dev_error, kErrWaitFull);
+          return false;
+        }
+        __nanosleep(64);
+      }
+    }
+    // (the prologue's threads made their writes visible to the async proxy, which the
+    // copies read through, before publishing them)
+    return true;
+  };
+
   if (warp >= 8) setmaxnreg_dec<kRegsOther>();  // warpgroup 2
   if (warp == 8) {
     // ------------------------------------------------------------ code producer (both)
@@ -244,11 +273,13 @@ __global__ void __launch_bounds__(gemm2::kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t inflight = 0;  // bit s: stage s was loaded; bit 16+s: parity of that load
-      for (int64_t tile = pair_id; tile < tiles && ok; tile += npairs) {
+      uint32_t ti = 0;  // tiles of this CTA's walk so far
+      for (int64_t tile = pair_id; tile < tiles && ok; tile += npairs, ++ti) {
         const int64_t mt = tile % m_tiles;
         const int64_t nt = tile / m_tiles;
         const int32_t arow = static_cast<int32_t>(mt * 2 * kRows + kRows * rank);
         const int32_t brow = static_cast<int32_t>(nt * kBN + (kBN / 2) * rank);
+        if (!wait_tile_ready(ti)) { ok = false; break; }
         for (int ks = 0; ks < k_stages; ++ks) {
           if (!mbar_wait_cluster(empty_bar(stage), phase ^ 1u, kErrWaitEmpty)) { ok = false; break; }
           // both CTAs' copies land on CTA 0's barrier, which expects all four (rows past
@@ -266,6 +297,52 @@ __global__ void __launch_bounds__(gemm2::kThreads, 1)
       if (even)
         for (int s = 0; s < kStages; ++s)
           if ((inflight >> s) & 1u) mbar_wait_cluster(full_bar(s), (inflight >> (16 + s)) & 1u, kErrWaitFull);
+    } else if (p.cta_flags != nullptr) {
+      // lanes 1-31: the flags of each tile's token tile, ahead of the producers. Relaxed
+      // polls, then an acquire fence once all are seen; lane 1 then counts the tile ready
+      // (release, CTA scope) for the producers.
+      const unsigned mask = 0xfffffffeu;
+      uint32_t ti = 0;
+      for (int64_t tile = pair_id; tile < tiles; tile += npairs, ++ti) {
+        const int64_t t = (tile % m_tiles) * 2 + rank;  // this CTA's 128-row token tile
+        if (t < p.q_mtiles) {
+          const uint64_t t0 = globaltimer_ns();
+          bool stalled = false;
+          while (true) {
+            bool mine = true;
+            for (int st = lane - 1; st < p.q_strips; st += 31) {
+              // strip st: units v = tile * npair + pair, split over q_cps CTAs as
+              // [sunits c / cps, sunits (c + 1) / cps); those holding units of token tile t
+              const int64_t npair = min(4, p.q_nbp2 - 4 * st);
+              const int64_t sunits = p.q_mtiles * npair;
+              const int64_t u0 = t * npair, u1 = (t + 1) * npair - 1;
+              int64_t c = u0 * p.q_cps / sunits;
+              while (c > 0 && sunits * c / p.q_cps > u0) --c;
+              while (c + 1 < p.q_cps && sunits * (c + 1) / p.q_cps <= u0) ++c;
+              for (; c < p.q_cps && sunits * c / p.q_cps <= u1; ++c) {
+                unsigned long long v;
+                asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];"
+                             : "=l"(v)
+                             : "l"(p.cta_flags + st * p.q_cps + c)
+                             : "memory");
+                mine = mine && v == p.q_epoch;
+              }
+            }
+            if (__all_sync(mask, mine)) break;
+            // (a warp-wide decision: every lane leaves the loop together)
+            if (__any_sync(mask, globaltimer_ns() - t0 > kWaitLimitNs)) { stalled = true; break; }
+            __nanosleep(128);
+          }
+          if (stalled) {
+            if (lane == 1) atomicOr(&g_dev_error, kErrWaitFull);
+            break;
+          }
+          asm volatile("fence.acq_rel.gpu;" ::: "memory");
+        }
+        __syncwarp(mask);
+        if (lane == 1) asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(tiles_ready), "r"(ti + 1)
+                                    : "memory");
+      }
     }
   } else if (warp == 10) {
     // ------------------------------------------------------------ scale producer (both)
@@ -273,10 +350,12 @@ __global__ void __launch_bounds__(gemm2::kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t inflight = 0;
-      for (int64_t tile = pair_id; tile < tiles && ok; tile += npairs) {
+      uint32_t ti = 0;
+      for (int64_t tile = pair_id; tile < tiles && ok; tile += npairs, ++ti) {
         const int64_t mt = tile % m_tiles;
         const int64_t nt = tile / m_tiles;
         const int64_t ga = mt * 2 + rank;                        // this CTA's X row group
+        if (!wait_tile_ready(ti)) { ok = false; break; }
         const bool has_a = ga < sf_groups_a;                     // rows past M: no scales
         const int ngb = (nt * 2 + 1 < sf_groups_b) ? 2 : 1;      // W row groups of the tile
         for (int ks = 0; ks < k_stages; ++ks) {

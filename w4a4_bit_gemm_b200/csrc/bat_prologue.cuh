@@ -98,7 +98,13 @@ struct PrologueParams {
   const int64_t* slots;
   int64_t kv_heads;
   int64_t kv_slots;
+  // optional completion flags (linear mode): CTA i stores `epoch` into cta_flags[i]
+  // (release, GPU scope) once all its codes and scales are written; null: none. (CTA i
+  // covers strip i / cps, units [sunits (i % cps) / cps, sunits (i % cps + 1) / cps).)
+  unsigned long long* cta_flags;
+  unsigned long long epoch;
 };
+
 
 
 
@@ -289,6 +295,7 @@ __global__ void __launch_bounds__(pro::kThreads, 1)
       reinterpret_cast<volatile uint32_t*>(base_ptr + (tmem_slot - base));
   // clip ratios of the strip's blocks: [2 * kStrip] lo, then [2 * kStrip] hi
   float* ratios = reinterpret_cast<float*>(base_ptr + (bars - base) + 256);
+
   // A and the strip's B_b, staged for the P build (s > 1): A [s][s], then [2 * kStrip][t][t]
   const bool staged = p.ls > 0;
   const int fa = 1 << (2 * p.ls), fb = 1 << (10 - 2 * p.ls);  // s*s and t*t
@@ -564,10 +571,21 @@ __global__ void __launch_bounds__(pro::kThreads, 1)
     }
   }
 
+  // with completion flags, the codes and scales are read by a running GEMM's tensor copies
+  // (async proxy): every thread orders its stores before them here
+  if (p.cta_flags != nullptr) asm volatile("fence.proxy.async.global;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+  // every thread's stores are done (barrier above): publish them for a GEMM that starts on
+  // this CTA's token tiles. (Publishing every unit as it was stored instead, with one
+  // GPU-scope release per unit from a warp of its own, made the prefill_o step 25 us
+  // slower.)
+  if (threadIdx.x == 0 && p.cta_flags != nullptr) {
+    __threadfence();
+    st_release_gpu_u64(p.cta_flags + blockIdx.x, p.epoch);
+  }
 }
 
 __global__ void bat_clip_ratio_kernel(const float* g, int64_t n, float* r) {
