@@ -45,8 +45,6 @@
 // not.
 #pragma once
 
-#include <cooperative_groups.h>
-
 #include "bat_common.cuh"
 #include "bat_gemm.cuh"
 
