@@ -36,9 +36,9 @@
 // Split-K sum: rows [o 128 / S, (o+1) 128 / S) of the tile belong to rank o. Every other
 // rank sends its fp32 partial of such a row (the row's token values, contiguous) into
 // rank o's shared memory with st.async, which counts the bytes on rank o's receive
-// barrier; the thread of rank o that holds the row's own partial in registers waits for
-// that barrier, adds the S partials in rank order (a fixed order, so the result does not
-// depend on timing) and stages the row for the write-out. (Plain remote stores followed
+// barrier; the thread of rank o that holds the row's own partial puts it beside them,
+// waits for that barrier, adds the S partials in rank order (a fixed order, so the result
+// does not depend on timing) and stages the row for the write-out. (Plain remote stores followed
 // by a cluster barrier were timed at about 1000 cycles per later local load of the
 // received data.) Every wait is bounded and reports
 // through the error word; every CTA takes part in both cluster barrier phases, error or
@@ -358,43 +358,46 @@ __global__ void __launch_bounds__(gemmd::kThreads, 1)
 
   if (warp < 4) {
     // (4) this CTA's rows [r0, r0 + nr) of the tile (all 128 when S = 1; the owned share
-    //     otherwise, summed over the S partials in rank order, its own from registers)
-    //     go to shared memory as [token][row] in the output type (over the drained W
-    //     ring), then to Y in 16-byte stores: one per 8 bf16 (4 fp32) outputs, not one
-    //     per value, which at these sizes is what the write-out costs
+    //     otherwise) are summed over the S partials in rank order and go to shared memory
+    //     as [token][row] in the output type (over the drained W ring), then to Y in
+    //     16-byte stores: one per 8 bf16 (4 fp32) outputs, not one per value. The thread
+    //     of an owned row first puts its own partial next to the peers' (same swizzled
+    //     layout), so that the sum is a rolled loop over shared memory: this code runs
+    //     once per launch, and with the benchmark's flushed L2 every new stretch of
+    //     straight-line code is fetched from memory.
     const int nr = kBM / S;
     const int r0 = rank * nr;
     const int esz = p.out_f32 ? 4 : 2;
     const uint32_t stage = base;
+    const bool own = rl >= r0 && rl < r0 + nr;
+    const uint32_t src = red + static_cast<uint32_t>((rl - r0) * kMaxNx * 4);
+    if (own) {
+      const uint32_t dst = src + static_cast<uint32_t>(rank * nr * kMaxNx * 4);
+#pragma unroll
+      for (int c = 0; c < kMaxNx / 4; ++c)
+        if (4 * c < nx)
+          st_shared_v4(dst + 16 * (c ^ (rl & 7)), r[(4 * c) >> 5][(4 * c) & 31],
+                       r[(4 * c + 1) >> 5][(4 * c + 1) & 31], r[(4 * c + 2) >> 5][(4 * c + 2) & 31],
+                       r[(4 * c + 3) >> 5][(4 * c + 3) & 31]);
+    }
     // the peers' partials of the owned rows have landed (every CTA waits for all it is
     // sent, so none exits while a peer still writes into it)
     const bool recv = S == 1 || mbar_wait(red_bar, 0, kErrWaitFull);
-    if (got && recv && rl >= r0 && rl < r0 + nr) {
-      const uint32_t src = red + static_cast<uint32_t>((rl - r0) * kMaxNx * 4);
-#pragma unroll
-      for (int c = 0; c < kMaxNx / 4; ++c) {
-        if (4 * c >= p.M) break;
-        float a[4] = {__uint_as_float(r[(4 * c) >> 5][(4 * c) & 31]),
-                      __uint_as_float(r[(4 * c + 1) >> 5][(4 * c + 1) & 31]),
-                      __uint_as_float(r[(4 * c + 2) >> 5][(4 * c + 2) & 31]),
-                      __uint_as_float(r[(4 * c + 3) >> 5][(4 * c + 3) & 31])};
-        if (S > 1) {
-          float t[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-          for (int q = 0; q < S; ++q) {
-            float v[4] = {a[0], a[1], a[2], a[3]};
-            if (q != rank) {
-              const uint4 w = lds_v4_u32(src + static_cast<uint32_t>((q * nr * kMaxNx + 4 * (c ^ (rl & 7))) * 4));
-              v[0] = __uint_as_float(w.x);
-              v[1] = __uint_as_float(w.y);
-              v[2] = __uint_as_float(w.z);
-              v[3] = __uint_as_float(w.w);
-            }
-            t[0] += v[0];
-            t[1] += v[1];
-            t[2] += v[2];
-            t[3] += v[3];
-          }
-          a[0] = t[0]; a[1] = t[1]; a[2] = t[2]; a[3] = t[3];
+    if (got && recv && own) {
+      const int nc = static_cast<int>((p.M + 3) / 4);
+#pragma unroll 1
+      for (int c = 0; c < nc; ++c) {
+        const uint32_t cs = static_cast<uint32_t>(4 * (c ^ (rl & 7)) * 4);
+        uint4 w = lds_v4_u32(src + cs);
+        float a[4] = {__uint_as_float(w.x), __uint_as_float(w.y), __uint_as_float(w.z),
+                      __uint_as_float(w.w)};
+#pragma unroll 1
+        for (int q = 1; q < S; ++q) {
+          w = lds_v4_u32(src + static_cast<uint32_t>(q * nr * kMaxNx * 4) + cs);
+          a[0] += __uint_as_float(w.x);
+          a[1] += __uint_as_float(w.y);
+          a[2] += __uint_as_float(w.z);
+          a[3] += __uint_as_float(w.w);
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
