@@ -41,6 +41,12 @@ def test_sizes_match_documented_layout(L):
     assert bat.bat_mxfp4_codes_bytes(4, 48) == 0
     assert bat.bat_mxfp4_scales_bytes(0, 64) == 0
     assert bat.bat_linear_workspace_bytes(100, 64) == 3328 + formats.scale_bytes(100, 2)
+    # decode sizes (<= 64 rows) and CTA-pair sizes (> 128 rows): codes and scales each
+    # rounded to 256 bytes, then 4 KB of per-CTA completion flags for the two kernels
+    up = lambda v: (v + 255) // 256 * 256
+    for rows, k in [(16, 4096), (1, 32), (64, 12288), (300, 2048), (16384, 4096), (129, 4128)]:
+        want = up(rows * k // 2) + up(formats.scale_bytes(rows, k // 32)) + 4096
+        assert bat.bat_linear_workspace_bytes(rows, k) == want, (rows, k)
 
 
 def test_status_strings(L):
