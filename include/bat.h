@@ -321,10 +321,15 @@ BAT_API bat_status_t bat_kv_dequantize(const void* cache_codes, const void* cach
  *
  *   Xq : M x K MXFP4 activations; Wq : N x K MXFP4 weights (Xq->k == Wq->k).
  *   Y  : device [M][N] row-major, bf16 or fp32 per `out_dtype`, 16-byte aligned.
+ * Kernels: M > 128 runs on CTA pairs (256 x 256 tiles); M <= 64 (and K <= 16384) on the
+ * decode kernel, Y^T = Wq . Xq^T with K split over a cluster of up to 8 CTAs; otherwise
+ * on one SM per tile (split K over a cluster when one row of tiles leaves SMs idle).
+ * Every summation order is fixed: the result does not depend on timing.
  * Errors: BAT_ERR_INVALID_ARG (a NULL pointer, an unknown out_dtype, rows < 1 or
  * k < 32), BAT_ERR_SHAPE (Xq->k != Wq->k, k % 32, k or rows over their limits),
- * BAT_ERR_ALIGN (codes, scales or Y not 16-byte aligned), BAT_ERR_UNSUPPORTED,
- * BAT_ERR_CUDA; nothing is launched on an argument error.
+ * BAT_ERR_ALIGN (codes, scales or Y not 16-byte aligned), BAT_ERR_UNSUPPORTED (also:
+ * the decode kernel's clusters cannot be resident on this device), BAT_ERR_CUDA;
+ * nothing is launched on an argument error.
  */
 BAT_API bat_status_t bat_mxfp4_gemm(const bat_mxfp4_t* Xq, const bat_mxfp4_t* Wq, void* Y,
                             bat_out_dtype_t out_dtype, void* stream);
