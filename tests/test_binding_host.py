@@ -88,6 +88,31 @@ def test_valid_calls_reach_the_library(rec):
         "bat_clip_ratios", "bat_kv_quantize", "bat_kv_dequantize"]
 
 
+def test_linear_fused_flag_marshalled(monkeypatch):
+    """bat_linear passes fused as the int argument before the stream (0 by default)."""
+    seen = []
+
+    class _Lib(_RecordingLib):
+        def __getattr__(self, name):
+            if name == "bat_linear":
+                def rec_linear(*args):
+                    seen.append(args)
+                    return 0
+                return rec_linear
+            return super().__getattr__(name)
+
+    monkeypatch.setattr(bat, "_lib", _Lib(bat.lib()))
+    monkeypatch.setattr(bat, "_DEVICE_TYPE", "cpu")
+    monkeypatch.setattr(bat, "_stream", lambda s: None)
+    M, N, K = 8, 16, 128
+    A, B = _factors(K)
+    Wq = bat.MXFP4.empty(N, K, device="cpu")
+    bat.bat_linear(_bf16(M, K), Wq, A, B)
+    bat.bat_linear(_bf16(M, K), Wq, A, B, fused=True)
+    assert len(seen) == 2
+    assert len(seen[0]) == 13 and seen[0][11] == 0 and seen[1][11] == 1
+
+
 def test_undersized_buffers_are_refused(rec):
     M, N, K = 8, 16, 64
     A, B = _factors(K)
