@@ -26,10 +26,10 @@
 // finishes. Xq, its scales and Y are only touched after griddepcontrol.wait, or, inside
 // a linear layer, after the row quantizer's completion flags (q_flags): each of its q_ctas
 // CTAs stores this call's epoch there with release semantics once its outputs are
-// written, and the four epilogue warps wait (acquire, bounded) for all of them. The
-// flags resolve a few microseconds earlier than the grid dependency, which waits for
-// the whole quantizer grid to retire. That kernel never writes the weights, and the
-// layer says so (w_static): the weight copies and the weight scales then start at once.
+// written, and the four epilogue warps wait (acquire, bounded) for all of them; the grid
+// dependency would wait for the whole quantizer grid to retire. That kernel never writes
+// the weights, and the layer says so (w_static): the weight copies and the weight scales
+// then start at once.
 // Otherwise the producer only prefetches the W boxes into L2 (the point of coherence, so
 // a later write would still be seen) before waiting.
 //
@@ -38,11 +38,9 @@
 // rank o's shared memory with st.async, which counts the bytes on rank o's receive
 // barrier; the thread of rank o that holds the row's own partial puts it beside them,
 // waits for that barrier, adds the S partials in rank order (a fixed order, so the result
-// does not depend on timing) and stages the row for the write-out. (Plain remote stores followed
-// by a cluster barrier were timed at about 1000 cycles per later local load of the
-// received data.) Every wait is bounded and reports
-// through the error word; every CTA takes part in both cluster barrier phases, error or
-// not.
+// does not depend on timing) and stages the row for the write-out; no cluster barrier
+// follows the sends. Every wait is bounded and reports through the error word; every CTA
+// takes part in the one cluster barrier phase (all CTAs started), error or not.
 #pragma once
 
 #include "bat_common.cuh"
